@@ -1,0 +1,177 @@
+"""ctypes wrapper over ``liboracle_nf4.so`` (test infrastructure only).
+
+Each function takes and returns numpy arrays and forwards to the C function of
+the same name in ``nf4_oracle.c``; the arithmetic lives there.
+"""
+import ctypes
+
+import numpy as np
+
+from .build_oracle import build
+
+__all__ = [
+    "norm_ppf", "codebook", "quantize", "dq_sum", "dq_mean", "double_quant", "absmax_hat",
+    "dequantize", "dequantize_range", "f32_to_bf16", "bf16_to_f32", "linear_bf16", "unpack",
+    "use_library",
+]
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = _bind(ctypes.CDLL(build()))
+    return _lib
+
+
+def _bind(L):
+    p = ctypes.c_void_p
+    i64 = ctypes.c_int64
+    L.orc_norm_ppf.argtypes = [ctypes.c_double]
+    L.orc_norm_ppf.restype = ctypes.c_double
+    L.orc_codebook.argtypes = [p]
+    L.orc_codebook.restype = None
+    L.orc_quantize_f32.argtypes = [p, i64, p, p]
+    L.orc_quantize_f32.restype = ctypes.c_int
+    L.orc_quantize_bf16.argtypes = [p, i64, p, p]
+    L.orc_quantize_bf16.restype = ctypes.c_int
+    L.orc_dq_sum.argtypes = [p, i64]
+    L.orc_dq_sum.restype = ctypes.c_double
+    L.orc_dq_mean.argtypes = [p, i64]
+    L.orc_dq_mean.restype = ctypes.c_float
+    L.orc_double_quant.argtypes = [p, i64, p, p, p]
+    L.orc_double_quant.restype = ctypes.c_int
+    L.orc_absmax_hat.argtypes = [p, p, ctypes.c_float, i64]
+    L.orc_absmax_hat.restype = ctypes.c_float
+    L.orc_dequantize_range.argtypes = [p, p, p, ctypes.c_float, i64, i64, p]
+    L.orc_dequantize_range.restype = ctypes.c_int
+    L.orc_f32_to_bf16.argtypes = [p, i64, p]
+    L.orc_f32_to_bf16.restype = None
+    L.orc_linear_bf16.argtypes = [p, i64, p, i64, i64, p]
+    L.orc_linear_bf16.restype = None
+    return L
+
+
+def use_library(path):
+    """Point the wrapper at another build of the oracle (used by the mutation
+    test, which builds deliberately broken copies); ``None`` restores the
+    default build."""
+    global _lib
+    _lib = None
+    if path is not None:
+        _lib = _bind(ctypes.CDLL(path))
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def norm_ppf(p: float) -> float:
+    return lib().orc_norm_ppf(float(p))
+
+
+def codebook() -> np.ndarray:
+    c = np.zeros(16, dtype=np.float32)
+    lib().orc_codebook(_ptr(c))
+    return c
+
+
+def quantize(w: np.ndarray):
+    """w: float32 array, or uint16 array of bf16 bit patterns; any shape with
+    size % 64 == 0.  Returns (wq uint8 [size/2], absmax float32 [size/64])."""
+    w = np.ascontiguousarray(w)
+    n = w.size
+    wq = np.zeros(n // 2, dtype=np.uint8)
+    absmax = np.zeros(n // 64, dtype=np.float32)
+    if w.dtype == np.float32:
+        rc = lib().orc_quantize_f32(_ptr(w), n, _ptr(wq), _ptr(absmax))
+    elif w.dtype == np.uint16:
+        rc = lib().orc_quantize_bf16(_ptr(w), n, _ptr(wq), _ptr(absmax))
+    else:
+        raise TypeError("oracle quantize takes float32 or bf16 bit patterns (uint16)")
+    if rc != 0:
+        raise ValueError("orc_quantize failed with %d" % rc)
+    return wq, absmax
+
+
+def dq_sum(absmax: np.ndarray) -> float:
+    a = np.ascontiguousarray(absmax, dtype=np.float32)
+    return lib().orc_dq_sum(_ptr(a), a.size)
+
+
+def dq_mean(absmax: np.ndarray) -> np.float32:
+    a = np.ascontiguousarray(absmax, dtype=np.float32)
+    return np.float32(lib().orc_dq_mean(_ptr(a), a.size))
+
+
+def double_quant(absmax: np.ndarray):
+    """Returns (absmax_q int8 [nb], absmax_scale float32 [ceil(nb/256)], mu float32)."""
+    a = np.ascontiguousarray(absmax, dtype=np.float32)
+    nb = a.size
+    q = np.zeros(nb, dtype=np.int8)
+    s = np.zeros((nb + 255) // 256, dtype=np.float32)
+    mu = np.zeros(1, dtype=np.float32)
+    rc = lib().orc_double_quant(_ptr(a), nb, _ptr(q), _ptr(s), _ptr(mu))
+    if rc != 0:
+        raise ValueError("orc_double_quant failed with %d" % rc)
+    return q, s, mu[0]
+
+
+def absmax_hat(absmax_q: np.ndarray, absmax_scale: np.ndarray, mu) -> np.ndarray:
+    q = np.ascontiguousarray(absmax_q, dtype=np.int8)
+    s = np.ascontiguousarray(absmax_scale, dtype=np.float32)
+    L = lib()
+    return np.array([L.orc_absmax_hat(_ptr(q), _ptr(s), float(mu), b) for b in range(q.size)],
+                    dtype=np.float32)
+
+
+def dequantize_range(wq, absmax_q, absmax_scale, mu, begin: int, count: int) -> np.ndarray:
+    wq = np.ascontiguousarray(wq, dtype=np.uint8)
+    q = np.ascontiguousarray(absmax_q, dtype=np.int8)
+    s = np.ascontiguousarray(absmax_scale, dtype=np.float32)
+    out = np.zeros(count, dtype=np.float32)
+    rc = lib().orc_dequantize_range(_ptr(wq), _ptr(q), _ptr(s), float(mu), int(begin), int(count),
+                                    _ptr(out))
+    if rc != 0:
+        raise ValueError("orc_dequantize_range failed with %d" % rc)
+    return out
+
+
+def dequantize(wq, absmax_q, absmax_scale, mu) -> np.ndarray:
+    return dequantize_range(wq, absmax_q, absmax_scale, mu, 0, 2 * np.asarray(wq).size)
+
+
+def f32_to_bf16(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.zeros(x.shape, dtype=np.uint16)
+    lib().orc_f32_to_bf16(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def bf16_to_f32(h: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns (no rounding involved)."""
+    h = np.ascontiguousarray(h, dtype=np.uint16)
+    return (h.astype(np.uint32) << 16).view(np.float32)
+
+
+def linear_bf16(x_bf16: np.ndarray, w_bf16: np.ndarray) -> np.ndarray:
+    """x_bf16 [m,k], w_bf16 [n,k] as uint16 bit patterns -> y float64 [m,n]."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    w = np.ascontiguousarray(w_bf16, dtype=np.uint16)
+    m, k = x.shape
+    n, k2 = w.shape
+    assert k == k2
+    y = np.zeros((m, n), dtype=np.float64)
+    lib().orc_linear_bf16(_ptr(x), m, _ptr(w), n, k, _ptr(y))
+    return y
+
+
+def unpack(wq: np.ndarray) -> np.ndarray:
+    """Packed bytes -> one index per element (high nibble first).  Pure layout."""
+    wq = np.asarray(wq, dtype=np.uint8)
+    out = np.empty(wq.size * 2, dtype=np.uint8)
+    out[0::2] = wq >> 4
+    out[1::2] = wq & 15
+    return out

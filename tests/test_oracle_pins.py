@@ -1,0 +1,363 @@
+"""Pins for the CPU oracle: each test ties an oracle function to something other
+than the oracle itself -- scipy's normal quantile function, the equal-mass
+property of the levels, exact rational argmin, the pages' printed figures,
+closed forms, hand-derived sums and mathematical error bounds.
+
+No GPU needed (not marked ``gpu``)."""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+
+f32 = np.float32
+
+
+def _levels():
+    return O.codebook()
+
+
+# ---------------------------------------------------------------------------
+# Levels: 16 normal quantiles, equal probability mass, normalised to [-1, 1],
+# with an exact zero (xyzblog page, section 2.2, principle ①; yololab page,
+# section on NF4 not being a generic FP4).
+# ---------------------------------------------------------------------------
+
+def test_codebook_invariants():
+    c = _levels()
+    assert c.dtype == np.float32 and c.shape == (16,)
+    assert np.all(np.diff(c) > 0), "levels must be strictly increasing"
+    assert c[0] == f32(-1.0) and c[15] == f32(1.0)
+    assert c[7] == f32(0.0) and np.signbit(c[7]) == False  # noqa: E712
+    assert int(np.sum(c < 0)) == 7 and int(np.sum(c > 0)) == 8
+    assert int(np.sum(c == 0)) == 1
+
+
+def test_norm_ppf_against_scipy():
+    from scipy.stats import norm
+    ps = np.concatenate([np.linspace(1e-6, 1 - 1e-6, 401), [1e-12, 1e-9, 0.5, 0.9677083333333333,
+                                                           1 - 1e-9]])
+    for p in ps:
+        x = O.norm_ppf(p)
+        ref = norm.ppf(p)
+        assert abs(x - ref) <= 4e-15 * max(1.0, abs(ref)), (p, x, ref)
+
+
+def test_levels_carry_equal_probability_mass():
+    """Undo the normalisation (multiply by Phi^-1 of the outermost probability)
+    and map back through the normal CDF: the positive levels must sit at
+    probabilities evenly spaced from delta towards 1/2 in 8 steps, the negative
+    ones in 7 steps (the equal-area construction)."""
+    from scipy.stats import norm
+    delta = 0.5 * ((1 - 1 / 30) + (1 - 1 / 32))
+    top = norm.ppf(delta)
+    c = _levels().astype(np.float64)
+    pos = np.sort(c[c > 0])[::-1]
+    neg = np.sort(-c[c < 0])[::-1]
+    p_pos = norm.cdf(pos * top)
+    p_neg = norm.cdf(neg * top)
+    np.testing.assert_allclose(p_pos, delta - np.arange(8) * (delta - 0.5) / 8, atol=1e-7)
+    np.testing.assert_allclose(p_neg, delta - np.arange(7) * (delta - 0.5) / 7, atol=1e-7)
+    # equal spacing in probability = equal probability mass between neighbours
+    assert np.allclose(np.diff(p_pos), -(delta - 0.5) / 8, atol=2e-7)
+
+
+# ---------------------------------------------------------------------------
+# Quantization: absmax per 64, x = w / absmax in fp32, nearest level (xyzblog
+# page, section 2.2 worked example; Figure 2-2).
+# ---------------------------------------------------------------------------
+
+def _exact_argmin(x: np.float32, c: np.ndarray) -> int:
+    """Index of the nearest level in exact rational arithmetic, ties to the
+    lower index."""
+    fx = Fraction(float(x))
+    best, best_d = 0, None
+    for i, ci in enumerate(c):
+        d = abs(fx - Fraction(float(ci)))
+        if best_d is None or d < best_d:
+            best, best_d = i, d
+    return best
+
+
+def test_quantize_is_exact_argmin_on_random_blocks():
+    rng = np.random.default_rng(11)
+    c = _levels()
+    w = (rng.standard_normal(64 * 12) * 0.02).astype(np.float32)
+    w[64 * 3: 64 * 4] *= 1e-30          # a block of tiny values
+    w[64 * 5: 64 * 6] = rng.integers(-3, 4, 64).astype(np.float32)  # integers, repeats
+    wq, absmax = O.quantize(w)
+    idx = O.unpack(wq)
+    for b in range(12):
+        blk = w[b * 64:(b + 1) * 64]
+        am = np.max(np.abs(blk))
+        assert absmax[b] == am
+        for j in range(64):
+            x = f32(blk[j]) / f32(am)       # IEEE fp32 division (numpy)
+            assert idx[b * 64 + j] == _exact_argmin(x, c), (b, j, blk[j], am)
+
+
+def test_quantize_at_and_around_every_midpoint():
+    """Place x exactly at each midpoint between neighbouring levels (when the
+    midpoint is an fp32 value), and one fp32 step either side of it."""
+    c = _levels()
+    vals = []
+    for j in range(15):
+        mid = (Fraction(float(c[j])) + Fraction(float(c[j + 1]))) / 2
+        m32 = f32(float(mid))
+        for v in (np.nextafter(m32, f32(-2)), m32, np.nextafter(m32, f32(2))):
+            vals.append(v)
+    vals = np.array(vals, dtype=np.float32)
+    n = len(vals)
+    pad = (-(n + 1)) % 64
+    w = np.concatenate([[f32(1.0)], vals, np.zeros(pad, np.float32)]).astype(np.float32)
+    wq, absmax = O.quantize(w)
+    idx = O.unpack(wq)
+    assert absmax[0] == 1.0
+    for i, v in enumerate(w):
+        assert idx[i] == _exact_argmin(v, c), (i, v)
+    # ties really occur and go to the lower index
+    ties = 0
+    for j in range(15):
+        mid = (Fraction(float(c[j])) + Fraction(float(c[j + 1]))) / 2
+        if Fraction(float(f32(float(mid)))) == mid:
+            ties += 1
+            pos = 1 + 3 * j + 1
+            assert idx[pos] == j
+    assert ties > 0
+
+
+def test_block_maximum_maps_to_an_end_level():
+    rng = np.random.default_rng(5)
+    w = (rng.standard_normal(64 * 50) * 0.02).astype(np.float32)
+    wq, absmax = O.quantize(w)
+    idx = O.unpack(wq)
+    for b in range(50):
+        blk = w[b * 64:(b + 1) * 64]
+        j = int(np.argmax(np.abs(blk)))
+        assert idx[b * 64 + j] == (15 if blk[j] > 0 else 0)
+
+
+def test_zero_block_and_negative_zero():
+    w = np.zeros(128, dtype=np.float32)
+    w[64:] = (np.arange(64, dtype=np.float32) - 32) / 64
+    w[70] = -0.0
+    wq, absmax = O.quantize(w)
+    idx = O.unpack(wq)
+    assert absmax[0] == 0.0 and np.all(idx[:64] == 7)
+    assert idx[70] == 7
+
+
+def test_packing_puts_the_even_element_in_the_high_nibble(golden):
+    ex = golden["block_layout_example"]
+    w = np.zeros(64, dtype=np.float32)
+    w[0], w[1] = 1.0, -1.0       # indices 15, 0
+    w[2], w[3] = 0.0, 1.0        # indices 7, 15
+    wq, _ = O.quantize(w)
+    assert wq.size * ex["codes_per_byte"] == 64
+    assert wq[0] == 0xF0 and wq[1] == 0x7F
+    assert np.all(wq[2:] == 0x77)
+
+
+def test_bf16_input_is_widened_exactly():
+    rng = np.random.default_rng(3)
+    wt = torch.from_numpy((rng.standard_normal(64 * 8) * 0.02).astype(np.float32)).to(torch.bfloat16)
+    bits = wt.view(torch.int16).numpy().view(np.uint16)
+    wq1, am1 = O.quantize(bits)
+    wq2, am2 = O.quantize(wt.float().numpy())
+    assert np.array_equal(wq1, wq2) and np.array_equal(am1, am2)
+
+
+# ---------------------------------------------------------------------------
+# bf16 rounding: the page's printed example and the IEEE tie rule.
+# ---------------------------------------------------------------------------
+
+def test_bf16_rounding_matches_the_page_example(golden):
+    ex = golden["bf16_rounding_example"]
+    x = np.array([f32(float(ex["input_decimal"]))], dtype=np.float32)
+    assert abs(float(x[0]) - ex["fp32_stored"]) < 1e-15
+    b = O.f32_to_bf16(x)
+    assert float(O.bf16_to_f32(b)[0]) == ex["bf16_stored"]
+
+
+def test_bf16_rounding_ties_to_even_and_matches_torch():
+    # 1 + 2^-8 is halfway between 1 and 1 + 2^-7: goes to 1 (even);
+    # 1 + 3 * 2^-8 is halfway between 1 + 2^-7 and 1 + 2^-6: goes to 1 + 2^-6.
+    x = np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8)], dtype=np.float32)
+    y = O.bf16_to_f32(O.f32_to_bf16(x))
+    assert y.tolist() == [1.0, 1 + 2 ** -6, -1.0]
+    rng = np.random.default_rng(9)
+    r = (rng.standard_normal(200000) * np.exp(rng.uniform(-20, 20, 200000))).astype(np.float32)
+    mine = O.f32_to_bf16(r)
+    ref = torch.from_numpy(r).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(mine, ref)
+
+
+# ---------------------------------------------------------------------------
+# Double quantization: closed-form storage, fixed summation order, 8-bit error
+# bound (xyzblog page, section 2.2 ②; zingnex page, paging and double-quant
+# section; yololab page, double quantization section).
+# ---------------------------------------------------------------------------
+
+def test_storage_overhead_closed_form(golden):
+    dq = golden["double_quant_overhead"]
+    n, k = 256, 4096
+    rng = np.random.default_rng(1)
+    w = (rng.standard_normal((n, k)) * 0.02).astype(np.float32)
+    wq, absmax = O.quantize(w)
+    q, s, mu = O.double_quant(absmax)
+    bits = (wq.nbytes + q.nbytes + s.nbytes) * 8 / (n * k)
+    assert bits == 4 + 8 / 64 + 32 / (64 * 256) == 4.126953125
+    assert dq["bits_per_param_absmax_fp32"] == 4 + absmax.nbytes * 8 / (n * k)
+    saving = dq["bits_per_param_absmax_fp32"] - bits
+    assert abs(saving - dq["saving_bits_per_param_approx"]) < 0.005
+    assert abs(saving - golden["double_quant_saving_forum"]["saving_bits_per_param_approx"]) < 0.005
+    assert abs(bits - dq["bits_per_param_after_dq_approx"]) < 0.005
+    fp = golden["footprint_70b"]
+    assert abs(fp["params"] * 16 / 8 / 1e9 - fp["fp16_gb_approx"]) < 1e-6
+    gb = fp["params"] * bits / 8 / 1e9
+    assert abs(gb - fp["nf4_gb_approx"]) / fp["nf4_gb_approx"] < 0.05
+
+
+def test_page_example_layout(golden):
+    ex = golden["block_layout_example"]
+    out = 3
+    w = (np.random.default_rng(2).standard_normal((out, ex["in_features"])) * 0.02).astype(np.float32)
+    wq, absmax = O.quantize(w)
+    assert absmax.size == out * ex["blocks_per_row"] == out * ex["in_features"] // ex["blocksize"]
+    assert wq.nbytes == ex["packed_fraction_of_fp16"] * (out * ex["in_features"] * 2)
+
+
+def test_dq_sum_follows_the_fixed_tree_order():
+    # Halving tree over a zero-padded chunk of 256: 1 + 2^53 rounds to 2^53
+    # (tie to even) at the h = 2 step, then 2^53 + 1 again rounds to 2^53.
+    # Summed left to right the same values would give 2^53 + 2.
+    a = np.array([1.0, 1.0, 2.0 ** 53, 0.0], dtype=np.float32)
+    assert O.dq_sum(a) == 2.0 ** 53
+    # with one more level (nb > 256) the chunk results are combined the same way
+    b = np.zeros(512, dtype=np.float32)
+    b[0], b[256] = 2.0 ** 53, 1.0
+    b[1] = 1.0
+    # chunk 0 -> 2^53 + 1 -> 2^53 (tie to even); chunk 1 -> 1; 2^53 + 1 -> 2^53
+    assert O.dq_sum(b) == 2.0 ** 53
+
+
+def test_dq_sum_is_the_exact_sum_when_representable():
+    rng = np.random.default_rng(4)
+    for nb in (1, 7, 256, 257, 1000, 70000):
+        a = (rng.uniform(0.01, 0.08, nb)).astype(np.float32)
+        exact = sum(Fraction(float(v)) for v in a)
+        assert Fraction(O.dq_sum(a)) == exact
+        mu = O.dq_mean(a)
+        true_mu = exact / nb
+        # one fp64 rounding then one fp32 rounding: within an fp32 ulp
+        assert abs(Fraction(float(mu)) - true_mu) <= Fraction(float(np.spacing(mu)))
+
+
+def test_double_quant_invariants_and_error_bound():
+    rng = np.random.default_rng(6)
+    nb = 1000  # 3 full blocks of 256 and a partial one
+    absmax = (np.abs(rng.standard_normal(nb)) * 0.03 + 0.01).astype(np.float32)
+    q, s, mu = O.double_quant(absmax)
+    assert q.dtype == np.int8 and s.size == 4
+    assert mu == O.dq_mean(absmax)
+    ahat = O.absmax_hat(q, s, mu)
+    for j in range(4):
+        lo, hi = 256 * j, min(256 * (j + 1), nb)
+        r = absmax[lo:hi].astype(np.float64) - float(mu)
+        assert s[j] == np.max(np.abs(f32(absmax[lo:hi]) - mu))
+        jm = int(np.argmax(np.abs(r)))
+        assert abs(int(q[lo + jm])) == 127
+        assert np.all(np.abs(q[lo:hi].astype(int)) <= 127)
+        assert np.all(np.sign(q[lo:hi]) * np.sign(r) >= 0)
+        order = np.argsort(absmax[lo:hi], kind="stable")
+        assert np.all(np.diff(q[lo:hi][order].astype(int)) >= 0)   # monotone in absmax
+        # 8-bit rounding error: at most half a step of s / 127, plus fp32 roundings
+        err = np.abs(ahat[lo:hi].astype(np.float64) - absmax[lo:hi])
+        assert np.all(err <= s[j] / 254 + 4 * np.spacing(np.float32(absmax[lo:hi].max())))
+
+
+def test_double_quant_constant_absmax_gives_zero_scale():
+    a = np.full(300, 0.037, dtype=np.float32)
+    q, s, mu = O.double_quant(a)
+    assert mu == f32(0.037) and np.all(s == 0) and np.all(q == 0)
+    assert np.all(O.absmax_hat(q, s, mu) == mu)
+
+
+# ---------------------------------------------------------------------------
+# Dequantization (technicalnotes page, section 5 dynamic dequantization).
+# ---------------------------------------------------------------------------
+
+def test_dequantize_error_bound_and_end_levels():
+    rng = np.random.default_rng(8)
+    n, k = 16, 1024
+    w = (rng.standard_normal((n, k)) * 0.02).astype(np.float32)
+    wq, absmax = O.quantize(w)
+    q, s, mu = O.double_quant(absmax)
+    wh = O.dequantize(wq, q, s, mu).reshape(n, k)
+    c = _levels().astype(np.float64)
+    half_gap = np.max(np.diff(c)) / 2
+    ahat = O.absmax_hat(q, s, mu).astype(np.float64)
+    wb = w.reshape(-1, 64).astype(np.float64)
+    whb = wh.reshape(-1, 64).astype(np.float64)
+    for b in range(wb.shape[0]):
+        bound = half_gap * absmax[b] + abs(ahat[b] - absmax[b]) + 1e-6 * absmax[b]
+        assert np.all(np.abs(whb[b] - wb[b]) <= bound)
+        j = int(np.argmax(np.abs(wb[b])))
+        assert whb[b, j] == np.sign(wb[b, j]) * f32(ahat[b])
+
+
+# ---------------------------------------------------------------------------
+# fp64 linear (xyzblog page, section 2.2 code walk: matmul_4bit = dequant + matmul).
+# ---------------------------------------------------------------------------
+
+def test_linear_against_numpy_float64_and_exact_integers():
+    rng = np.random.default_rng(10)
+    x = torch.from_numpy(rng.standard_normal((5, 96)).astype(np.float32)).to(torch.bfloat16)
+    w = torch.from_numpy((rng.standard_normal((7, 96)) * 0.02).astype(np.float32)).to(torch.bfloat16)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    wb = w.view(torch.int16).numpy().view(np.uint16)
+    y = O.linear_bf16(xb, wb)
+    ref = x.double().numpy() @ w.double().numpy().T
+    np.testing.assert_allclose(y, ref, rtol=1e-13, atol=1e-15)
+    xi = torch.tensor([[1, -2, 3], [0, 5, -1]], dtype=torch.bfloat16)
+    wi = torch.tensor([[2, 2, 2], [-1, 0, 4]], dtype=torch.bfloat16)
+    y = O.linear_bf16(xi.view(torch.int16).numpy().view(np.uint16),
+                      wi.view(torch.int16).numpy().view(np.uint16))
+    assert y.tolist() == [[4.0, 11.0], [8.0, -4.0]]
+
+
+def test_normalisation_is_a_true_division():
+    """x = w / absmax must be the correctly rounded quotient, not w * (1/absmax):
+    find weights where the two differ across a decision midpoint and check the
+    oracle follows the division."""
+    c = _levels()
+    found = 0
+    for a in (f32(0.7), f32(0.0311), f32(0.123456), f32(1.9e-3), f32(0.0517)):
+        recip = f32(1.0) / a
+        cases = []
+        for j in range(15):
+            mid = (Fraction(float(c[j])) + Fraction(float(c[j + 1]))) / 2
+            w0 = f32(float(mid * Fraction(float(a))))
+            w = w0
+            for _ in range(6):
+                w = np.nextafter(w, f32(-2))
+            for _ in range(13):
+                x_div = f32(w) / a
+                x_mul = f32(w) * recip
+                if _exact_argmin(x_div, c) != _exact_argmin(x_mul, c):
+                    cases.append(w)
+                w = np.nextafter(w, f32(2))
+        if not cases:
+            continue
+        blk = np.zeros(64, dtype=np.float32)
+        blk[0] = a
+        blk[1:1 + min(63, len(cases))] = cases[:63]
+        wq, absmax = O.quantize(blk)
+        idx = O.unpack(wq)
+        assert absmax[0] == a
+        for i in range(1, 1 + min(63, len(cases))):
+            assert idx[i] == _exact_argmin(f32(blk[i]) / a, c)
+        found += len(cases)
+    assert found > 0, "no weight distinguishes division from reciprocal multiply"
