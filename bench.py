@@ -1,0 +1,509 @@
+"""Benchmark of the NF4 hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--m 16]
+
+Workload (the decode configuration): the 224 linears of a Llama-7B-shaped
+decoder stack (32 layers x {q,k,v,o 4096x4096; gate,up 11008x4096; down
+4096x11008}), bf16 weights ~N(0, 0.02^2) quantized to NF4 + double quantization
+(3.34 GB), and bf16 activations ~N(0, 1) with M tokens.  One step = one decode
+pass: nf4_linear on every one of the 224 weights (fused dequant-GEMV), replayed
+from a CUDA graph.  The weights read per step are 26x the 126 MB L2, so every
+step streams from HBM.
+
+Printed: one JSON line.  ``value`` = whole-job HBM GB/s of algorithmic bytes
+(NF4 weight + metadata + X + Y) over the timed steps; extra legs in the same
+run report M = 1 and 4, the dequant-GEMM TFLOP/s at M = 4096 (K = 4096,
+N = 11008), quantize + double-quant and dequantize GB/s over the stack, the
+end-to-end rate through the C ABI with host buffers, the roofline of the GEMV
+kernel and the CPU oracle's rate on a bounded sample.
+
+``--impl reference`` times the CPU oracle (the reference arm) on a bounded
+sample of the same workload and prints the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "NF4 dequant-GEMV HBM GB/s (% peak); dequant-GEMM TFLOP/s at M=4096"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+WORKLOAD = "llama7b-shaped decode: 224 NF4+DQ linears (32 x q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008)"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def linear_bytes(n: int, k: int, m: int, y_bytes: int) -> int:
+    """Algorithmic bytes of one fused linear: packed codes, absmax codes, DQ
+    scales and mean, X read once, Y written once."""
+    nb = n * k // 64
+    return n * k // 2 + nb + 4 * ((nb + 255) // 256) + 4 + 2 * m * k + y_bytes * m * n
+
+
+def quant_bytes(n: int, k: int) -> int:
+    """Algorithmic bytes of quantize + double quant from bf16: read W, write
+    codes, absmax codes, scales and mean."""
+    nb = n * k // 64
+    return 2 * n * k + n * k // 2 + nb + 4 * ((nb + 255) // 256) + 4
+
+
+def dequant_bytes(n: int, k: int) -> int:
+    nb = n * k // 64
+    return n * k // 2 + nb + 4 * ((nb + 255) // 256) + 4 + 2 * n * k
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi sampled every 100 ms from before the warm-up until after the
+    timed region; summary() keeps the samples that fall inside the timed region
+    (widened by 150 ms on each side when the region is shorter than the
+    sampling interval)."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = ""
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        import datetime
+        rows = []
+        for r in csv.reader(io.StringIO(self.out or "")):
+            if len(r) < 10:
+                continue
+            try:
+                t = datetime.datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                continue
+            rows.append((t, [x.strip() for x in r[1:]]))
+        if not rows or self.t0 is None or self.t1 is None:
+            return None
+        inside = [f for t, f in rows if self.t0 <= t <= self.t1]
+        if not inside:
+            inside = [f for t, f in rows if self.t0 - 0.15 <= t <= self.t1 + 0.15]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(f[1]) for f in inside if num(f[1]) is not None]
+        mx = [num(f[2]) for f in inside if num(f[2]) is not None]
+        pw = [num(f[3]) for f in inside if num(f[3]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for f in inside:
+            for name, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_median": statistics.median(pw) if pw else None,
+                "reasons": sorted(reasons), "samples": len(inside)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (weak scaling: every rank runs its own copy of the
+# workload; no collective on the data path)
+# ---------------------------------------------------------------------------
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle on a bounded sample (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+def oracle_gemv_rate(m: int, budget_s: float):
+    """Oracle dequant-GEMV on a 512 x 4096 slab of a q_proj-shaped weight:
+    oracle quantize + double quant (untimed), then timed repetitions of
+    dequantize rows -> bf16 -> fp64 dot products with M tokens.  Returns
+    (GB/s of algorithmic bytes, description, seconds)."""
+    import numpy as np
+    import torch
+
+    import oracle as O
+    from quantized_linear_layers_nf4_b200 import synth
+    rows, k = 512, 4096
+    w = synth.weight_normal(rows, k, seed=synth.seed_for(4, 0), dtype=torch.bfloat16)
+    x = synth.activations(m, k, seed=synth.seed_for(2, 100 + m))
+    wh = w.view(torch.int16).numpy().view(np.uint16).reshape(-1)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    wq, am = O.quantize(wh)
+    q, s, mu = O.double_quant(am)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        d = O.dequantize_range(wq, q, s, mu, 0, rows * k)
+        wb = O.f32_to_bf16(d).reshape(rows, k)
+        O.linear_bf16(xb, wb)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    gbs = reps * linear_bytes(rows, k, m, 2) / el / 1e9
+    desc = ("oracle dequant-GEMV (dequantize, bf16 round, fp64 dot products) of a 512x4096 NF4+DQ "
+            "slab at M=%d, %d repetitions in %.1f s, one thread" % (m, reps, el))
+    return gbs, desc, el
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    t_all = time.perf_counter()
+    per_step = []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        gbs, desc, el = oracle_gemv_rate(args.m, budget_s=max(2.0, 8.0 / max(1, args.steps)))
+        if i >= args.warmup:
+            per_step.append((gbs, el))
+    value = statistics.mean(g for g, _ in per_step)
+    ms = 1000.0 * statistics.mean(e for _, e in per_step)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "m": args.m, "sample": "512x4096 slab"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "wall_s": round(time.perf_counter() - t_all, 1),
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU legs
+# ---------------------------------------------------------------------------
+def _events_time(fn, reps, stream):
+    import torch
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(reps):
+        fn()
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end) / 1000.0 / reps
+
+
+def gemv_traffic(kernel_src: str):
+    """DRAM bytes per launch of the GEMV kernel from the committed ncu summary,
+    or None when the kernel source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get("gemv")
+    if not ent:
+        return None
+    sha = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
+    if ent.get("source_sha") != sha:
+        return None
+    return ent.get("dram_bytes_per_launch_scaled")
+
+
+def run_ours(args, rank, world, local):
+    import torch
+
+    import quantized_linear_layers_nf4_b200 as nf4
+    from quantized_linear_layers_nf4_b200 import synth
+    from quantized_linear_layers_nf4_b200.build import build
+
+    if rank == 0:
+        build()
+    barrier(world)
+    nf4._lib.lib()
+    pk, pk_kind = peaks()
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    # ---- weights: 224 NF4 tensors (quantized on device from seeded bf16) ----
+    stack = synth.llama7b_stack(args.layers)
+    weights = []
+    for idx, (_, _, n, k) in enumerate(stack):
+        W = synth.weight_normal(n, k, seed=synth.seed_for(4, idx), dtype=torch.bfloat16, device=dev)
+        weights.append(nf4.quantize_weight(W))
+        del W
+    torch.cuda.synchronize()
+    shapes = sorted(set((w.n, w.k) for w in weights))
+
+    def decode_setup(m):
+        xs = {k: synth.activations(m, k, seed=synth.seed_for(2, 100 + m) + k, device=dev)
+              for k in set(k for _, k in shapes)}
+        ys = {n: torch.empty((m, n), dtype=torch.bfloat16, device=dev) for n in set(n for n, _ in shapes)}
+
+        def step():
+            for w in weights:
+                nf4.nf4_linear(xs[w.k], w, torch.bfloat16, out=ys[w.n])
+        step()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        torch.cuda.synchronize()
+        nbytes = sum(linear_bytes(w.n, w.k, m, 2) for w in weights)
+        return g, xs, ys, nbytes
+
+    # ---- main leg: decode pass at M = args.m ----
+    g, xs, ys, step_bytes = decode_setup(args.m)
+    clk = ClockSampler(local)
+    clk.start()
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    clk.mark_start()
+    start.record(stream)
+    for _ in range(args.steps):
+        g.replay()
+    end.record(stream)
+    end.synchronize()
+    clk.mark_end()
+    clk.stop()
+    barrier(world)
+    t_step = start.elapsed_time(end) / 1000.0 / args.steps
+    t_step_max = max_over_ranks(t_step, world)
+    total_bytes = sum_over_ranks(float(step_bytes), world)
+    value = total_bytes / t_step_max / 1e9
+    launches_per_step = len(weights)
+    avg_launch_s = t_step / launches_per_step
+    bytes_per_launch = step_bytes / launches_per_step
+
+    # ---- e2e: host buffers through the C ABI, copies inside the timed region ----
+    xh = {k: x.cpu().pin_memory() for k, x in xs.items()}
+    yh = {n: torch.empty(y.shape, dtype=y.dtype).pin_memory() for n, y in ys.items()}
+    h2d = sum(x.numel() * x.element_size() for x in xh.values())
+    d2h = sum(y.numel() * y.element_size() for y in yh.values())
+
+    def e2e_step():
+        for k, x in xh.items():
+            xs[k].copy_(x, non_blocking=True)
+        g.replay()
+        for n, y in ys.items():
+            yh[n].copy_(y, non_blocking=True)
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier(world)
+    t_e2e = max_over_ranks(_events_time(e2e_step, args.steps, stream), world)
+    e2e_value = total_bytes / t_e2e / 1e9
+    del g
+
+    # ---- extra legs (rank-local, reported for rank 0) ----
+    by_m = {args.m: round(step_bytes / t_step / 1e9, 1)}
+    for m in (1, 4, 16):
+        if m == args.m:
+            continue
+        gm, _, _, bm = decode_setup(m)
+        for _ in range(2):
+            gm.replay()
+        by_m[m] = round(bm / _events_time(gm.replay, max(2, args.steps // 2), stream) / 1e9, 1)
+        del gm
+
+    # dequant-GEMM at M = 4096, K = 4096, N = 11008
+    gemm = None
+    if not args.skip_gemm:
+        Wg = synth.weight_normal(11008, 4096, seed=synth.seed_for(3, 0), dtype=torch.bfloat16, device=dev)
+        wg = nf4.quantize_weight(Wg)
+        del Wg
+        Xg = synth.activations(4096, 4096, seed=synth.seed_for(3, 1), device=dev)
+        Yg = torch.empty((4096, 11008), dtype=torch.bfloat16, device=dev)
+        fn = lambda: nf4.nf4_linear(Xg, wg, torch.bfloat16, out=Yg)
+        fn()
+        t_g = _events_time(fn, 3, stream)
+        tflops = 2.0 * 4096 * 4096 * 11008 / t_g / 1e12
+        gemm = {"m": 4096, "k": 4096, "n": 11008, "tflops": round(tflops, 2),
+                "ms": round(t_g * 1e3, 3), "peak_tflops": pk["bf16_tflops"],
+                "frac": round(tflops / pk["bf16_tflops"], 4), "peak_kind": pk_kind + " burst bf16"}
+        del Xg, Yg, wg
+
+    # quantize + double quant, and dequantize, over the stack
+    qd = None
+    if not args.skip_quant:
+        maxn = max(n * k for n, k in shapes)
+        Wb = torch.empty(maxn, dtype=torch.bfloat16, device=dev)
+        out = torch.empty(maxn, dtype=torch.bfloat16, device=dev)
+        wq = torch.empty(maxn // 2, dtype=torch.uint8, device=dev)
+        am = torch.empty(maxn // 64, dtype=torch.float32, device=dev)
+        aq = torch.empty(maxn // 64, dtype=torch.int8, device=dev)
+        sc = torch.empty(maxn // 64 // 256 + 1, dtype=torch.float32, device=dev)
+        mu = torch.empty(1, dtype=torch.float32, device=dev)
+        ws = torch.empty(maxn // 64 // 256 + 2, dtype=torch.float64, device=dev)
+        Wb.normal_(0.0, 0.02)
+        sub = weights[:7]
+
+        def qstep():
+            for w in sub:
+                v = Wb[: w.n * w.k].view(w.n, w.k)
+                nf4.nf4_quantize(v, wq, am)
+                nf4.nf4_double_quant(am[: w.n * w.k // 64], aq, sc, mu, ws)
+
+        def dstep():
+            for w in sub:
+                nf4.nf4_dequantize(w, torch.bfloat16, out=out[: w.n * w.k].view(w.n, w.k))
+        qstep(); dstep()
+        tq = _events_time(qstep, 5, stream)
+        td = _events_time(dstep, 5, stream)
+        qb = sum(quant_bytes(w.n, w.k) for w in sub)
+        db = sum(dequant_bytes(w.n, w.k) for w in sub)
+        qd = {"quantize_dq_gbs": round(qb / tq / 1e9, 1), "dequantize_bf16_gbs": round(db / td / 1e9, 1),
+              "sample": "one decoder layer (7 tensors, 202M params) per rep, bf16 in/out"}
+        del Wb, out
+
+    clocks = clk.summary()
+    result = None
+    if rank == 0:
+        traffic = gemv_traffic(os.path.join(ROOT, "quantized_linear_layers_nf4_b200", "csrc", "nf4_gemv.cu"))
+        achieved = bytes_per_launch / avg_launch_s / 1e9
+        result = {
+            "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_step_max * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "m": args.m, "layers": args.layers,
+                       "weights_gb_per_step": round(step_bytes / 1e9, 3),
+                       "l2": "inputs larger than L2 (%.2f GB of NF4 weights per step vs 126 MB)"
+                             % (sum(w.nbytes() for w in weights) / 1e9),
+                       "y_dtype": "bf16", "parallelism": "replicas (weak scaling)"},
+            "frac_of_peak": round(value / world / pk["hbm_gbs"], 4),
+            "decode_gbs_by_m": by_m,
+            "gemm": gemm,
+            "quant": qd,
+            "roofline": {"bound": "hbm", "kernel": "k_nf4_gemv", "achieved": round(achieved, 1),
+                         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
+                         "traffic": traffic, "peak_kind": pk_kind,
+                         "algorithmic_bytes_per_launch": int(bytes_per_launch)},
+            "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+        }
+    return result
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--m", type=int, default=16, help="tokens per decode step (1..16)")
+    ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--skip-gemm", action="store_true")
+    ap.add_argument("--skip-quant", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+            return
+        result = run_ours(args, rank, world, local)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                gbs, desc, _ = oracle_gemv_rate(args.m, budget_s=10.0)
+                result["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1,
+                                          "kind": "oracle", "sample": desc}
+            else:
+                result["cpu_baseline"] = None
+            print(json.dumps(result), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

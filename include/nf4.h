@@ -1,0 +1,191 @@
+/*
+ * nf4.h -- C ABI of libnf4.so: NF4 weight quantization, double quantization,
+ * dequantization and the fused dequantize + bf16 linear, for NVIDIA B200
+ * (sm_100a).
+ *
+ * Sources (web pages, cited by title and section):
+ *   [P1] "Tim Dettmers 如何用 bitsandbytes 與 QLoRA 降低 LLM 訓練門檻？" (yololab.net)
+ *   [P3] "bitsandbytes：让大语言模型在消费级硬件上运行的量化神器" (zingnex.cn)
+ *   [P4] "LLM 相關知識" (technicalnotes, tag qlora)
+ *   [P5] "篇2-bitsandbytes-具体观-算法与实现剖析" (xyzblog)
+ *
+ * General rules for every entry point:
+ *   - All tensor arguments are DEVICE pointers on the current CUDA device, except
+ *     the nf4_weight_t struct itself, which lives in host memory and borrows
+ *     device pointers.  The caller allocates and frees every buffer; the library
+ *     never allocates, never frees and never synchronizes the host.
+ *   - Work is enqueued on `stream` (NULL = the legacy default stream) and runs
+ *     asynchronously; outputs are valid once the stream reaches that point.
+ *   - Arguments are validated on the host BEFORE anything is launched; on an
+ *     error nothing is enqueued and the status says why.  A launch failure
+ *     reported by the runtime maps to NF4_ERR_CUDA.
+ *   - Inputs must be finite (documented precondition, not checked on device).
+ *   - Layouts are row-major and dense.  "Element e" of a weight W[n, k] is
+ *     W[e / k][e % k]; blocks of 64 are consecutive runs of elements.
+ *   - The library requires a compute-capability 10.x device; other devices get
+ *     NF4_ERR_UNSUPPORTED.
+ */
+#ifndef NF4_H
+#define NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t (a pointer to the runtime's opaque stream object). */
+struct CUstream_st;
+typedef struct CUstream_st* nf4_stream_t;
+
+typedef enum nf4_status {
+    NF4_OK = 0,
+    NF4_ERR_NULL = -1,            /* a required pointer is NULL */
+    NF4_ERR_SHAPE = -2,           /* a size is out of range or not a multiple of the block size */
+    NF4_ERR_ALIGN = -3,           /* a pointer is not 16-byte aligned */
+    NF4_ERR_DTYPE = -4,           /* unsupported dtype code */
+    NF4_ERR_STATE = -5,           /* nf4_weight_t has a bad magic, version or block size */
+    NF4_ERR_WORKSPACE = -6,       /* workspace missing or smaller than required */
+    NF4_ERR_CUDA = -7,            /* the CUDA runtime reported an error */
+    NF4_ERR_DEVICE_TIMEOUT = -8,  /* a bounded device-side wait ran out (written to dev_status) */
+    NF4_ERR_UNSUPPORTED = -9      /* current device is not compute capability 10.x */
+} nf4_status_t;
+
+/* Element types of weights, activations and outputs. */
+typedef enum nf4_dtype {
+    NF4_F32 = 0,   /* IEEE binary32 */
+    NF4_BF16 = 1   /* bfloat16 (top half of a binary32) */
+} nf4_dtype_t;
+
+#define NF4_ABI_VERSION 1
+#define NF4_BLOCKSIZE 64          /* weights per absmax ([P5] §2.2 example: "split by 64") */
+#define NF4_BLOCKSIZE2 256        /* absmax values per double-quantization block */
+#define NF4_WEIGHT_MAGIC 0x4E463442u /* "NF4B" */
+#define NF4_WEIGHT_VERSION 1u
+
+/*
+ * A quantized weight W[n, k] (out_features n, in_features k) as produced by
+ * nf4_quantize + nf4_double_quant: the nested quantization state of [P5] §2.2
+ * code walk (packed 4-bit weight, absmax quantized again as "state2", plus the
+ * offset that double quantization subtracts).  Host struct; the pointers are
+ * device pointers owned by the caller.
+ *   wq            uint8  [n*k/2]      two 4-bit level indices per byte, element 2i
+ *                                     in the high nibble of byte i
+ *   absmax_q      int8   [n*k/64]     double-quantized absmax codes
+ *   absmax_scale  fp32   [ceil(n*k/64/256)]  one scale per 256 absmax values
+ *   absmax_offset fp32   [1]          the mean subtracted before double quantization
+ */
+typedef struct nf4_weight {
+    uint32_t magic;       /* NF4_WEIGHT_MAGIC */
+    uint32_t version;     /* NF4_WEIGHT_VERSION */
+    int64_t n;            /* rows (out_features) */
+    int64_t k;            /* columns (in_features) */
+    int32_t blocksize;    /* must be NF4_BLOCKSIZE */
+    int32_t blocksize2;   /* must be NF4_BLOCKSIZE2 */
+    const uint8_t* wq;
+    const int8_t* absmax_q;
+    const float* absmax_scale;
+    const float* absmax_offset;
+} nf4_weight_t;
+
+/* ABI version of the loaded library (NF4_ABI_VERSION it was built with). */
+int nf4_abi_version(void);
+
+/* Static, human-readable name of a status code. */
+const char* nf4_status_str(int status);
+
+/* The 16 NF4 levels the library uses, ascending, copied to host memory
+ * `levels_out[16]` ([P5] §2.2 principle ①: N(0,1) quantiles normalised to
+ * [-1, 1]; [P1] section on NF4 not being a generic FP4).  Returns NF4_OK or
+ * NF4_ERR_NULL.  Host-only; launches nothing. */
+nf4_status_t nf4_codebook(float* levels_out);
+
+/*
+ * nf4_quantize -- blockwise NF4 quantization ([P5] §2.2 worked example and
+ * Figure 2-2 steps 1-4; [P1] "NF4 不是一般四位元浮點格式").
+ * For every block b of 64 consecutive elements of W:
+ *     absmax[b] = max_j |w_j|;  x_j = w_j / absmax[b]  (IEEE fp32, round to nearest even);
+ *     idx_j = index of the level nearest to x_j, ties to the lower index
+ *     (a block whose absmax is 0 maps every element to the zero level, index 7);
+ *     wq[32b + i] = (idx_{2i} << 4) | idx_{2i+1}.
+ *   W        device, [n, k] of w_dtype (NF4_F32 or NF4_BF16; bf16 is widened exactly)
+ *   wq       device, uint8 [n*k/2]       (output)
+ *   absmax   device, fp32  [n*k/64]      (output)
+ * Errors: NF4_ERR_NULL, NF4_ERR_SHAPE (n <= 0, k <= 0 or n*k % 64 != 0),
+ * NF4_ERR_ALIGN (W or wq not 16-byte aligned, absmax not 4-byte aligned),
+ * NF4_ERR_DTYPE, NF4_ERR_UNSUPPORTED, NF4_ERR_CUDA.
+ */
+nf4_status_t nf4_quantize(const void* W, nf4_dtype_t w_dtype, int64_t n, int64_t k,
+                          uint8_t* wq, float* absmax, nf4_stream_t stream);
+
+/* Bytes of workspace nf4_double_quant needs for nb absmax values (0 if nb <= 0). */
+size_t nf4_double_quant_workspace_bytes(int64_t nb);
+
+/*
+ * nf4_double_quant -- double quantization of the absmax constants ([P5] §2.2
+ * principle ② and Figure 2-2 step 5; [P1] "Double quantization 連 scale 本身也壓縮";
+ * [P3] "分页优化器与双量化").
+ *     mu = fp32(S / nb), S the fp64 sum of all absmax in a fixed tree order:
+ *          the list is cut into chunks of 256 (last chunk zero-padded), each chunk
+ *          reduced by a[i] += a[i + h] for h = 128, 64, ..., 1, the chunk results
+ *          form the next list, until one value is left;
+ *     r_b = fp32(absmax[b] - mu);
+ *     per block j of 256 absmax: s_j = max |r_b|,
+ *          q_b = round_half_even(fp32(fp32(r_b / s_j) * 127)), q_b = 0 when s_j = 0.
+ *   absmax        device, fp32 [nb]                 (input)
+ *   workspace     device, >= nf4_double_quant_workspace_bytes(nb), 8-byte aligned;
+ *                 scratch, contents undefined afterwards
+ *   absmax_q      device, int8 [nb]                 (output)
+ *   absmax_scale  device, fp32 [ceil(nb/256)]       (output)
+ *   absmax_offset device, fp32 [1]                  (output: mu)
+ * Errors: NF4_ERR_NULL, NF4_ERR_SHAPE (nb <= 0), NF4_ERR_ALIGN, NF4_ERR_WORKSPACE,
+ * NF4_ERR_UNSUPPORTED, NF4_ERR_CUDA.
+ */
+nf4_status_t nf4_double_quant(const float* absmax, int64_t nb, void* workspace,
+                              size_t workspace_bytes, int8_t* absmax_q, float* absmax_scale,
+                              float* absmax_offset, nf4_stream_t stream);
+
+/*
+ * nf4_dequantize -- NF4 + double-quantization state back to real values ([P4]
+ * §5 "動態反量化": restore the 4-bit weights to the compute dtype; [P1] the frozen
+ * 4-bit base is dequantized in forward and backward).  For element e in block b:
+ *     a_b = fp32(fp32(fp32(q_b / 127) * s_{b/256}) + mu);
+ *     out[e] = fp32(c[idx_e] * a_b)          for out_dtype NF4_F32,
+ *     out[e] = bf16_round_nearest_even(...)  for out_dtype NF4_BF16.
+ *   w    host struct (validated: magic, version, block sizes, n*k % 64 == 0)
+ *   out  device, [n, k] of out_dtype, 16-byte aligned  (output)
+ * Errors: NF4_ERR_NULL, NF4_ERR_STATE, NF4_ERR_SHAPE, NF4_ERR_ALIGN, NF4_ERR_DTYPE,
+ * NF4_ERR_UNSUPPORTED, NF4_ERR_CUDA.
+ */
+nf4_status_t nf4_dequantize(const nf4_weight_t* w, void* out, nf4_dtype_t out_dtype,
+                            nf4_stream_t stream);
+
+/*
+ * nf4_linear -- Y = X * What^T with What the bf16 dequantized weight, fused:
+ * the weight is dequantized tile by tile on chip and never written out ([P5]
+ * §2.2 code walk: matmul_4bit(x, weight, bias, quant_state) dequantizes and
+ * multiplies; [P4] §5: per layer, 4-bit weights are restored to BF16 for the
+ * matrix multiply and discarded; [P1] "量化速度取決於硬體與 kernel": without fusion
+ * 4-bit can be slower than fp16, and the batch size moves the work between
+ * memory- and compute-bound).  What[r][c] = bf16_round(fp32(c[idx] * a_b)); the
+ * products are accumulated in fp32 in an unspecified order.  Small m (decode)
+ * runs a bandwidth-bound dequant-GEMV on the tensor cores; large m (prefill)
+ * runs a tcgen05 dequant-GEMM.
+ *   X          device, bf16 [m, k], 16-byte aligned rows (k % 64 == 0 required)
+ *   m          rows of X (tokens), >= 1
+ *   w          host struct describing the [n, k] quantized weight
+ *   Y          device, [m, n] of y_dtype (NF4_F32 or NF4_BF16), 16-byte aligned (output)
+ *   dev_status device int32 [1] or NULL; kernels with bounded waits write
+ *              NF4_ERR_DEVICE_TIMEOUT there if a wait runs out (never cleared by
+ *              the library; the caller zeroes it)
+ * Errors: NF4_ERR_NULL, NF4_ERR_STATE, NF4_ERR_SHAPE (m < 1, k % 64 != 0),
+ * NF4_ERR_ALIGN, NF4_ERR_DTYPE, NF4_ERR_UNSUPPORTED, NF4_ERR_CUDA.
+ */
+nf4_status_t nf4_linear(const void* X, int64_t m, const nf4_weight_t* w, void* Y,
+                        nf4_dtype_t y_dtype, int32_t* dev_status, nf4_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NF4_H */

@@ -1,0 +1,154 @@
+"""NF4 (4-bit NormalFloat) weight quantization with double quantization, and the
+fused dequantize + bf16 linear, for NVIDIA B200 (sm_100a).
+
+The work is done by ``lib/libnf4.so`` (C ABI in ``include/nf4.h``); this module
+only marshals PyTorch device tensors and the current CUDA stream into those
+calls.  Functions carry the C names:
+
+* ``nf4_quantize(W)`` -> ``(wq, absmax)``
+* ``nf4_double_quant(absmax)`` -> ``(absmax_q, absmax_scale, absmax_offset)``
+* ``nf4_dequantize(weight, dtype)`` -> dense tensor
+* ``nf4_linear(X, weight, dtype)`` -> ``Y = X @ W_hat^T``
+
+``quantize_weight(W)`` runs the first two and returns an ``NF4Weight``.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import NF4_BF16, NF4_F32, NF4Error, nf4_weight_t
+
+__all__ = ["NF4Weight", "NF4Error", "nf4_quantize", "nf4_double_quant", "nf4_dequantize",
+           "nf4_linear", "quantize_weight", "nf4_codebook", "library_path"]
+
+_DTYPES = {torch.float32: NF4_F32, torch.bfloat16: NF4_BF16}
+
+
+def library_path() -> str:
+    return _lib.LIB_PATH
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: torch.Tensor) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _need_cuda(t: torch.Tensor, name: str) -> None:
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def nf4_codebook() -> torch.Tensor:
+    """The 16 levels the library uses (host copy)."""
+    out = torch.zeros(16, dtype=torch.float32)
+    _lib.check(_lib.lib().nf4_codebook(_ptr(out)), "nf4_codebook")
+    return out
+
+
+def nf4_quantize(W: torch.Tensor, wq: torch.Tensor | None = None, absmax: torch.Tensor | None = None,
+                 stream=None):
+    """Blockwise NF4 quantization of a 2-D fp32/bf16 CUDA tensor [n, k]."""
+    _need_cuda(W, "W")
+    if W.dim() != 2 or W.dtype not in _DTYPES:
+        raise ValueError("W must be a 2-D float32 or bfloat16 tensor")
+    n, k = W.shape
+    numel = n * k
+    if wq is None:
+        wq = torch.empty(numel // 2, dtype=torch.uint8, device=W.device)
+    if absmax is None:
+        absmax = torch.empty(numel // 64, dtype=torch.float32, device=W.device)
+    _lib.check(_lib.lib().nf4_quantize(_ptr(W), _DTYPES[W.dtype], n, k, _ptr(wq), _ptr(absmax),
+                                       _stream(stream)), "nf4_quantize")
+    return wq, absmax
+
+
+def nf4_double_quant(absmax: torch.Tensor, absmax_q: torch.Tensor | None = None,
+                     absmax_scale: torch.Tensor | None = None,
+                     absmax_offset: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None, stream=None):
+    """Double quantization of the fp32 absmax vector."""
+    _need_cuda(absmax, "absmax")
+    nb = absmax.numel()
+    L = _lib.lib()
+    ws_bytes = L.nf4_double_quant_workspace_bytes(nb)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 8) // 8 + 1, dtype=torch.float64, device=absmax.device)
+    if absmax_q is None:
+        absmax_q = torch.empty(nb, dtype=torch.int8, device=absmax.device)
+    if absmax_scale is None:
+        absmax_scale = torch.empty((nb + 255) // 256, dtype=torch.float32, device=absmax.device)
+    if absmax_offset is None:
+        absmax_offset = torch.empty(1, dtype=torch.float32, device=absmax.device)
+    _lib.check(L.nf4_double_quant(_ptr(absmax), nb, _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _ptr(absmax_q),
+                                  _ptr(absmax_scale), _ptr(absmax_offset), _stream(stream)),
+               "nf4_double_quant")
+    return absmax_q, absmax_scale, absmax_offset
+
+
+@dataclass
+class NF4Weight:
+    """A quantized [n, k] weight: device tensors plus the C struct that borrows them."""
+    n: int
+    k: int
+    wq: torch.Tensor
+    absmax_q: torch.Tensor
+    absmax_scale: torch.Tensor
+    absmax_offset: torch.Tensor
+
+    def struct(self) -> nf4_weight_t:
+        return nf4_weight_t(_lib.NF4_WEIGHT_MAGIC, _lib.NF4_WEIGHT_VERSION, self.n, self.k,
+                            _lib.NF4_BLOCKSIZE, _lib.NF4_BLOCKSIZE2, self.wq.data_ptr(),
+                            self.absmax_q.data_ptr(), self.absmax_scale.data_ptr(),
+                            self.absmax_offset.data_ptr())
+
+    def nbytes(self) -> int:
+        return (self.wq.numel() + self.absmax_q.numel() + 4 * self.absmax_scale.numel())
+
+
+def quantize_weight(W: torch.Tensor, stream=None) -> NF4Weight:
+    """nf4_quantize followed by nf4_double_quant; the fp32 absmax is dropped."""
+    wq, absmax = nf4_quantize(W, stream=stream)
+    q, s, mu = nf4_double_quant(absmax, stream=stream)
+    return NF4Weight(W.shape[0], W.shape[1], wq, q, s, mu)
+
+
+def nf4_dequantize(weight: NF4Weight, dtype=torch.bfloat16, out: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    if dtype not in _DTYPES:
+        raise ValueError("dtype must be float32 or bfloat16")
+    if out is None:
+        out = torch.empty((weight.n, weight.k), dtype=dtype, device=weight.wq.device)
+    st = weight.struct()
+    _lib.check(_lib.lib().nf4_dequantize(ctypes.byref(st), _ptr(out), _DTYPES[dtype],
+                                         _stream(stream)), "nf4_dequantize")
+    return out
+
+
+def nf4_linear(X: torch.Tensor, weight: NF4Weight, dtype=torch.bfloat16,
+               out: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """Y = X @ W_hat^T for bf16 X [m, k]; Y [m, n] in ``dtype`` (bf16 or fp32)."""
+    _need_cuda(X, "X")
+    if X.dtype != torch.bfloat16 or X.dim() != 2:
+        raise ValueError("X must be a 2-D bfloat16 tensor")
+    if dtype not in _DTYPES:
+        raise ValueError("dtype must be float32 or bfloat16")
+    m = X.shape[0]
+    if out is None:
+        out = torch.empty((m, weight.n), dtype=dtype, device=X.device)
+    st = weight.struct()
+    ds = ctypes.c_void_p(0) if dev_status is None else _ptr(dev_status)
+    _lib.check(_lib.lib().nf4_linear(_ptr(X), m, ctypes.byref(st), _ptr(out), _DTYPES[dtype], ds,
+                                     _stream(stream)), "nf4_linear")
+    return out

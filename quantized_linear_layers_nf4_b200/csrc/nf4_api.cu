@@ -1,0 +1,163 @@
+// nf4_api.cu -- the extern "C" entry points of libnf4.so (declared in include/nf4.h).
+//
+// Each entry point validates its arguments on the host, then enqueues kernels
+// on the caller's stream.  Nothing is launched when validation fails, nothing
+// is allocated, and the host is never synchronized.
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "nf4.h"
+#include "nf4_internal.h"
+#include "nf4_levels.h"
+
+namespace nf4 {
+
+cudaError_t current_device(DeviceInfo* out) {
+    static std::mutex mu;
+    static DeviceInfo cache[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[dev].device != dev) {
+        DeviceInfo d;
+        d.device = dev;
+        if ((e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        if ((e = cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess) return e;
+        if ((e = cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess) return e;
+        int optin = 0;
+        if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
+        d.smem_optin = static_cast<size_t>(optin);
+        cache[dev] = d;
+    }
+    *out = cache[dev];
+    return cudaSuccess;
+}
+
+}  // namespace nf4
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Device check shared by every launching entry point.
+nf4_status_t device_ok(nf4::DeviceInfo* dev) {
+    if (nf4::current_device(dev) != cudaSuccess) {
+        cudaGetLastError();
+        return NF4_ERR_CUDA;
+    }
+    if (dev->major != 10) return NF4_ERR_UNSUPPORTED;
+    return NF4_OK;
+}
+
+nf4_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? NF4_OK : NF4_ERR_CUDA; }
+
+nf4_status_t check_weight(const nf4_weight_t* w) {
+    if (!w) return NF4_ERR_NULL;
+    if (w->magic != NF4_WEIGHT_MAGIC || w->version != NF4_WEIGHT_VERSION ||
+        w->blocksize != NF4_BLOCKSIZE || w->blocksize2 != NF4_BLOCKSIZE2)
+        return NF4_ERR_STATE;
+    if (!w->wq || !w->absmax_q || !w->absmax_scale || !w->absmax_offset) return NF4_ERR_NULL;
+    if (w->n <= 0 || w->k <= 0) return NF4_ERR_SHAPE;
+    if (w->n > INT64_MAX / w->k) return NF4_ERR_SHAPE;
+    if ((w->n * w->k) % NF4_BLOCKSIZE != 0) return NF4_ERR_SHAPE;
+    if (!aligned(w->wq, 16) || !aligned(w->absmax_scale, 4) || !aligned(w->absmax_offset, 4))
+        return NF4_ERR_ALIGN;
+    return NF4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int nf4_abi_version(void) { return NF4_ABI_VERSION; }
+
+const char* nf4_status_str(int status) {
+    switch (status) {
+        case NF4_OK: return "NF4_OK";
+        case NF4_ERR_NULL: return "NF4_ERR_NULL: a required pointer is NULL";
+        case NF4_ERR_SHAPE: return "NF4_ERR_SHAPE: size out of range or not a multiple of the block size";
+        case NF4_ERR_ALIGN: return "NF4_ERR_ALIGN: pointer not 16-byte aligned";
+        case NF4_ERR_DTYPE: return "NF4_ERR_DTYPE: unsupported dtype";
+        case NF4_ERR_STATE: return "NF4_ERR_STATE: bad nf4_weight_t magic, version or block size";
+        case NF4_ERR_WORKSPACE: return "NF4_ERR_WORKSPACE: workspace missing or too small";
+        case NF4_ERR_CUDA: return "NF4_ERR_CUDA: CUDA runtime error";
+        case NF4_ERR_DEVICE_TIMEOUT: return "NF4_ERR_DEVICE_TIMEOUT: a bounded device wait ran out";
+        case NF4_ERR_UNSUPPORTED: return "NF4_ERR_UNSUPPORTED: device is not compute capability 10.x";
+        default: return "unknown nf4 status";
+    }
+}
+
+nf4_status_t nf4_codebook(float* levels_out) {
+    if (!levels_out) return NF4_ERR_NULL;
+    static const float levels[16] = NF4_LEVELS_INIT;
+    std::memcpy(levels_out, levels, sizeof levels);
+    return NF4_OK;
+}
+
+nf4_status_t nf4_quantize(const void* W, nf4_dtype_t w_dtype, int64_t n, int64_t k, uint8_t* wq,
+                          float* absmax, nf4_stream_t stream) {
+    if (!W || !wq || !absmax) return NF4_ERR_NULL;
+    if (w_dtype != NF4_F32 && w_dtype != NF4_BF16) return NF4_ERR_DTYPE;
+    if (n <= 0 || k <= 0 || n > INT64_MAX / k || (n * k) % NF4_BLOCKSIZE != 0) return NF4_ERR_SHAPE;
+    if (!aligned(W, 16) || !aligned(wq, 16) || !aligned(absmax, 4)) return NF4_ERR_ALIGN;
+    nf4::DeviceInfo dev;
+    nf4_status_t st = device_ok(&dev);
+    if (st != NF4_OK) return st;
+    return from_cuda(nf4::launch_quantize(W, w_dtype == NF4_BF16, n * k, wq, absmax, dev,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t nf4_double_quant_workspace_bytes(int64_t nb) { return nf4::dq_workspace_bytes(nb); }
+
+nf4_status_t nf4_double_quant(const float* absmax, int64_t nb, void* workspace,
+                              size_t workspace_bytes, int8_t* absmax_q, float* absmax_scale,
+                              float* absmax_offset, nf4_stream_t stream) {
+    if (!absmax || !absmax_q || !absmax_scale || !absmax_offset) return NF4_ERR_NULL;
+    if (nb <= 0 || nb > nf4::dq_max_nb()) return NF4_ERR_SHAPE;
+    if (!workspace || workspace_bytes < nf4::dq_workspace_bytes(nb)) return NF4_ERR_WORKSPACE;
+    if (!aligned(absmax, 4) || !aligned(absmax_scale, 4) || !aligned(absmax_offset, 4) ||
+        !aligned(workspace, 8))
+        return NF4_ERR_ALIGN;
+    nf4::DeviceInfo dev;
+    nf4_status_t st = device_ok(&dev);
+    if (st != NF4_OK) return st;
+    return from_cuda(nf4::launch_double_quant(absmax, nb, static_cast<double*>(workspace), absmax_q,
+                                              absmax_scale, absmax_offset, dev,
+                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nf4_status_t nf4_dequantize(const nf4_weight_t* w, void* out, nf4_dtype_t out_dtype,
+                            nf4_stream_t stream) {
+    nf4_status_t st = check_weight(w);
+    if (st != NF4_OK) return st;
+    if (!out) return NF4_ERR_NULL;
+    if (out_dtype != NF4_F32 && out_dtype != NF4_BF16) return NF4_ERR_DTYPE;
+    if (!aligned(out, 16)) return NF4_ERR_ALIGN;
+    nf4::DeviceInfo dev;
+    if ((st = device_ok(&dev)) != NF4_OK) return st;
+    return from_cuda(nf4::launch_dequantize(w->wq, w->absmax_q, w->absmax_scale, w->absmax_offset,
+                                            w->n * w->k, out, out_dtype == NF4_BF16, dev,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nf4_status_t nf4_linear(const void* X, int64_t m, const nf4_weight_t* w, void* Y,
+                        nf4_dtype_t y_dtype, int32_t* dev_status, nf4_stream_t stream) {
+    nf4_status_t st = check_weight(w);
+    if (st != NF4_OK) return st;
+    if (!X || !Y) return NF4_ERR_NULL;
+    if (y_dtype != NF4_F32 && y_dtype != NF4_BF16) return NF4_ERR_DTYPE;
+    if (m < 1 || w->k % NF4_BLOCKSIZE != 0) return NF4_ERR_SHAPE;
+    if (m > INT64_MAX / w->k || m > INT64_MAX / w->n) return NF4_ERR_SHAPE;
+    if (!aligned(X, 16) || !aligned(Y, 16) || (dev_status && !aligned(dev_status, 4)))
+        return NF4_ERR_ALIGN;
+    nf4::DeviceInfo dev;
+    if ((st = device_ok(&dev)) != NF4_OK) return st;
+    return from_cuda(nf4::launch_linear(X, m, w->wq, w->absmax_q, w->absmax_scale, w->absmax_offset,
+                                        w->n, w->k, Y, y_dtype == NF4_BF16, dev_status, dev,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,73 @@
+// nf4_dequant.cu -- NF4 + double-quantization state back to fp32 / bf16 (sm_100a).
+//
+// Source: page "LLM 相關知識" (technicalnotes, tag qlora), §5 "動態反量化": the 4-bit
+// weights are restored to the compute dtype layer by layer; page "Tim Dettmers
+// 如何用 bitsandbytes 與 QLoRA 降低 LLM 訓練門檻？", section on QLoRA: the frozen 4-bit
+// base is dequantized in forward and backward.
+//
+// HBM-bound: reads 0.5 B/param of codes (+1 B per 64 of absmax codes) and
+// writes 2 (bf16) or 4 (fp32) B/param.  Each lane decodes one 32-bit word of
+// codes (8 elements) with the 16 levels held in shared memory and writes 16 or
+// 32 bytes with 128-bit stores.
+#include "nf4_common.cuh"
+#include "nf4_internal.h"
+
+namespace nf4 {
+
+template <bool kBf16Out>
+__global__ void __launch_bounds__(256) k_nf4_dequantize(const uint32_t* __restrict__ wq32,
+                                                        const int8_t* __restrict__ absmax_q,
+                                                        const float* __restrict__ absmax_scale,
+                                                        const float* __restrict__ mu_ptr,
+                                                        int64_t n_groups, void* __restrict__ out) {
+    __shared__ float lv[16];
+    if (threadIdx.x < 16) lv[threadIdx.x] = kLevels[threadIdx.x];
+    __syncthreads();
+    const float mu = __ldg(mu_ptr);
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < n_groups;
+         g += stride) {
+        const uint32_t packed = __ldcs(wq32 + g);
+        const int64_t b = g >> 3;  // 64-element block
+        const float a = absmax_hat(__ldg(absmax_q + b), __ldg(absmax_scale + (b >> 8)), mu);
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t byte = (packed >> (8 * i)) & 0xffu;
+            v[2 * i] = __fmul_rn(lv[byte >> 4], a);        // element 2i: high nibble
+            v[2 * i + 1] = __fmul_rn(lv[byte & 15u], a);
+        }
+        if (kBf16Out) {
+            uint4 o;
+            o.x = pack_bf16x2(v[0], v[1]);
+            o.y = pack_bf16x2(v[2], v[3]);
+            o.z = pack_bf16x2(v[4], v[5]);
+            o.w = pack_bf16x2(v[6], v[7]);
+            __stcs(reinterpret_cast<uint4*>(out) + g, o);
+        } else {
+            float4* o = reinterpret_cast<float4*>(out) + 2 * g;
+            __stcs(o, make_float4(v[0], v[1], v[2], v[3]));
+            __stcs(o + 1, make_float4(v[4], v[5], v[6], v[7]));
+        }
+    }
+}
+
+cudaError_t launch_dequantize(const uint8_t* wq, const int8_t* absmax_q, const float* absmax_scale,
+                              const float* absmax_offset, int64_t n_elem, void* out, bool out_bf16,
+                              const DeviceInfo& dev, cudaStream_t stream) {
+    const int64_t n_groups = n_elem / 8;
+    int64_t blocks = (n_groups + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(dev.sm_count) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    const uint32_t* wq32 = reinterpret_cast<const uint32_t*>(wq);
+    if (out_bf16)
+        k_nf4_dequantize<true><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+            wq32, absmax_q, absmax_scale, absmax_offset, n_groups, out);
+    else
+        k_nf4_dequantize<false><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+            wq32, absmax_q, absmax_scale, absmax_offset, n_groups, out);
+    return cudaGetLastError();
+}
+
+}  // namespace nf4

@@ -1,0 +1,41 @@
+// nf4_internal.h -- launchers behind the C ABI (nf4_api.cu validates, these launch).
+// Every launcher enqueues on `stream` and returns the cudaGetLastError() of its
+// launches.  Arguments arrive already validated.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace nf4 {
+
+struct DeviceInfo {
+    int device = -1;
+    int sm_count = 0;
+    int major = 0;
+    int minor = 0;
+    size_t smem_optin = 0;
+};
+
+// Properties of the current device (cached per device).
+cudaError_t current_device(DeviceInfo* out);
+
+cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n_elem, uint8_t* wq, float* absmax,
+                            const DeviceInfo& dev, cudaStream_t stream);
+
+// Maximum number of absmax values double quantization accepts in one call.
+int64_t dq_max_nb();
+size_t dq_workspace_bytes(int64_t nb);
+cudaError_t launch_double_quant(const float* absmax, int64_t nb, double* workspace, int8_t* absmax_q,
+                                float* absmax_scale, float* absmax_offset, const DeviceInfo& dev,
+                                cudaStream_t stream);
+
+cudaError_t launch_dequantize(const uint8_t* wq, const int8_t* absmax_q, const float* absmax_scale,
+                              const float* absmax_offset, int64_t n_elem, void* out, bool out_bf16,
+                              const DeviceInfo& dev, cudaStream_t stream);
+
+cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
+                          const float* absmax_scale, const float* absmax_offset, int64_t n,
+                          int64_t k, void* Y, bool y_bf16, int32_t* dev_status,
+                          const DeviceInfo& dev, cudaStream_t stream);
+
+}  // namespace nf4

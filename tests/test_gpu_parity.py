@@ -1,0 +1,270 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle on the
+same seeded inputs.
+
+Bar: packed codes, absmax, double-quantized absmax codes and scales, the mean
+and the dequantized weights (fp32 and bf16) bit-exact; the fused linear within
+a relative Frobenius error of 2e-3 (fp32 output) against an fp64 GEMM on the
+bf16-dequantized weight.  Full-size configurations are checked on whole arrays
+for quantization / double quantization and on sampled rows for dequantization
+and the linear."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from quantized_linear_layers_nf4_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+LINEAR_TOL = 2e-3
+
+
+@pytest.fixture(scope="module")
+def nf4():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from quantized_linear_layers_nf4_b200.build import build
+    build()
+    import quantized_linear_layers_nf4_b200 as m
+    return m
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    """Host copy of a tensor for the oracle: fp32 as float32, bf16 as uint16 bits."""
+    t = t.detach().contiguous().cpu()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16).reshape(-1)
+    return t.numpy().reshape(-1)
+
+
+def _gpu_chain(nf4, W):
+    wq, absmax = nf4.nf4_quantize(W)
+    q, s, mu = nf4.nf4_double_quant(absmax)
+    weight = nf4.NF4Weight(W.shape[0], W.shape[1], wq, q, s, mu)
+    return weight, absmax
+
+
+def _oracle_chain(Wh):
+    wq, absmax = O.quantize(Wh)
+    q, s, mu = O.double_quant(absmax)
+    return wq, absmax, q, s, mu
+
+
+def _assert_equal(gpu: torch.Tensor, ref: np.ndarray, what: str):
+    g = gpu.detach().cpu().numpy().reshape(-1)
+    ref = np.asarray(ref).reshape(-1)
+    assert g.shape == ref.shape, (what, g.shape, ref.shape)
+    if g.dtype == np.float32:
+        g, ref = g.view(np.uint32), ref.astype(np.float32).view(np.uint32)
+    bad = np.flatnonzero(g != ref)
+    assert bad.size == 0, "%s: %d mismatches, first at %s: gpu %s oracle %s" % (
+        what, bad.size, bad[:5], g[bad[:5]], ref[bad[:5]])
+
+
+def _check_quant(nf4, W, full_dequant=True, rows=None):
+    """Quantize + double-quant + dequant on the GPU and compare with the oracle.
+    Returns (weight, oracle arrays) for further checks."""
+    weight, absmax = _gpu_chain(nf4, W)
+    n, k = W.shape
+    Wh = _bits(W)
+    owq, oam, oq, os_, omu = _oracle_chain(Wh)
+    _assert_equal(absmax, oam, "absmax")
+    _assert_equal(weight.wq, owq, "packed codes")
+    _assert_equal(weight.absmax_q, oq, "absmax_q")
+    _assert_equal(weight.absmax_scale, os_, "absmax_scale")
+    _assert_equal(weight.absmax_offset, np.array([omu], np.float32), "absmax_offset (mean)")
+    if full_dequant:
+        d32 = nf4.nf4_dequantize(weight, torch.float32)
+        d16 = nf4.nf4_dequantize(weight, torch.bfloat16)
+        ref = O.dequantize(owq, oq, os_, omu)
+        _assert_equal(d32, ref, "dequant fp32")
+        _assert_equal(d16.view(torch.int16).view(-1), O.f32_to_bf16(ref).view(np.int16), "dequant bf16")
+    else:
+        d32 = nf4.nf4_dequantize(weight, torch.float32)
+        d16 = nf4.nf4_dequantize(weight, torch.bfloat16)
+        for r in rows:
+            ref = O.dequantize_range(owq, oq, os_, omu, r * k, k)
+            _assert_equal(d32[r], ref, "dequant fp32 row %d" % r)
+            _assert_equal(d16[r].view(torch.int16), O.f32_to_bf16(ref).view(np.int16),
+                          "dequant bf16 row %d" % r)
+        del d32, d16
+    return weight, (owq, oq, os_, omu)
+
+
+def _rel_fro(y: np.ndarray, ref: np.ndarray) -> float:
+    return float(np.linalg.norm(y.astype(np.float64) - ref) / max(np.linalg.norm(ref), 1e-300))
+
+
+def _check_linear(nf4, X, weight, orc, token_rows=None, weight_rows=None, tol=LINEAR_TOL):
+    """nf4_linear vs the oracle's fp64 GEMM on the bf16-dequantized weight, on
+    the sampled token rows x weight rows.  Returns the fp32 relative error."""
+    owq, oq, os_, omu = orc
+    m, k = X.shape
+    n = weight.n
+    T = np.arange(m) if token_rows is None else np.asarray(token_rows)
+    R = np.arange(n) if weight_rows is None else np.asarray(weight_rows)
+    Y32 = nf4.nf4_linear(X, weight, torch.float32)
+    Y16 = nf4.nf4_linear(X, weight, torch.bfloat16)
+    torch.cuda.synchronize()
+    wrows = np.stack([O.f32_to_bf16(O.dequantize_range(owq, oq, os_, omu, int(r) * k, k)) for r in R])
+    xb = _bits(X).reshape(m, k)[T]
+    ref = O.linear_bf16(np.ascontiguousarray(xb), np.ascontiguousarray(wrows))
+    y32 = Y32.cpu().numpy()[np.ix_(T, R)]
+    e32 = _rel_fro(y32, ref)
+    assert e32 <= tol, "linear fp32 rel-Frobenius %.3g > %.3g" % (e32, tol)
+    # the bf16 output is the fp32 result of the same kernel rounded once
+    y16 = Y16.float().cpu().numpy()[np.ix_(T, R)]
+    y32r = torch.from_numpy(np.ascontiguousarray(y32)).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(y16, y32r), "bf16 output is not the rounded fp32 output"
+    e16 = _rel_fro(y16, ref)
+    assert e16 <= 2 * tol, "linear bf16 rel-Frobenius %.3g" % e16
+    return e32
+
+
+# ---------------------------------------------------------------------------
+# Small cases: several tiles and ragged tails, both input dtypes.
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("n,k", [(1, 64), (3, 640), (5, 192), (64, 4096), (257, 320), (100, 6400),
+                                 (2, 32)])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_quantize_chain_small(nf4, n, k, dtype):
+    W = synth.weight_normal(n, k, seed=n * 7 + k, std=0.02, dtype=dtype, device="cuda")
+    _check_quant(nf4, W)
+
+
+def test_edge_values(nf4):
+    n, k = 8, 512
+    W = synth.weight_normal(n, k, seed=77, std=0.02, dtype=torch.float32, device="cuda")
+    W[0, 0:64] = 0.0                                 # zero block
+    W[0, 64:128] = -0.0                              # negative-zero block
+    W[1, 0:64] = 0.0
+    W[1, 5] = -3.5                                   # single non-zero
+    W[2, 0:64] = 0.25                                # constant block
+    W[2, 64:128] = 1e-40                             # subnormals
+    W[2, 130] = -1e-39
+    W[3, 0:64] = torch.linspace(-1e30, 1e30, 64)     # huge values
+    W[4, :] = 0.0                                    # a zero row (zero absmax, mean shifts)
+    lv = torch.from_numpy(O.codebook()).cuda()
+    W[5, 0:16] = lv                                  # exact levels, absmax 1
+    W[5, 16:31] = (lv[:-1] + lv[1:]) / 2             # fp32-rounded midpoints
+    W[6, 0:64] = torch.arange(64, dtype=torch.float32, device="cuda") - 31.5
+    _check_quant(nf4, W)
+
+
+def test_cfg1_full_chain_and_linear(nf4):
+    """1024 x 1024 fp32 weight (seed 0), X 16 x 1024 bf16 (seed 1): everything
+    checked on the whole output."""
+    W = synth.weight_normal(1024, 1024, seed=0, std=0.02, dtype=torch.float32, device="cuda")
+    X = synth.activations(16, 1024, seed=1, device="cuda")
+    weight, orc = _check_quant(nf4, W)
+    _check_linear(nf4, X, weight, orc)
+
+
+@pytest.mark.parametrize("m", [1, 2, 4, 7, 8, 15, 16, 17, 33, 64])
+def test_linear_token_counts(nf4, m):
+    n, k = 200, 576
+    W = synth.weight_normal(n, k, seed=300 + m, dtype=torch.bfloat16, device="cuda")
+    X = synth.activations(m, k, seed=400 + m, device="cuda")
+    weight, orc = _check_quant(nf4, W)
+    _check_linear(nf4, X, weight, orc)
+
+
+@pytest.mark.parametrize("n,k", [(8, 64), (1, 128), (9, 64), (24, 1088), (1000, 256)])
+def test_linear_ragged_shapes(nf4, n, k):
+    W = synth.weight_normal(n, k, seed=500 + n, dtype=torch.bfloat16, device="cuda")
+    X = synth.activations(5, k, seed=600 + n, device="cuda")
+    weight, orc = _check_quant(nf4, W)
+    _check_linear(nf4, X, weight, orc)
+
+
+def test_deterministic_and_stream_aware(nf4):
+    W = synth.weight_normal(512, 1024, seed=9, dtype=torch.bfloat16, device="cuda")
+    X = synth.activations(16, 1024, seed=10, device="cuda")
+    a, _ = _gpu_chain(nf4, W)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        b, _ = _gpu_chain(nf4, W)
+        yb = nf4.nf4_linear(X, b, torch.float32)
+    s.synchronize()
+    ya = nf4.nf4_linear(X, a, torch.float32)
+    torch.cuda.synchronize()
+    for name in ("wq", "absmax_q", "absmax_scale", "absmax_offset"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name
+    assert torch.equal(ya, yb)
+
+
+def test_dev_status_stays_clear(nf4):
+    W = synth.weight_normal(256, 512, seed=11, dtype=torch.bfloat16, device="cuda")
+    X = synth.activations(3, 512, seed=12, device="cuda")
+    weight, _ = _gpu_chain(nf4, W)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nf4.nf4_linear(X, weight, torch.float32, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+
+
+def test_errors_on_gpu(nf4):
+    W = torch.zeros(3, 7, device="cuda")
+    with pytest.raises(nf4.NF4Error):
+        nf4.nf4_quantize(W)
+    with pytest.raises(ValueError):
+        nf4.nf4_quantize(torch.zeros(4, 64))          # host tensor
+    W = synth.weight_normal(64, 96, seed=1, dtype=torch.bfloat16, device="cuda")
+    weight, _ = _gpu_chain(nf4, W)                    # 64*96 is a multiple of 64
+    X = synth.activations(2, 96, seed=2, device="cuda")
+    with pytest.raises(nf4.NF4Error):                 # but k = 96 is not, for the linear
+        nf4.nf4_linear(X, weight)
+
+
+# ---------------------------------------------------------------------------
+# Full-size configurations (the shapes the benchmark runs): whole arrays for
+# quantization and double quantization, sampled rows for dequant and linear.
+# ---------------------------------------------------------------------------
+
+def _sample_rows(n, count, seed):
+    rng = np.random.default_rng(seed)
+    rows = set([0, n - 1, n // 2]) | set(rng.choice(n, size=min(count, n), replace=False).tolist())
+    return np.array(sorted(rows))
+
+
+@pytest.mark.parametrize("n,k", [(4096, 4096), (11008, 4096), (4096, 11008)])
+def test_cfg2_decode_shapes(nf4, n, k):
+    W = synth.weight_normal(n, k, seed=synth.seed_for(2, n // 64 + k // 64), dtype=torch.bfloat16,
+                            device="cuda")
+    rows = _sample_rows(n, 48, n + k)
+    weight, orc = _check_quant(nf4, W, full_dequant=False, rows=rows)
+    for m in (1, 4, 16):
+        X = synth.activations(m, k, seed=synth.seed_for(2, 100 + m), device="cuda")
+        _check_linear(nf4, X, weight, orc, weight_rows=_sample_rows(n, 192, m))
+
+
+def test_cfg3_prefill_gemm(nf4):
+    m, k, n = 4096, 4096, 11008
+    W = synth.weight_normal(n, k, seed=synth.seed_for(3, 0), dtype=torch.bfloat16, device="cuda")
+    X = synth.activations(m, k, seed=synth.seed_for(3, 1), device="cuda")
+    weight, orc = _check_quant(nf4, W, full_dequant=False, rows=_sample_rows(n, 16, 3))
+    _check_linear(nf4, X, weight, orc, token_rows=_sample_rows(m, 48, 31),
+                  weight_rows=_sample_rows(n, 160, 32))
+
+
+def test_cfg4_layer_stack_sample(nf4):
+    """Two decoder layers of the 7B-shaped stack (14 of the 224 tensors), each
+    checked on whole arrays."""
+    stack = synth.llama7b_stack()
+    for idx in (0, 1, 2, 3, 4, 5, 6, 7 * 31 + 4, 7 * 31 + 6):
+        _, name, n, k = stack[idx]
+        W = synth.weight_normal(n, k, seed=synth.seed_for(4, idx), dtype=torch.bfloat16, device="cuda")
+        _check_quant(nf4, W, full_dequant=False, rows=_sample_rows(n, 8, idx))
+
+
+def test_cfg5_heavy_tailed_stress_layer(nf4):
+    n, k = 28672, 8192
+    W = synth.weight_student_t(n, k, seed=synth.seed_for(5, 0), device="cuda")
+    rows = _sample_rows(n, 24, 5)
+    weight, orc = _check_quant(nf4, W, full_dequant=False, rows=rows)
+    del W
+    for m in (1, 16, 512, 4096):
+        X = synth.activations(m, k, seed=synth.seed_for(5, m), device="cuda")
+        T = None if m <= 16 else _sample_rows(m, 24, m)
+        _check_linear(nf4, X, weight, orc, token_rows=T, weight_rows=_sample_rows(n, 96, m + 1))
