@@ -146,6 +146,33 @@ nf4_status_t nf4_double_quant(const float* absmax, int64_t nb, void* workspace,
                               size_t workspace_bytes, int8_t* absmax_q, float* absmax_scale,
                               float* absmax_offset, nf4_stream_t stream);
 
+/* Largest nb that nf4_double_quant_noalloc accepts: 65536 blocks of 256 absmax
+ * values, i.e. weights of up to 2^30 elements per call. */
+#define NF4_DQ_NOALLOC_MAX_NB 16777216
+
+/*
+ * nf4_double_quant_noalloc -- the same double quantization as nf4_double_quant,
+ * with identical outputs, but without a workspace argument and without
+ * allocating anything.  The pages have no counterpart to this entry point; it
+ * exists for callers that cannot allocate device memory: a plugin or custom op
+ * inside a host framework that owns all device memory and gives it no
+ * allocator, or a deployment whose memory plan is fixed at start-up.
+ *   Scratch: a fixed array of NF4_DQ_NOALLOC_MAX_NB / 256 doubles (512 KiB) in
+ *   device memory, held by every GPU that loads the library until the process
+ *   exits.  The first call on a device (with that device current) looks up the
+ *   array's device address; make that first call before any stream capture.
+ *   Every call on a device shares the array, so calls that overlap on the GPU
+ *   (different streams or host threads) race and must be ordered by the
+ *   caller.  No part of the array needs to start at zero.
+ *   absmax, absmax_q, absmax_scale, absmax_offset: as for nf4_double_quant.
+ * Errors: NF4_ERR_NULL, NF4_ERR_SHAPE (nb <= 0), NF4_ERR_WORKSPACE (nb >
+ * NF4_DQ_NOALLOC_MAX_NB: the request does not fit the fixed scratch),
+ * NF4_ERR_ALIGN, NF4_ERR_UNSUPPORTED, NF4_ERR_CUDA.
+ */
+nf4_status_t nf4_double_quant_noalloc(const float* absmax, int64_t nb, int8_t* absmax_q,
+                                      float* absmax_scale, float* absmax_offset,
+                                      nf4_stream_t stream);
+
 /*
  * nf4_dequantize -- NF4 + double-quantization state back to real values ([P4]
  * §5 "動態反量化": restore the 4-bit weights to the compute dtype; [P1] the frozen
