@@ -212,6 +212,25 @@ nf4_status_t nf4_dequantize(const nf4_weight_t* w, void* out, nf4_dtype_t out_dt
 nf4_status_t nf4_linear(const void* X, int64_t m, const nf4_weight_t* w, void* Y,
                         nf4_dtype_t y_dtype, int32_t* dev_status, nf4_stream_t stream);
 
+/* Flag for nf4_linear_ex: the weight and its quantization state were NOT written
+ * by the work enqueued immediately before this call on the stream (the usual
+ * case at inference time, when weights are quantized once at load time).  The
+ * kernel is then launched as a programmatic dependent launch: it may start
+ * loading the weight while the preceding kernel is still running, and reads X
+ * and writes Y only after that kernel has completed. */
+#define NF4_LINEAR_WEIGHTS_EARLY 1u
+
+/*
+ * nf4_linear_ex -- nf4_linear with launch flags (0 or NF4_LINEAR_WEIGHTS_EARLY);
+ * same arithmetic and results.  Arguments and errors as for nf4_linear, plus
+ * NF4_ERR_DTYPE for an unknown flag bit.  Same source passages as nf4_linear;
+ * the overlap of consecutive layers follows the per-layer dequantize-then-
+ * multiply loop of [P4] §5, where layer N+1's weights do not depend on layer N.
+ */
+nf4_status_t nf4_linear_ex(const void* X, int64_t m, const nf4_weight_t* w, void* Y,
+                           nf4_dtype_t y_dtype, int32_t* dev_status, uint32_t flags,
+                           nf4_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -23,7 +23,7 @@ from . import _lib
 from ._lib import NF4_BF16, NF4_F32, NF4Error, nf4_weight_t
 
 __all__ = ["NF4Weight", "NF4Error", "nf4_quantize", "nf4_double_quant", "nf4_dequantize",
-           "nf4_linear", "quantize_weight", "nf4_codebook", "library_path"]
+           "nf4_linear", "nf4_linear_ex", "quantize_weight", "nf4_codebook", "library_path"]
 
 _DTYPES = {torch.float32: NF4_F32, torch.bfloat16: NF4_BF16}
 
@@ -135,10 +135,21 @@ def nf4_dequantize(weight: NF4Weight, dtype=torch.bfloat16, out: torch.Tensor | 
     return out
 
 
+def nf4_linear_ex(X, weight, dtype=torch.bfloat16, out=None, dev_status=None, stream=None,
+                  flags: int = 0):
+    """Same as nf4_linear with the C flags word (0 or NF4_LINEAR_WEIGHTS_EARLY)."""
+    return nf4_linear(X, weight, dtype, out, dev_status, stream,
+                      weights_early=bool(flags & _lib.NF4_LINEAR_WEIGHTS_EARLY))
+
+
 def nf4_linear(X: torch.Tensor, weight: NF4Weight, dtype=torch.bfloat16,
                out: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
-               stream=None) -> torch.Tensor:
-    """Y = X @ W_hat^T for bf16 X [m, k]; Y [m, n] in ``dtype`` (bf16 or fp32)."""
+               stream=None, weights_early: bool = False) -> torch.Tensor:
+    """Y = X @ W_hat^T for bf16 X [m, k]; Y [m, n] in ``dtype`` (bf16 or fp32).
+
+    ``weights_early=True`` calls ``nf4_linear_ex`` with NF4_LINEAR_WEIGHTS_EARLY:
+    the weight was not written by the work just before this call on the stream,
+    so its loads may overlap that work (programmatic dependent launch)."""
     _need_cuda(X, "X")
     if X.dtype != torch.bfloat16 or X.dim() != 2:
         raise ValueError("X must be a 2-D bfloat16 tensor")
@@ -149,6 +160,7 @@ def nf4_linear(X: torch.Tensor, weight: NF4Weight, dtype=torch.bfloat16,
         out = torch.empty((m, weight.n), dtype=dtype, device=X.device)
     st = weight.struct()
     ds = ctypes.c_void_p(0) if dev_status is None else _ptr(dev_status)
-    _lib.check(_lib.lib().nf4_linear(_ptr(X), m, ctypes.byref(st), _ptr(out), _DTYPES[dtype], ds,
-                                     _stream(stream)), "nf4_linear")
+    flags = _lib.NF4_LINEAR_WEIGHTS_EARLY if weights_early else 0
+    _lib.check(_lib.lib().nf4_linear_ex(_ptr(X), m, ctypes.byref(st), _ptr(out), _DTYPES[dtype], ds,
+                                        flags, _stream(stream)), "nf4_linear_ex")
     return out

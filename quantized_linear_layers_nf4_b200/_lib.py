@@ -20,6 +20,7 @@ NF4_WEIGHT_MAGIC = 0x4E463442
 NF4_WEIGHT_VERSION = 1
 NF4_ABI_VERSION = 1
 NF4_DQ_NOALLOC_MAX_NB = 16777216
+NF4_LINEAR_WEIGHTS_EARLY = 1
 
 # Every function include/nf4.h declares, with (restype, argtypes).
 _p = ctypes.c_void_p
@@ -44,6 +45,8 @@ SIGNATURES = {
     "nf4_double_quant_noalloc": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p]),
     "nf4_dequantize": (ctypes.c_int, [ctypes.POINTER(nf4_weight_t), _p, ctypes.c_int, _p]),
     "nf4_linear": (ctypes.c_int, [_p, _i64, ctypes.POINTER(nf4_weight_t), _p, ctypes.c_int, _p, _p]),
+    "nf4_linear_ex": (ctypes.c_int, [_p, _i64, ctypes.POINTER(nf4_weight_t), _p, ctypes.c_int, _p,
+                                     ctypes.c_uint32, _p]),
 }
 
 

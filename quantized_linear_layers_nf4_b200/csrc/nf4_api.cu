@@ -143,12 +143,13 @@ nf4_status_t nf4_dequantize(const nf4_weight_t* w, void* out, nf4_dtype_t out_dt
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
-nf4_status_t nf4_linear(const void* X, int64_t m, const nf4_weight_t* w, void* Y,
-                        nf4_dtype_t y_dtype, int32_t* dev_status, nf4_stream_t stream) {
+nf4_status_t nf4_linear_ex(const void* X, int64_t m, const nf4_weight_t* w, void* Y,
+                           nf4_dtype_t y_dtype, int32_t* dev_status, uint32_t flags, nf4_stream_t stream) {
     nf4_status_t st = check_weight(w);
     if (st != NF4_OK) return st;
     if (!X || !Y) return NF4_ERR_NULL;
     if (y_dtype != NF4_F32 && y_dtype != NF4_BF16) return NF4_ERR_DTYPE;
+    if ((flags & ~static_cast<uint32_t>(NF4_LINEAR_WEIGHTS_EARLY)) != 0) return NF4_ERR_DTYPE;
     if (m < 1 || w->k % NF4_BLOCKSIZE != 0) return NF4_ERR_SHAPE;
     if (m > INT64_MAX / w->k || m > INT64_MAX / w->n) return NF4_ERR_SHAPE;
     if (!aligned(X, 16) || !aligned(Y, 16) || (dev_status && !aligned(dev_status, 4)))
@@ -156,8 +157,14 @@ nf4_status_t nf4_linear(const void* X, int64_t m, const nf4_weight_t* w, void* Y
     nf4::DeviceInfo dev;
     if ((st = device_ok(&dev)) != NF4_OK) return st;
     return from_cuda(nf4::launch_linear(X, m, w->wq, w->absmax_q, w->absmax_scale, w->absmax_offset,
-                                        w->n, w->k, Y, y_dtype == NF4_BF16, dev_status, dev,
+                                        w->n, w->k, Y, y_dtype == NF4_BF16, dev_status,
+                                        (flags & NF4_LINEAR_WEIGHTS_EARLY) != 0, dev,
                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nf4_status_t nf4_linear(const void* X, int64_t m, const nf4_weight_t* w, void* Y,
+                        nf4_dtype_t y_dtype, int32_t* dev_status, nf4_stream_t stream) {
+    return nf4_linear_ex(X, m, w, Y, y_dtype, dev_status, 0u, stream);
 }
 
 }  // extern "C"

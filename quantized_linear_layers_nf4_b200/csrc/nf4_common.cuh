@@ -58,10 +58,23 @@ __device__ __forceinline__ int quantize_one(float w, float a) {
     return encode_nf4(__fdiv_rn(w, a));
 }
 
+// fp32(q / 127), the correctly rounded quotient, for an int8 code q, without a
+// division: one multiply by the rounded reciprocal and one residual
+// correction (Markstein's method, IBM J. Res. Dev. 34(1), 1990): with
+// r = q * RN(1/127) and e = q - 127 r (exact by FMA), r + e * RN(1/127) rounds
+// to the IEEE quotient.  Checked exhaustively for all 256 codes (exact rational
+// arithmetic, tests/test_div127.py) and bit-for-bit by every dequant parity test.
+__device__ __forceinline__ float div127(float q) {
+    constexpr float kInv = 1.0f / 127.0f;  // RN(1/127)
+    const float r = __fmul_rn(q, kInv);
+    const float e = __fmaf_rn(-r, 127.0f, q);
+    return __fmaf_rn(e, kInv, r);
+}
+
 // Reconstructed absmax from its double-quantized code:
 // a = fp32(fp32(fp32(q / 127) * s) + mu).
 __device__ __forceinline__ float absmax_hat(int q, float s, float mu) {
-    return __fadd_rn(__fmul_rn(__fdiv_rn(static_cast<float>(q), 127.0f), s), mu);
+    return __fadd_rn(__fmul_rn(div127(static_cast<float>(q)), s), mu);
 }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t h16) {

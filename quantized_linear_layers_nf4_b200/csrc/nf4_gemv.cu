@@ -7,137 +7,486 @@
 // 取決於硬體與 kernel，不只位元數" (unfused 4-bit can lose to fp16; batch size moves the
 // work between memory- and compute-bound).
 //
-// Y[t, r] = sum_c X[t, c] * What[r, c],  What[r, c] = bf16(fp32(level[idx] * a_block)).
+//   Y[t, r] = sum_c X[t, c] * What[r, c],   What[r, c] = bf16(fp32(level[idx] * a_block)).
 //
-// The multiply-adds run on the tensor cores (mma.sync m16n8k16, bf16 in, fp32
-// accumulate) with the tokens as the MMA's M side (zero-padded to 16) and eight
-// weight rows as its N side, so the CUDA cores only decode.  The k order inside
-// each MMA is a permutation of the true k order (each lane takes 32 consecutive
-// weights of one row), applied identically to X and the weights, so the dot
-// products are unchanged.  Decode: one 256-entry table maps a packed byte to
-// the two fp32 levels it encodes; each level is multiplied by the block's
-// reconstructed absmax in fp32 and rounded to bf16, exactly as nf4_dequantize
-// does.
+// The operation is HBM-bound: per weight 0.5 B of codes plus 1/64 B of absmax
+// code must stream from HBM.  Design (one CTA = 128 weight rows x a slice of k):
+//
+// * A producer warp streams 256-wide k stages through a 3-deep shared-memory
+//   ring with TMA (no multicast): a [128 rows x 128 B] tile of packed codes and
+//   the matching [16 tokens x 256] tile of X, both 128-byte swizzled so the
+//   consumers' reads are bank-conflict free.  Its 32 lanes also reconstruct the
+//   stage's absmax values (loaded one stage ahead, so their latency hides behind
+//   the ring).  mbarriers carry full/empty state; every wait is bounded.
+// * Eight consumer warps: warp w owns 64-block (w % 4) of every stage for 64
+//   of the 128 rows, so one X fragment serves 8 MMAs.  The multiply-adds run on the tensor
+//   cores (mma.sync m16n8k16, bf16 in, fp32 accumulate) with the 16 token slots
+//   as the MMA's M side (zero-filled beyond m) and 8 weight rows as its N side.
+//   Each lane owns 16 consecutive weights of a block row; the MMA k order is a
+//   permutation of the true k order applied identically to X and the weights.
+// * Decode: a 256-entry table maps a packed byte to the two fp32 levels it
+//   encodes (replicated 16x so a half-warp's lookups never share a bank); each
+//   level is multiplied by the block's reconstructed absmax in fp32 and rounded
+//   to bf16 -- the same values nf4_dequantize produces.
+// * Split-k: the CTAs of a thread-block cluster share a row tile and split k;
+//   their fp32 partials are added through distributed shared memory in a fixed
+//   rank order, so results are deterministic and no global scratch is needed.
 #include "nf4_common.cuh"
 #include "nf4_internal.h"
+#include "nf4_ptx.cuh"
+#include "nf4_tmap.h"
 
 namespace nf4 {
+namespace gemv {
 
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+constexpr int kRows = 128;                       // weight rows per CTA
+constexpr int kStageK = 256;                     // k per pipeline stage
+constexpr int kRing = 3;                         // stages in flight per CTA
+constexpr int kConsumers = 8;                    // consumer warps
+constexpr int kTiles = 8;                        // 8-row MMA tiles per consumer warp (64 rows)
+constexpr int kThreads = 32 * (kConsumers + 1);  // + one producer warp
+constexpr int kWBytes = kRows * kStageK / 2;     // 16384: packed codes of a stage
+constexpr int kXBox = 16 * 64 * 2;               // 2048: X box of 16 tokens x 64 k (bf16)
+constexpr int kXBytes = 4 * kXBox;               // 8192
+constexpr int kTmaBytes = kWBytes + kXBytes;     // bytes a stage receives by TMA
+constexpr int kAhatBytes = 4 * kRows * 4;        // 2048: reconstructed absmax, [row][block]
+constexpr int kStageBytes = kTmaBytes + kAhatBytes;  // 26624 = 26 KiB (keeps 1 KiB alignment)
+constexpr int kLutBytes = 16 * 256 * 8;          // 32768
+constexpr int kRingBytes = kRing * kStageBytes;
+constexpr int kSmemBytes = 1024 /*alignment slack*/ + kRingBytes + kLutBytes + 2 * kRing * 8;
+static_assert(kStageBytes % 1024 == 0, "stages keep the 1 KiB alignment the 128-byte swizzle needs");
+static_assert(4 * 16 * kRows * 4 + 16 * kRows * 4 <= kRingBytes, "reduction fits in the ring");
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
     asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};\n"
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ void load_x32(const __nv_bfloat16* __restrict__ row, int64_t c0, bool ok,
-                                         uint32_t (&w)[16]) {
-    if (ok) {
-        const uint4* p = reinterpret_cast<const uint4*>(row + c0);
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint64_t lds_b64(uint32_t addr) {
+    uint64_t v;
+    asm volatile("ld.shared.b64 %0, [%1];" : "=l"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint64_t dup_f32x2(float a) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(a));
+    return r;
+}
+
+// Two levels (one packed byte) times the block's absmax, each product rounded
+// to fp32 (one packed f32x2 multiply), then both rounded to bf16: the high
+// nibble (lower k) lands in the low half.
+__device__ __forceinline__ uint32_t scale_pack(uint64_t levels, uint64_t aa) {
+    uint32_t out;
+    asm("{\n\t.reg .b64 r;\n\t.reg .f32 lo, hi;\n\t"
+        "mul.rn.f32x2 r, %1, %2;\n\t"
+        "mov.b64 {lo, hi}, r;\n\t"
+        "cvt.rn.bf16x2.f32 %0, hi, lo;\n\t}"
+        : "=r"(out)
+        : "l"(levels), "l"(aa));
+    return out;
+}
+
+// The producer's per-stage absmax inputs.  Lane l owns rows l + 32 u (u = 0..3)
+// and the stage's 4 blocks of each: the 4 int8 codes of a row packed in one
+// word, and the (at most two) double-quantization scales its 4 blocks use.
+struct AbsmaxIn {
+    uint32_t q[4];
+    float s_lo[4], s_hi[4];
+};
+
+__device__ __forceinline__ void load_absmax_in(AbsmaxIn& a, const int8_t* __restrict__ absmax_q,
+                                               const float* __restrict__ absmax_scale, int64_t row0,
+                                               int lane, int st, int64_t n, int64_t kblocks,
+                                               bool aligned4) {
+    const int64_t kb0 = static_cast<int64_t>(st) * 4;
+    if (aligned4) {
+        // k % 256 == 0 and an aligned code array: a row's 4 codes of a stage are
+        // one aligned word.  Every load is unconditional (rows past n are
+        // clamped; their results are never stored) and lands directly in its
+        // field, so nothing waits for it until the stage is used.
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint4 v = __ldg(p + q);
-            w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+        for (int u = 0; u < 4; ++u) {
+            int64_t grow = row0 + lane + 32 * u;
+            grow = grow < n ? grow : n - 1;
+            const int64_t b0 = grow * kblocks + kb0;
+            a.q[u] = __ldg(reinterpret_cast<const uint32_t*>(absmax_q + b0));
+            a.s_lo[u] = __ldg(absmax_scale + (b0 >> 8));
+            a.s_hi[u] = __ldg(absmax_scale + ((b0 + 3) >> 8));
         }
-    } else {
+        return;
+    }
+    // general shapes: gather the codes byte by byte (stalls, but correct)
 #pragma unroll
-        for (int q = 0; q < 16; ++q) w[q] = 0u;
+    for (int u = 0; u < 4; ++u) {
+        const int64_t grow = row0 + lane + 32 * u;
+        uint32_t q = 0;
+        float lo = 0.0f, hi = 0.0f;
+        if (grow < n) {
+            const int64_t b0 = grow * kblocks + kb0;
+            const int64_t nvalid = kblocks - kb0;  // >= 1
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                if (b < nvalid)
+                    q |= static_cast<uint32_t>(static_cast<uint8_t>(__ldg(absmax_q + b0 + b))) << (8 * b);
+            const int64_t blast = b0 + (nvalid < 4 ? nvalid : 4) - 1;
+            lo = __ldg(absmax_scale + (b0 >> 8));
+            hi = __ldg(absmax_scale + (blast >> 8));
+        }
+        a.q[u] = q;
+        a.s_lo[u] = lo;
+        a.s_hi[u] = hi;
     }
 }
 
-// One warp computes an 8-row x 16-token tile of Y^T over all of k.
-// Lane (g = lane / 4, i = lane % 4): weight row r0 + g, tokens g and g + 8,
-// and within each 128-wide span of k the 32 columns [32 i, 32 i + 32).
-template <bool kBf16Out>
-__global__ void __launch_bounds__(128) k_nf4_gemv_simple(
-    const __nv_bfloat16* __restrict__ X, int m, int64_t k, const uint8_t* __restrict__ wq,
-    const int8_t* __restrict__ absmax_q, const float* __restrict__ absmax_scale,
-    const float* __restrict__ mu_ptr, int64_t n, void* __restrict__ Y) {
-    __shared__ float2 lut[256];  // byte -> (level of its high nibble, level of its low nibble)
-    for (int e = threadIdx.x; e < 256; e += blockDim.x)
-        lut[e] = make_float2(kLevels[e >> 4], kLevels[e & 15]);
+// Keeps the compiler from hoisting work that uses `a` above the point where
+// this is called (the values pass through an opaque asm).
+__device__ __forceinline__ void pin(AbsmaxIn& a) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        asm volatile("" : "+r"(a.q[u]), "+f"(a.s_lo[u]), "+f"(a.s_hi[u]));
+}
+
+constexpr int kPrefetch = 3;  // stages of absmax inputs in flight per producer lane
+
+template <bool kBf16Out, bool kM16>
+__global__ void __launch_bounds__(kThreads, 2)
+k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+           const int8_t* __restrict__ absmax_q, const float* __restrict__ absmax_scale,
+           const float* __restrict__ mu_ptr, int m, int64_t n, int64_t k, int cluster, int weights_early,
+           void* __restrict__ Y, int32_t* __restrict__ dev_status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* ring = smem;
+    float2* lut = reinterpret_cast<float2*>(smem + kRingBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRingBytes + kLutBytes);
+    uint64_t* empty = full + kRing;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRows;
+    const int64_t kblocks = k / 64;
+    const int n_stages = static_cast<int>((k + kStageK - 1) / kStageK);
+    const int rank = static_cast<int>(blockIdx.y);
+    const int s0 = static_cast<int>((static_cast<int64_t>(n_stages) * rank) / cluster);
+    const int s1 = static_cast<int>((static_cast<int64_t>(n_stages) * (rank + 1)) / cluster);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kRing; ++s) {
+            mbar_init(&full[s], 2);   // the TMA bytes' arrive + the absmax-ready arrive
+            mbar_init(&empty[s], kConsumers);
+        }
+        fence_mbar_init();
+    }
+    grid_launch_dependents();  // the next kernel on the stream may start its prologue
     __syncthreads();
 
-    const float mu = __ldg(mu_ptr);
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int g = lane >> 2;
-    const int i = lane & 3;
-    const int64_t row0 = (static_cast<int64_t>(blockIdx.x) * 4 + warp) * 8;
-    if (row0 >= n) return;
-    const int64_t row = (row0 + g < n) ? row0 + g : n - 1;  // clamped; its outputs are not stored
-    const uint8_t* wrow = wq + row * (k / 2);
-    const int64_t blk_row = row * (k / 64);
-    const bool tok_lo = g < m;
-    const bool tok_hi = g + 8 < m;
-    const __nv_bfloat16* x_lo = X + static_cast<int64_t>(tok_lo ? g : 0) * k;
-    const __nv_bfloat16* x_hi = X + static_cast<int64_t>(tok_hi ? g + 8 : 0) * k;
+    bool timed_out = false;
+    if (warp == kConsumers) {
+        // ------------------------------ producer ------------------------------
+        if (lane == 0) {
+            prefetch_tensormap(&tm_w);
+            prefetch_tensormap(&tm_x);
+        }
+        if (!weights_early) grid_dependency_wait();
+        const float mu = __ldg(mu_ptr);
+        int last_use[kRing];
+#pragma unroll
+        for (int s = 0; s < kRing; ++s) last_use[s] = -1;
+        bool x_ready = !weights_early;  // X (the previous kernel's output) may be read
+        const int n_pre = (s1 - s0) < kRing ? (s1 - s0) : kRing;
+        const bool aligned4 = (kblocks & 3) == 0 && (reinterpret_cast<uintptr_t>(absmax_q) & 3) == 0;
+        AbsmaxIn pre[kPrefetch];
+#pragma unroll
+        for (int d = 0; d < kPrefetch; ++d)
+            load_absmax_in(pre[d], absmax_q, absmax_scale, row0, lane, min(s0 + d, n_stages - 1), n, kblocks, aligned4);
+        for (int st0 = s0; st0 < s1 && !timed_out; st0 += kPrefetch) {
+#pragma unroll
+            for (int d = 0; d < kPrefetch; ++d) {
+                const int st = st0 + d;
+                if (st >= s1) break;
+                const int j = st - s0;
+                const int slot = j % kRing;
+                const int use = j / kRing;
+                if (j >= kRing && !__all_sync(kFull, mbar_wait(&empty[slot], (use - 1) & 1))) {
+                    timed_out = true;
+                    break;
+                }
+                uint8_t* stage = ring + slot * kStageBytes;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&full[slot], kTmaBytes);
+                    tma_load_2d(stage, &tm_w, st * (kStageK / 2), static_cast<int32_t>(row0), &full[slot]);
+                    if (x_ready) {
+#pragma unroll
+                        for (int b = 0; b < 4; ++b)
+                            tma_load_2d(stage + kWBytes + b * kXBox, &tm_x, st * kStageK + 64 * b, 0, &full[slot]);
+                    }
+                    last_use[slot] = use;
+                }
+                pin(pre[d]);  // the copies above are issued before the absmax work below
+                // reconstructed absmax a = fp32(fp32(fp32(q / 127) * s) + mu) of this stage.
+                // Blocks past k or rows past n get q = s = 0 (a = mu, finite): X is
+                // zero-filled there, so their products vanish.
+                const uint32_t ahat = smem_u32(stage + kTmaBytes);  // [row][block] floats
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int row = lane + 32 * u;
+                    const int64_t b0 = (row0 + row) * kblocks + static_cast<int64_t>(st) * 4;
+                    float a4[4];
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        const float sc = (((b0 + b) >> 8) == (b0 >> 8)) ? pre[d].s_lo[u] : pre[d].s_hi[u];
+                        const float qf = static_cast<float>(static_cast<int8_t>((pre[d].q[u] >> (8 * b)) & 0xffu));
+                        a4[b] = __fadd_rn(__fmul_rn(div127(qf), sc), mu);
+                    }
+                    sts128(ahat + row * 16u, make_uint4(__float_as_uint(a4[0]), __float_as_uint(a4[1]),
+                                                        __float_as_uint(a4[2]), __float_as_uint(a4[3])));
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full[slot]);
+                // (unconditional, clamped to a valid stage, so no select waits on the loads)
+                load_absmax_in(pre[d], absmax_q, absmax_scale, row0, lane, min(st + kPrefetch, n_stages - 1), n,
+                               kblocks, aligned4);
+                if (!x_ready && j + 1 == n_pre) {
+                    // weights of the first stages are in flight; now wait for the
+                    // preceding kernel before touching X
+                    grid_dependency_wait();
+                    x_ready = true;
+                    if (lane == 0)
+                        for (int jj = 0; jj <= j; ++jj) {
+                            uint8_t* stg = ring + (jj % kRing) * kStageBytes;
+#pragma unroll
+                            for (int b = 0; b < 4; ++b)
+                                tma_load_2d(stg + kWBytes + b * kXBox, &tm_x, (s0 + jj) * kStageK + 64 * b, 0,
+                                            &full[jj % kRing]);
+                        }
+                }
+            }
+        }
+        if (!x_ready) grid_dependency_wait();
+        // on a timeout leave no copy in flight: wait (bounded) for every stage issued
+        if (timed_out && lane == 0)
+            for (int s = 0; s < kRing; ++s)
+                if (last_use[s] >= 0) mbar_wait(&full[s], last_use[s] & 1);
+    } else {
+        // ------------------------------ consumers -----------------------------
+        // byte -> (level of high nibble, level of low nibble), 16 copies so that
+        // the 16 lanes of a half-warp always read distinct banks
+        // (consecutive threads write consecutive 16-byte chunks: 2 copies each)
+        for (int c = threadIdx.x; c < kLutBytes / 16; c += 32 * kConsumers) {
+            const int b = c >> 3;
+            const uint32_t hi = __float_as_uint(kLevels[b >> 4]), lo = __float_as_uint(kLevels[b & 15]);
+            sts128(smem_u32(lut) + 16u * c, make_uint4(hi, lo, hi, lo));
+        }
+        named_bar_sync(1, 32 * kConsumers);
 
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const int64_t n_spans = (k + 127) / 128;
-    for (int64_t sp = 0; sp < n_spans; ++sp) {
-        const int64_t c0 = sp * 128 + 32 * i;  // first column of this lane's run
-        const bool ok = c0 < k;                 // k % 64 == 0: a run is all in or all out
-        uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-        float a = 0.0f;
-        if (ok) {
-            raw = __ldcs(reinterpret_cast<const uint4*>(wrow + c0 / 2));
-            const int64_t b = blk_row + c0 / 64;
-            a = absmax_hat(__ldg(absmax_q + b), __ldg(absmax_scale + (b >> 8)), mu);
-        }
-        uint32_t xl[16], xh[16];
-        load_x32(x_lo, c0, ok && tok_lo, xl);
-        load_x32(x_hi, c0, ok && tok_hi, xh);
-        const uint32_t r[4] = {raw.x, raw.y, raw.z, raw.w};
+        const int g = lane >> 2;
+        const int i = lane & 3;
+        const int blk = warp & 3;          // 64-block of the stage
+        const int rbase = (warp >> 2) * 64;  // first of this warp's 64 rows
+        const uint32_t lut_lane = smem_u32(lut) + (lane & 15) * 8u;
+        float acc[kTiles][4];
 #pragma unroll
-        for (int s = 0; s < 8; ++s) {
-            const uint32_t word = r[s >> 1] >> (16 * (s & 1));
-            const float2 p0 = lut[word & 0xffu];           // columns c0+4s, c0+4s+1
-            const float2 p1 = lut[(word >> 8) & 0xffu];    // columns c0+4s+2, c0+4s+3
-            const uint32_t b0 = pack_bf16x2(__fmul_rn(p0.x, a), __fmul_rn(p0.y, a));
-            const uint32_t b1 = pack_bf16x2(__fmul_rn(p1.x, a), __fmul_rn(p1.y, a));
-            mma_bf16_16816(acc, xl[2 * s], xh[2 * s], xl[2 * s + 1], xh[2 * s + 1], b0, b1);
+        for (int t = 0; t < kTiles; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+
+        for (int st = s0; st < s1; ++st) {
+            const int j = st - s0;
+            const int slot = j % kRing;
+            // every lane polls; the warp proceeds only if all of them saw the stage
+            if (!__all_sync(kFull, mbar_wait(&full[slot], (j / kRing) & 1))) {
+                timed_out = true;
+                break;
+            }
+            const uint32_t stage = smem_u32(ring + slot * kStageBytes);
+            // X fragments: tokens g and g + 8, k = 16 i .. 16 i + 15 of this warp's block
+            const uint32_t xb = stage + kWBytes + blk * kXBox;
+            const uint4 xa0 = lds128(xb + g * 128 + (((2 * i) ^ g) << 4));
+            const uint4 xa1 = lds128(xb + g * 128 + (((2 * i + 1) ^ g) << 4));
+            uint4 xc0 = make_uint4(0u, 0u, 0u, 0u), xc1 = xc0;
+            if (kM16) {
+                xc0 = lds128(xb + (g + 8) * 128 + (((2 * i) ^ g) << 4));
+                xc1 = lds128(xb + (g + 8) * 128 + (((2 * i + 1) ^ g) << 4));
+            }
+            const uint32_t xa[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
+            const uint32_t xc[8] = {xc0.x, xc0.y, xc0.z, xc0.w, xc1.x, xc1.y, xc1.z, xc1.w};
+            const uint32_t wb = stage + (rbase + g) * 128 + ((((2 * blk + (i >> 1)) ^ g) << 4) + ((i & 1) << 3));
+            const uint32_t ab = stage + kTmaBytes + ((rbase + g) * 4 + blk) * 4;
+#pragma unroll
+            for (int t = 0; t < kTiles; ++t) {
+                const uint2 raw = lds64(wb + t * 8 * 128);
+                const uint64_t aa = dup_f32x2(lds_f32(ab + 128 * t));
+                uint32_t bw[8];
+#pragma unroll
+                for (int b = 0; b < 8; ++b) {
+                    const uint32_t word = (b < 4) ? raw.x : raw.y;
+                    const uint32_t byte = (word >> (8 * (b & 3))) & 0xffu;
+                    bw[b] = scale_pack(lds_b64(lut_lane + byte * 128u), aa);
+                }
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_16816(acc[t], xa[2 * s], xc[2 * s], xa[2 * s + 1], xc[2 * s + 1], bw[2 * s], bw[2 * s + 1]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
         }
+
+        // fold the consumer warps: red[blk][token][row] (the two row halves of a
+        // block land in disjoint rows of the same buffer)
+        __syncwarp();
+        named_bar_sync(1, 32 * kConsumers);  // every consumer is done with the ring
+        float* red = reinterpret_cast<float*>(ring) + blk * 16 * kRows;
+#pragma unroll
+        for (int t = 0; t < kTiles; ++t) {
+            const int r = rbase + 8 * t + 2 * i;
+            *reinterpret_cast<float2*>(&red[g * kRows + r]) = make_float2(acc[t][0], acc[t][1]);
+            *reinterpret_cast<float2*>(&red[(g + 8) * kRows + r]) = make_float2(acc[t][2], acc[t][3]);
+        }
+        grid_dependency_wait();  // Y may still be in use by the preceding kernel
     }
-    // acc[0..1] = Y[g][row0 + 2i + {0,1}], acc[2..3] = Y[g + 8][row0 + 2i + {0,1}]
+    if (timed_out) record_timeout(dev_status);
+    __syncthreads();
+    const float4* red4 = reinterpret_cast<const float4*>(ring);
+    float4* part4 = reinterpret_cast<float4*>(ring) + 4 * 16 * kRows / 4;
+    constexpr int kQ = 16 * kRows / 4;  // float4s per block buffer
+    for (int e = threadIdx.x; e < kQ; e += kThreads) {
+        const float4 a = red4[e], b = red4[kQ + e], c = red4[2 * kQ + e], d = red4[3 * kQ + e];
+        part4[e] = make_float4(((a.x + b.x) + c.x) + d.x, ((a.y + b.y) + c.y) + d.y,
+                               ((a.z + b.z) + c.z) + d.z, ((a.w + b.w) + c.w) + d.w);
+    }
+
+    // cluster split-k: rank r adds rows [r * 128 / C, (r + 1) * 128 / C) over all ranks in rank order
+    cluster_sync();
+    const int rows_per_rank = kRows / cluster;
+    const int quads = rows_per_rank / 4;
+    const int r_lo = rank * rows_per_rank;
+    const uint32_t part_addr = smem_u32(part4);
+    for (int e = threadIdx.x; e < m * quads; e += kThreads) {
+        const int tok = e / quads;
+        const int r = r_lo + 4 * (e % quads);
+        const uint32_t off = static_cast<uint32_t>((tok * kRows + r) * 4);
+        float4 v[8];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int t = g + 8 * h;
-        if (t >= m) continue;
+        for (int q = 0; q < 8; ++q)
+            if (q < cluster) v[q] = ld_shared_cluster_f32x4(map_shared_rank(part_addr + off, q));
+        float4 sum = v[0];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int64_t r = row0 + 2 * i + e;
-            if (r >= n) continue;
-            const float v = acc[2 * h + e];
+        for (int q = 1; q < 8; ++q)
+            if (q < cluster) sum = make_float4(sum.x + v[q].x, sum.y + v[q].y, sum.z + v[q].z, sum.w + v[q].w);
+        const float o[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int64_t grow = row0 + r + c;
+            if (grow >= n) break;
             if (kBf16Out)
-                reinterpret_cast<__nv_bfloat16*>(Y)[static_cast<int64_t>(t) * n + r] = __float2bfloat16_rn(v);
+                reinterpret_cast<__nv_bfloat16*>(Y)[static_cast<int64_t>(tok) * n + grow] = __float2bfloat16_rn(o[c]);
             else
-                reinterpret_cast<float*>(Y)[static_cast<int64_t>(t) * n + r] = v;
+                reinterpret_cast<float*>(Y)[static_cast<int64_t>(tok) * n + grow] = o[c];
         }
     }
+    cluster_sync();  // keep this CTA's partials alive until every rank has read them
+}
+
+}  // namespace gemv
+
+// Cluster size (k split) for a weight of n rows and k columns: the smallest of
+// 1, 2, 4, 8 that gives at least one CTA per SM, without giving any CTA an
+// empty k range.
+static int gemv_cluster(int64_t n, int64_t k, int sm_count) {
+    const int64_t tiles = (n + gemv::kRows - 1) / gemv::kRows;
+    const int64_t stages = (k + gemv::kStageK - 1) / gemv::kStageK;
+    int c = 1;
+    while (c < 8 && tiles * c < sm_count && 2 * c <= stages) c *= 2;
+    return c;
+}
+
+template <bool kBf16Out, bool kM16>
+static cudaError_t launch_gemv(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const int8_t* absmax_q,
+                               const float* absmax_scale, const float* absmax_offset, int mt, int64_t n,
+                               int64_t k, int cluster, bool weights_early, void* Yt, int32_t* dev_status,
+                               int device, cudaStream_t stream) {
+    static bool attr_set[64] = {};
+    if (!attr_set[device]) {
+        const cudaError_t e = cudaFuncSetAttribute(gemv::k_nf4_gemv<kBf16Out, kM16>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, gemv::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set[device] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((n + gemv::kRows - 1) / gemv::kRows), cluster, 1);
+    cfg.blockDim = dim3(gemv::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = gemv::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = cluster;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = weights_early ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, gemv::k_nf4_gemv<kBf16Out, kM16>, tm_w, tm_x, absmax_q, absmax_scale,
+                              absmax_offset, mt, n, k, cluster, weights_early ? 1 : 0, Yt, dev_status);
 }
 
 cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                           const float* absmax_scale, const float* absmax_offset, int64_t n,
-                          int64_t k, void* Y, bool y_bf16, int32_t* dev_status,
+                          int64_t k, void* Y, bool y_bf16, int32_t* dev_status, bool weights_early,
                           const DeviceInfo& dev, cudaStream_t stream) {
-    (void)dev_status;
-    (void)dev;
-    const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
-    const unsigned blocks = static_cast<unsigned>((n + 31) / 32);
+    if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
+    CUtensorMap tm_w;
+    cudaError_t e = tmap_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, static_cast<uint64_t>(k / 2),
+                            static_cast<uint64_t>(n), static_cast<uint64_t>(k / 2), 128, gemv::kRows,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    const int cluster = gemv_cluster(n, k, dev.sm_count);
     const size_t ybytes = y_bf16 ? 2 : 4;
+    const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
     for (int64_t t0 = 0; t0 < m; t0 += 16) {
         const int mt = static_cast<int>((m - t0) < 16 ? (m - t0) : 16);
+        CUtensorMap tm_x;
+        e = tmap_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Xb + t0 * k, static_cast<uint64_t>(k),
+                    static_cast<uint64_t>(mt), static_cast<uint64_t>(k * 2), 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (e != cudaSuccess) return e;
         void* Yt = static_cast<char*>(Y) + static_cast<size_t>(t0) * n * ybytes;
         if (y_bf16)
-            k_nf4_gemv_simple<true><<<blocks, 128, 0, stream>>>(Xb + t0 * k, mt, k, wq, absmax_q,
-                                                                absmax_scale, absmax_offset, n, Yt);
+            e = (mt > 8) ? launch_gemv<true, true>(tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt, n, k,
+                                                   cluster, weights_early, Yt, dev_status, dev.device, stream)
+                         : launch_gemv<true, false>(tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt, n, k,
+                                                    cluster, weights_early, Yt, dev_status, dev.device, stream);
         else
-            k_nf4_gemv_simple<false><<<blocks, 128, 0, stream>>>(Xb + t0 * k, mt, k, wq, absmax_q,
-                                                                 absmax_scale, absmax_offset, n, Yt);
-        const cudaError_t e = cudaGetLastError();
+            e = (mt > 8) ? launch_gemv<false, true>(tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt, n, k,
+                                                    cluster, weights_early, Yt, dev_status, dev.device, stream)
+                         : launch_gemv<false, false>(tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt, n,
+                                                     k, cluster, weights_early, Yt, dev_status, dev.device, stream);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -35,7 +35,7 @@ cudaError_t launch_dequantize(const uint8_t* wq, const int8_t* absmax_q, const f
 
 cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                           const float* absmax_scale, const float* absmax_offset, int64_t n,
-                          int64_t k, void* Y, bool y_bf16, int32_t* dev_status,
+                          int64_t k, void* Y, bool y_bf16, int32_t* dev_status, bool weights_early,
                           const DeviceInfo& dev, cudaStream_t stream);
 
 }  // namespace nf4

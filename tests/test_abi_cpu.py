@@ -127,6 +127,10 @@ def test_weight_struct_validation(L):
     assert lin(FAKE, 4, ctypes.byref(_weight()), FAKE, 9, None, None) == -4
     assert lin(ODD, 4, ctypes.byref(_weight()), FAKE, 1, None, None) == -3
     assert lin(None, 4, ctypes.byref(_weight()), FAKE, 1, None, None) == -1
+    lex = L.nf4_linear_ex
+    assert lex(FAKE, 4, ctypes.byref(_weight()), FAKE, 1, None, 2, None) == -4   # unknown flag bit
+    assert lex(FAKE, 4, ctypes.byref(_weight(magic=3)), FAKE, 1, None, 1, None) == -5
+    assert lex(FAKE, 0, ctypes.byref(_weight()), FAKE, 1, None, 1, None) == -2
 
 
 def test_valid_call_without_a_gpu_reports_instead_of_crashing(L):

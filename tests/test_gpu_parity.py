@@ -194,6 +194,30 @@ def test_deterministic_and_stream_aware(nf4):
     assert torch.equal(ya, yb)
 
 
+def test_weights_early_launch_gives_identical_results(nf4):
+    """NF4_LINEAR_WEIGHTS_EARLY changes only when the weight loads may start;
+    a chain of dependent linears (each reading the previous output) must give
+    bit-identical results with and without it."""
+    k = 1024
+    ws = [nf4.quantize_weight(synth.weight_normal(k, k, seed=700 + j, dtype=torch.bfloat16, device="cuda"))
+          for j in range(4)]
+    X0 = synth.activations(7, k, seed=701, device="cuda")
+
+    def chain(early):
+        x = X0
+        for w in ws:
+            x = nf4.nf4_linear(x, w, torch.bfloat16, weights_early=early)
+        return x
+    a = chain(False)
+    b = chain(True)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        c = chain(True)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(a, c)
+
+
 def test_dev_status_stays_clear(nf4):
     W = synth.weight_normal(256, 512, seed=11, dtype=torch.bfloat16, device="cuda")
     X = synth.activations(3, 512, seed=12, device="cuda")
