@@ -1,0 +1,405 @@
+// nf4_gemm.cu -- fused dequantize + linear for large batches (prefill), sm_100a tcgen05.
+//
+// Sources: page "篇2-bitsandbytes-具体观-算法与实现剖析" (xyzblog), §2.2 code walk
+// (matmul_4bit = dequantize + matmul) and §2.5 (per-architecture 4-bit GEMM
+// files: prior art for older tensor cores); page "LLM 相關知識" (technicalnotes),
+// §5 "動態反量化" (weights restored to BF16 per layer for the matmul); page "Tim
+// Dettmers 如何用 bitsandbytes 與 QLoRA 降低 LLM 訓練門檻？", section "量化速度取決於硬體與
+// kernel": with large batches the work is compute-bound.
+//
+//   Y[t, r] = sum_c X[t, c] * What[r, c],   What = bf16(fp32(level[idx] * a_block)).
+//
+// One CTA computes a 256 (tokens) x 256 (weight rows) tile of Y with the
+// 5th-generation tensor cores: two 128 x 256 fp32 accumulators in tensor memory
+// (all 512 columns), bf16 operands from shared memory in the canonical K-major
+// 128-byte swizzled layout, 64 k per stage.
+//
+// * Warp 0 streams X tiles [256 x 64] with TMA; warp 2 streams the packed
+//   4-bit tile [256 rows x 32 bytes] with TMA (no multicast anywhere).
+// * Warps 4..11 (256 threads, one weight row each) dequantize on the CUDA
+//   cores: per (row, 64-block) they reconstruct the absmax, multiply the 16
+//   levels by it in fp32 and round to bf16 (the same values nf4_dequantize
+//   produces), split that 16-entry table into byte planes and decode each
+//   nibble with byte permutes -- no table lookups in shared memory, so the
+//   tensor core keeps the shared-memory bandwidth for its operands.  Each
+//   thread writes its 128-byte row of the swizzled B tile.
+// * One thread of warp 1 issues tcgen05.mma (M = 128, N = 256, K = 16) for
+//   both halves of the token tile, reusing the decoded weight tile, and
+//   releases stages with tcgen05.commit.
+// * After the k loop the dequant warps read the accumulators (tcgen05.ld) and
+//   store Y.
+// Every mbarrier wait is bounded; a wait that runs out records
+// NF4_ERR_DEVICE_TIMEOUT, the CTA drains what it issued and frees its tensor
+// memory before returning.
+#include "nf4_common.cuh"
+#include "nf4_internal.h"
+#include "nf4_ptx.cuh"
+#include "nf4_tmap.h"
+
+namespace nf4 {
+namespace gemm {
+
+constexpr int kBM = 256;  // tokens per CTA tile (two 128-row MMA halves)
+constexpr int kBN = 256;  // weight rows per CTA tile (MMA N)
+constexpr int kBK = 64;   // k per stage: one 128-byte swizzle row of bf16
+constexpr int kStagesA = 3;
+constexpr int kStagesB = 2;
+constexpr int kStagesP = 4;
+constexpr int kABytes = kBM * kBK * 2;  // 32768
+constexpr int kBBytes = kBN * kBK * 2;  // 32768
+constexpr int kPBytes = kBN * kBK / 2;  // 8192
+constexpr int kDequantWarps = 8;
+constexpr int kThreads = 32 * (4 + kDequantWarps);
+constexpr uint32_t kTmemCols = 512;
+constexpr int kOffB = kStagesA * kABytes;
+constexpr int kOffP = kOffB + kStagesB * kBBytes;
+constexpr int kOffBar = kOffP + kStagesP * kPBytes;
+constexpr int kNumBars = 2 * kStagesA + 2 * kStagesB + 2 * kStagesP + 2;
+constexpr int kSmemBytes = 1024 + kOffBar + kNumBars * 8 + 16;
+
+// Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major,
+// N = 256, M = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((128 >> 4) << 24);
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// (a & ~c) | (b & c)
+__device__ __forceinline__ uint32_t select_bytes(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xD8;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+// bf16 table of one (row, block), as byte planes: plane h[q] holds the high
+// bytes of entries 4q..4q+3, plane l[q] their low bytes.
+struct Planes {
+    uint32_t h[4], l[4];
+};
+
+// T[i] = bf16(fp32(c_i * a)) for the 16 levels (pairs of levels multiplied by
+// one packed f32x2 multiply), split into byte planes.
+__device__ __forceinline__ void build_planes(const uint64_t (&cpair)[8], float a, Planes& P) {
+    uint64_t aa;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(aa) : "f"(a));
+    uint32_t t[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        asm("{\n\t.reg .b64 r;\n\t.reg .f32 lo, hi;\n\t"
+            "mul.rn.f32x2 r, %1, %2;\n\t"
+            "mov.b64 {lo, hi}, r;\n\t"
+            "cvt.rn.bf16x2.f32 %0, hi, lo;\n\t}"
+            : "=r"(t[j])
+            : "l"(cpair[j]), "l"(aa));
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        P.h[q] = prmt(t[2 * q], t[2 * q + 1], 0x7531);
+        P.l[q] = prmt(t[2 * q], t[2 * q + 1], 0x6420);
+    }
+}
+
+// Four nibbles (the low 16 bits of s; s ^ 0x8888 in sx) -> two bf16x2 words in
+// k order.  For a nibble n < 8 the first permute picks T[n]'s byte and the
+// second yields a sign fill; for n >= 8 the other way round; a byte mask built
+// from each nibble's top bit selects the right one.  Nibble order in a packed
+// byte is (element 2i high, element 2i+1 low), so the final permutes swap
+// each pair back into k order.
+__device__ __forceinline__ void decode4(uint32_t s, uint32_t sx, const Planes& P, uint32_t& o0, uint32_t& o1) {
+    const uint32_t hA = prmt(P.h[0], P.h[1], s);
+    const uint32_t hB = prmt(P.h[2], P.h[3], sx);
+    const uint32_t lA = prmt(P.l[0], P.l[1], s);
+    const uint32_t lB = prmt(P.l[2], P.l[3], sx);
+    const uint32_t m = prmt(s << 4, s, 0xD9C8);  // byte k = 0xff iff nibble k >= 8
+    const uint32_t h = select_bytes(hA, hB, m);
+    const uint32_t l = select_bytes(lA, lB, m);
+    o0 = prmt(l, h, 0x4051);
+    o1 = prmt(l, h, 0x6273);
+}
+
+template <bool kBf16Out>
+__global__ void __launch_bounds__(kThreads, 1)
+k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+           const int8_t* __restrict__ absmax_q, const float* __restrict__ absmax_scale,
+           const float* __restrict__ mu_ptr, int64_t m, int64_t n, int64_t k, void* __restrict__ Y,
+           int32_t* __restrict__ dev_status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+    uint64_t* full_a = bars;
+    uint64_t* empty_a = full_a + kStagesA;
+    uint64_t* full_b = empty_a + kStagesA;
+    uint64_t* empty_b = full_b + kStagesB;
+    uint64_t* full_p = empty_b + kStagesB;
+    uint64_t* empty_p = full_p + kStagesP;
+    uint64_t* acc_ready = empty_p + kStagesP;
+    uint64_t* drained = acc_ready + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kBN;
+    const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kBM;
+    const int nk = static_cast<int>(k / kBK);
+    const uint32_t sbase = smem_u32(smem);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStagesA; ++s) {
+            mbar_init(&full_a[s], 1);
+            mbar_init(&empty_a[s], 1);
+        }
+        for (int s = 0; s < kStagesB; ++s) {
+            mbar_init(&full_b[s], kDequantWarps);
+            mbar_init(&empty_b[s], 1);
+        }
+        for (int s = 0; s < kStagesP; ++s) {
+            mbar_init(&full_p[s], 1);
+            mbar_init(&empty_p[s], kDequantWarps);
+        }
+        mbar_init(acc_ready, 1);
+        mbar_init(drained, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    bool timed_out = false;
+    if (warp == 0) {
+        // ---------------------------- X producer ----------------------------
+        if (lane == 0) {
+            prefetch_tensormap(&tm_x);
+            int issued = 0;
+            for (int kt = 0; kt < nk; ++kt) {
+                const int s = kt % kStagesA;
+                if (kt >= kStagesA && !mbar_wait(&empty_a[s], ((kt / kStagesA) - 1) & 1)) {
+                    timed_out = true;
+                    break;
+                }
+                mbar_arrive_expect_tx(&full_a[s], kABytes);
+                tma_load_2d(smem + s * kABytes, &tm_x, kt * kBK, static_cast<int32_t>(m0), &full_a[s]);
+                issued = kt + 1;
+            }
+            if (timed_out)  // leave no copy in flight
+                for (int kt = (issued > kStagesA ? issued - kStagesA : 0); kt < issued; ++kt)
+                    mbar_wait(&full_a[kt % kStagesA], (kt / kStagesA) & 1);
+        }
+    } else if (warp == 2) {
+        // ------------------------ packed-weight producer ----------------------
+        if (lane == 0) {
+            prefetch_tensormap(&tm_w);
+            int issued = 0;
+            for (int kt = 0; kt < nk; ++kt) {
+                const int s = kt % kStagesP;
+                if (kt >= kStagesP && !mbar_wait(&empty_p[s], ((kt / kStagesP) - 1) & 1)) {
+                    timed_out = true;
+                    break;
+                }
+                mbar_arrive_expect_tx(&full_p[s], kPBytes);
+                tma_load_2d(smem + kOffP + s * kPBytes, &tm_w, kt * (kBK / 2), static_cast<int32_t>(n0),
+                            &full_p[s]);
+                issued = kt + 1;
+            }
+            if (timed_out)
+                for (int kt = (issued > kStagesP ? issued - kStagesP : 0); kt < issued; ++kt)
+                    mbar_wait(&full_p[kt % kStagesP], (kt / kStagesP) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------ MMA issuer ----------------------------
+        if (lane == 0) {
+            for (int kt = 0; kt < nk; ++kt) {
+                const int sa = kt % kStagesA;
+                const int sb = kt % kStagesB;
+                if (!mbar_wait(&full_a[sa], (kt / kStagesA) & 1) || !mbar_wait(&full_b[sb], (kt / kStagesB) & 1)) {
+                    timed_out = true;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a_addr = sbase + sa * kABytes;
+                const uint32_t b_addr = sbase + kOffB + sb * kBBytes;
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int j = 0; j < kBK / 16; ++j)
+                        tc_mma_bf16(tmem + h * 256, smem_desc_sw128(a_addr + h * (128 * 128) + 32 * j),
+                                    smem_desc_sw128(b_addr + 32 * j), kIdesc, (kt > 0 || j > 0) ? 1u : 0u);
+                tc_commit(&empty_a[sa]);
+                tc_commit(&empty_b[sb]);
+            }
+            tc_commit(timed_out ? drained : acc_ready);
+            if (timed_out) mbar_wait(drained, 0);  // issued MMAs finish before TMEM is freed
+        }
+    } else if (warp >= 4) {
+        // ------------------------ dequantize, then epilogue --------------------
+        const int t = threadIdx.x - 128;  // weight row of the tile
+        const int64_t row_c = (n0 + t < n) ? n0 + t : n - 1;  // rows past n: computed, never stored
+        const int64_t kblocks = k / 64;
+        const float mu = __ldg(mu_ptr);
+        uint64_t cpair[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) cpair[j] = pack_f32x2(kLevels[2 * j], kLevels[2 * j + 1]);
+        const uint32_t prow = sbase + kOffP + t * 32;
+        const uint32_t brow = sbase + kOffB + t * 128;
+        const uint32_t swz = static_cast<uint32_t>(t & 7);
+        // Absmax inputs.  With k % 256 == 0 (and an aligned code array) the codes
+        // of 4 consecutive stages are one aligned word and share one scale (a
+        // group of 4 blocks never straddles a 256-block boundary); each group is
+        // loaded one group ahead so the load latency hides behind 4 stages.
+        const bool grouped = (kblocks & 3) == 0 && (reinterpret_cast<uintptr_t>(absmax_q) & 3) == 0;
+        const int64_t rbase = row_c * kblocks;
+        uint32_t qw_next = 0, qw_cur = 0;
+        float s_next = 0.0f, s_cur = 0.0f;
+        if (grouped) {
+            qw_next = __ldg(reinterpret_cast<const uint32_t*>(absmax_q + rbase));
+            s_next = __ldg(absmax_scale + (rbase >> 8));
+        }
+        for (int kt = 0; kt < nk; ++kt) {
+            const int sp = kt % kStagesP;
+            const int sb = kt % kStagesB;
+            int q;
+            float sc;
+            if (grouped) {
+                if ((kt & 3) == 0) {
+                    qw_cur = qw_next;
+                    s_cur = s_next;
+                    const int64_t nb = rbase + ((kt + 4 < nk) ? kt + 4 : kt);
+                    qw_next = __ldg(reinterpret_cast<const uint32_t*>(absmax_q + nb));
+                    s_next = __ldg(absmax_scale + (nb >> 8));
+                }
+                q = static_cast<int8_t>((qw_cur >> (8 * (kt & 3))) & 0xffu);
+                sc = s_cur;
+            } else {
+                const int64_t bidx = rbase + kt;
+                q = __ldg(absmax_q + bidx);
+                sc = __ldg(absmax_scale + (bidx >> 8));
+            }
+            if (!__all_sync(kFull, mbar_wait(&full_p[sp], (kt / kStagesP) & 1))) {
+                timed_out = true;
+                break;
+            }
+            const uint4 r0 = lds128(prow + sp * kPBytes);
+            const uint4 r1 = lds128(prow + sp * kPBytes + 16);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty_p[sp]);
+            Planes P;
+            build_planes(cpair, absmax_hat(q, sc, mu), P);
+            if (kt >= kStagesB && !__all_sync(kFull, mbar_wait(&empty_b[sb], ((kt / kStagesB) - 1) & 1))) {
+                timed_out = true;
+                break;
+            }
+            const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+            const uint32_t bst = brow + sb * kBBytes;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint32_t x = w[c] ^ 0x88888888u;
+                uint32_t o0, o1, o2, o3;
+                decode4(w[c], x, P, o0, o1);
+                decode4(w[c] >> 16, x >> 16, P, o2, o3);
+                sts128(bst + ((c ^ swz) << 4), o0, o1, o2, o3);
+            }
+            fence_proxy_async_shared();  // generic-proxy writes -> tensor-core reads
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full_b[sb]);
+        }
+        // epilogue: accumulators -> Y
+        const bool ok = !timed_out && __all_sync(kFull, mbar_wait(acc_ready, 0));
+        if (!ok) timed_out = true;
+        tc_fence_after();
+        const int wd = warp - 4;
+        const int half = wd >> 2;
+        const int quarter = warp & 3;  // tensor-memory lanes this warp may access
+        const int64_t tok = m0 + half * 128 + quarter * 32 + lane;
+        const bool vec = kBf16Out ? (n % 8 == 0) : (n % 4 == 0);
+#pragma unroll 1
+        for (int cc = 0; cc < kBN / 32; ++cc) {
+            uint32_t r[32];
+            if (ok) tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * 256 + cc * 32, r);
+            const int64_t col0 = n0 + cc * 32;
+            if (!ok || tok >= m || col0 >= n) continue;
+            if (kBf16Out) {
+                __nv_bfloat16* yrow = reinterpret_cast<__nv_bfloat16*>(Y) + tok * n;
+                if (vec && col0 + 32 <= n) {
+                    uint32_t p[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        p[e] = pack_bf16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
+                    uint4* dst = reinterpret_cast<uint4*>(yrow + col0);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(p[4 * e], p[4 * e + 1], p[4 * e + 2], p[4 * e + 3]);
+                } else {
+                    for (int e = 0; e < 32 && col0 + e < n; ++e) yrow[col0 + e] = __float2bfloat16_rn(__uint_as_float(r[e]));
+                }
+            } else {
+                float* yrow = reinterpret_cast<float*>(Y) + tok * n;
+                if (vec && col0 + 32 <= n) {
+                    uint4* dst = reinterpret_cast<uint4*>(yrow + col0);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) dst[e] = make_uint4(r[4 * e], r[4 * e + 1], r[4 * e + 2], r[4 * e + 3]);
+                } else {
+                    for (int e = 0; e < 32 && col0 + e < n; ++e) yrow[col0 + e] = __uint_as_float(r[e]);
+                }
+            }
+        }
+    }
+    if (timed_out) record_timeout(dev_status);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace gemm
+
+cudaError_t launch_gemm(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
+                        const float* absmax_scale, const float* absmax_offset, int64_t n, int64_t k, void* Y,
+                        bool y_bf16, int32_t* dev_status, const DeviceInfo& dev, cudaStream_t stream) {
+    static bool attr_set[64][2] = {};
+    if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
+    const void* fn = y_bf16 ? reinterpret_cast<const void*>(&gemm::k_nf4_gemm<true>)
+                            : reinterpret_cast<const void*>(&gemm::k_nf4_gemm<false>);
+    if (!attr_set[dev.device][y_bf16]) {
+        const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set[dev.device][y_bf16] = true;
+    }
+    CUtensorMap tm_x, tm_w;
+    cudaError_t e = tmap_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, static_cast<uint64_t>(k),
+                            static_cast<uint64_t>(m), static_cast<uint64_t>(k * 2), gemm::kBK, gemm::kBM,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    e = tmap_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n),
+                static_cast<uint64_t>(k / 2), gemm::kBK / 2, gemm::kBN, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (e != cudaSuccess) return e;
+    const dim3 grid(static_cast<unsigned>((n + gemm::kBN - 1) / gemm::kBN),
+                    static_cast<unsigned>((m + gemm::kBM - 1) / gemm::kBM));
+    if (y_bf16)
+        gemm::k_nf4_gemm<true><<<grid, gemm::kThreads, gemm::kSmemBytes, stream>>>(
+            tm_x, tm_w, absmax_q, absmax_scale, absmax_offset, m, n, k, Y, dev_status);
+    else
+        gemm::k_nf4_gemm<false><<<grid, gemm::kThreads, gemm::kSmemBytes, stream>>>(
+            tm_x, tm_w, absmax_q, absmax_scale, absmax_offset, m, n, k, Y, dev_status);
+    return cudaGetLastError();
+}
+
+}  // namespace nf4

@@ -462,6 +462,9 @@ cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int
                           int64_t k, void* Y, bool y_bf16, int32_t* dev_status, bool weights_early,
                           const DeviceInfo& dev, cudaStream_t stream) {
     if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
+    if (m > kGemvMaxTokens)
+        return launch_gemm(X, m, wq, absmax_q, absmax_scale, absmax_offset, n, k, Y, y_bf16, dev_status, dev,
+                           stream);
     CUtensorMap tm_w;
     cudaError_t e = tmap_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, static_cast<uint64_t>(k / 2),
                             static_cast<uint64_t>(n), static_cast<uint64_t>(k / 2), 128, gemv::kRows,

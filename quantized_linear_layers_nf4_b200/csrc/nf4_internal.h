@@ -38,4 +38,11 @@ cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int
                           int64_t k, void* Y, bool y_bf16, int32_t* dev_status, bool weights_early,
                           const DeviceInfo& dev, cudaStream_t stream);
 
+cudaError_t launch_gemm(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
+                        const float* absmax_scale, const float* absmax_offset, int64_t n, int64_t k, void* Y,
+                        bool y_bf16, int32_t* dev_status, const DeviceInfo& dev, cudaStream_t stream);
+
+// Token counts up to this run the decode GEMV; larger ones the tcgen05 GEMM.
+constexpr int64_t kGemvMaxTokens = 16;
+
 }  // namespace nf4

@@ -170,6 +170,17 @@ def test_linear_token_counts(nf4, m):
     _check_linear(nf4, X, weight, orc)
 
 
+@pytest.mark.parametrize("m,n,k", [(17, 64, 64), (257, 300, 192), (300, 520, 640), (1024, 1024, 1024),
+                                   (64, 8, 128), (513, 2048, 256)])
+def test_gemm_path_ragged_tiles(nf4, m, n, k):
+    """m > 16 runs the tcgen05 GEMM: tiles of 256 tokens x 256 weight rows with
+    ragged edges in both, several k stages."""
+    W = synth.weight_normal(n, k, seed=800 + m + n, dtype=torch.bfloat16, device="cuda")
+    X = synth.activations(m, k, seed=900 + m, device="cuda")
+    weight, orc = _check_quant(nf4, W, full_dequant=False, rows=[0, n - 1])
+    _check_linear(nf4, X, weight, orc)
+
+
 @pytest.mark.parametrize("n,k", [(8, 64), (1, 128), (9, 64), (24, 1088), (1000, 256)])
 def test_linear_ragged_shapes(nf4, n, k):
     W = synth.weight_normal(n, k, seed=500 + n, dtype=torch.bfloat16, device="cuda")
