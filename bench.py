@@ -316,6 +316,8 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize()
     shapes = sorted(set((w.n, w.k) for w in weights))
 
+    early = not args.no_weights_early
+
     def decode_setup(m):
         xs = {k: synth.activations(m, k, seed=synth.seed_for(2, 100 + m) + k, device=dev)
               for k in set(k for _, k in shapes)}
@@ -323,7 +325,7 @@ def run_ours(args, rank, world, local):
 
         def step():
             for w in weights:
-                nf4.nf4_linear(xs[w.k], w, torch.bfloat16, out=ys[w.n], weights_early=True)
+                nf4.nf4_linear(xs[w.k], w, torch.bfloat16, out=ys[w.n], weights_early=early)
         step()
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
@@ -455,8 +457,9 @@ def run_ours(args, rank, world, local):
                        "l2": "inputs larger than L2 (%.2f GB of NF4 weights per step vs 126 MB)"
                              % (sum(w.nbytes() for w in weights) / 1e9),
                        "y_dtype": "bf16", "parallelism": "replicas (weak scaling)",
-                       "launch": "CUDA graph of nf4_linear_ex(NF4_LINEAR_WEIGHTS_EARLY): programmatic "
-                                 "dependent launches, weight loads overlap the previous layer"},
+                       "launch": ("CUDA graph of nf4_linear_ex(NF4_LINEAR_WEIGHTS_EARLY): programmatic "
+                                  "dependent launches, weight loads overlap the previous layer") if early
+                                 else "CUDA graph of nf4_linear: each layer starts after the previous ends"},
             "frac_of_peak": round(value / world / pk["hbm_gbs"], 4),
             "decode_gbs_by_m": by_m,
             "gemm": gemm,
@@ -481,6 +484,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--m", type=int, default=16, help="tokens per decode step (1..16)")
     ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--no-weights-early", action="store_true",
+                    help="launch each linear without programmatic dependent launch")
     ap.add_argument("--skip-gemm", action="store_true")
     ap.add_argument("--skip-quant", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -55,7 +55,10 @@ constexpr int kLutBytes = 16 * 256 * 8;          // 32768
 constexpr int kRingBytes = kRing * kStageBytes;
 constexpr int kSmemBytes = 1024 /*alignment slack*/ + kRingBytes + kLutBytes + 2 * kRing * 8;
 static_assert(kStageBytes % 1024 == 0, "stages keep the 1 KiB alignment the 128-byte swizzle needs");
-static_assert(4 * 16 * kRows * 4 + 16 * kRows * 4 <= kRingBytes, "reduction fits in the ring");
+// Per-block partial sums are stored [token][row] with a padded token pitch so
+// that the 8 row groups of a warp write distinct banks.
+constexpr int kRedPitch = kRows + 8;
+static_assert(4 * 16 * kRedPitch * 4 + 16 * kRows * 4 <= kRingBytes, "reduction fits in the ring");
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
@@ -206,7 +209,6 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
         }
         fence_mbar_init();
     }
-    grid_launch_dependents();  // the next kernel on the stream may start its prologue
     __syncthreads();
 
     bool timed_out = false;
@@ -292,6 +294,9 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
             }
         }
         if (!x_ready) grid_dependency_wait();
+        // every copy of this CTA is issued: the next kernel on the stream may
+        // start its prologue (its weight prefetch overlaps our last stages)
+        grid_launch_dependents();
         // on a timeout leave no copy in flight: wait (bounded) for every stage issued
         if (timed_out && lane == 0)
             for (int s = 0; s < kRing; ++s)
@@ -307,6 +312,9 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
             sts128(smem_u32(lut) + 16u * c, make_uint4(hi, lo, hi, lo));
         }
         named_bar_sync(1, 32 * kConsumers);
+        // Under a programmatic dependent launch, sleep here (rather than poll
+        // the ring) until the preceding kernel has finished; otherwise a no-op.
+        grid_dependency_wait();
 
         const int g = lane >> 2;
         const int i = lane & 3;
@@ -362,22 +370,27 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
         // block land in disjoint rows of the same buffer)
         __syncwarp();
         named_bar_sync(1, 32 * kConsumers);  // every consumer is done with the ring
-        float* red = reinterpret_cast<float*>(ring) + blk * 16 * kRows;
+        float* red = reinterpret_cast<float*>(ring) + blk * 16 * kRedPitch;
 #pragma unroll
         for (int t = 0; t < kTiles; ++t) {
             const int r = rbase + 8 * t + 2 * i;
-            *reinterpret_cast<float2*>(&red[g * kRows + r]) = make_float2(acc[t][0], acc[t][1]);
-            *reinterpret_cast<float2*>(&red[(g + 8) * kRows + r]) = make_float2(acc[t][2], acc[t][3]);
+            *reinterpret_cast<float2*>(&red[g * kRedPitch + r]) = make_float2(acc[t][0], acc[t][1]);
+            *reinterpret_cast<float2*>(&red[(g + 8) * kRedPitch + r]) = make_float2(acc[t][2], acc[t][3]);
         }
         grid_dependency_wait();  // Y may still be in use by the preceding kernel
     }
     if (timed_out) record_timeout(dev_status);
     __syncthreads();
-    const float4* red4 = reinterpret_cast<const float4*>(ring);
-    float4* part4 = reinterpret_cast<float4*>(ring) + 4 * 16 * kRows / 4;
-    constexpr int kQ = 16 * kRows / 4;  // float4s per block buffer
+    const float* redf = reinterpret_cast<const float*>(ring);
+    float4* part4 = reinterpret_cast<float4*>(ring) + 4 * 16 * kRedPitch / 4;
+    constexpr int kQ = 16 * kRows / 4;  // float4s of partial sums per CTA
+    constexpr int kB = 16 * kRedPitch;  // floats per block buffer
     for (int e = threadIdx.x; e < kQ; e += kThreads) {
-        const float4 a = red4[e], b = red4[kQ + e], c = red4[2 * kQ + e], d = red4[3 * kQ + e];
+        const int off = (e / (kRows / 4)) * kRedPitch + 4 * (e % (kRows / 4));
+        const float4 a = *reinterpret_cast<const float4*>(redf + off);
+        const float4 b = *reinterpret_cast<const float4*>(redf + kB + off);
+        const float4 c = *reinterpret_cast<const float4*>(redf + 2 * kB + off);
+        const float4 d = *reinterpret_cast<const float4*>(redf + 3 * kB + off);
         part4[e] = make_float4(((a.x + b.x) + c.x) + d.x, ((a.y + b.y) + c.y) + d.y,
                                ((a.z + b.z) + c.z) + d.z, ((a.w + b.w) + c.w) + d.w);
     }
