@@ -44,17 +44,23 @@ constexpr int kStageK = 256;                     // k per pipeline stage
 constexpr int kRing = 3;                         // stages in flight per CTA
 constexpr int kConsumers = 8;                    // consumer warps
 constexpr int kTiles = 8;                        // 8-row MMA tiles per consumer warp (64 rows)
-constexpr int kThreads = 32 * (kConsumers + 1);  // + one producer warp
+constexpr int kThreads = 32 * kConsumers;        // no dedicated producer warp
 constexpr int kWBytes = kRows * kStageK / 2;     // 16384: packed codes of a stage
 constexpr int kXBox = 16 * 64 * 2;               // 2048: X box of 16 tokens x 64 k (bf16)
 constexpr int kXBytes = 4 * kXBox;               // 8192
 constexpr int kTmaBytes = kWBytes + kXBytes;     // bytes a stage receives by TMA
-constexpr int kAhatBytes = 4 * kRows * 4;        // 2048: reconstructed absmax, [row][block]
-constexpr int kStageBytes = kTmaBytes + kAhatBytes;  // 26624 = 26 KiB (keeps 1 KiB alignment)
+constexpr int kStageBytes = kTmaBytes;           // 24576 (keeps 1 KiB alignment)
+constexpr int kAring = 4;                        // reconstructed-absmax tables in flight
+constexpr int kAhatBytes = 4 * kRows * 4;        // 2048: one stage's table, [row][block]
 constexpr int kLutBytes = 16 * 256 * 8;          // 32768
 constexpr int kRingBytes = kRing * kStageBytes;
-constexpr int kSmemBytes = 1024 /*alignment slack*/ + kRingBytes + kLutBytes + 2 * kRing * 8;
+constexpr int kAhatOff = kRingBytes;
+constexpr int kLutOff = kAhatOff + kAring * kAhatBytes;
+constexpr int kBarOff = kLutOff + kLutBytes;
+// two CTAs per SM: (113 KiB + 1 KiB reserved) x 2 within the SM's 228 KiB
+constexpr int kSmemBytes = kBarOff + (kRing + kAring) * 8 + 2 * kRing * 4;
 static_assert(kStageBytes % 1024 == 0, "stages keep the 1 KiB alignment the 128-byte swizzle needs");
+static_assert(kSmemBytes + 1024 <= 228 * 1024 / 2, "two CTAs fit on an SM");
 // Per-block partial sums are stored [token][row] with a padded token pitch so
 // that the 8 row groups of a warp write distinct banks.
 constexpr int kRedPitch = kRows + 8;
@@ -118,67 +124,79 @@ __device__ __forceinline__ uint32_t scale_pack(uint64_t levels, uint64_t aa) {
     return out;
 }
 
-// The producer's per-stage absmax inputs.  Lane l owns rows l + 32 u (u = 0..3)
-// and the stage's 4 blocks of each: the 4 int8 codes of a row packed in one
-// word, and the (at most two) double-quantization scales its 4 blocks use.
+// Reconstructed-absmax inputs of one stage for one thread.  Thread t owns row
+// (t mod 128) of the tile and blocks 2 (t div 128) + {0, 1} of the stage: the
+// row's 4 int8 codes of the stage packed in one word, and the
+// double-quantization scales of the thread's two blocks.
 struct AbsmaxIn {
-    uint32_t q[4];
-    float s_lo[4], s_hi[4];
+    uint32_t q;
+    float s0, s1;
 };
 
 __device__ __forceinline__ void load_absmax_in(AbsmaxIn& a, const int8_t* __restrict__ absmax_q,
-                                               const float* __restrict__ absmax_scale, int64_t row0,
-                                               int lane, int st, int64_t n, int64_t kblocks,
-                                               bool aligned4) {
-    const int64_t kb0 = static_cast<int64_t>(st) * 4;
+                                               const float* __restrict__ absmax_scale, int64_t grow, int half,
+                                               int st, int64_t n, int64_t kblocks, bool aligned4) {
+    const int64_t kb = static_cast<int64_t>(st) * 4;
     if (aligned4) {
         // k % 256 == 0 and an aligned code array: a row's 4 codes of a stage are
         // one aligned word.  Every load is unconditional (rows past n are
-        // clamped; their results are never stored) and lands directly in its
-        // field, so nothing waits for it until the stage is used.
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            int64_t grow = row0 + lane + 32 * u;
-            grow = grow < n ? grow : n - 1;
-            const int64_t b0 = grow * kblocks + kb0;
-            a.q[u] = __ldg(reinterpret_cast<const uint32_t*>(absmax_q + b0));
-            a.s_lo[u] = __ldg(absmax_scale + (b0 >> 8));
-            a.s_hi[u] = __ldg(absmax_scale + ((b0 + 3) >> 8));
-        }
+        // clamped; their results are never stored), so nothing waits for it
+        // until the stage is used.
+        const int64_t r = grow < n ? grow : n - 1;
+        const int64_t b0 = r * kblocks + kb + 2 * half;
+        a.q = __ldg(reinterpret_cast<const uint32_t*>(absmax_q + (b0 - 2 * half)));
+        a.s0 = __ldg(absmax_scale + (b0 >> 8));
+        a.s1 = __ldg(absmax_scale + ((b0 + 1) >> 8));
         return;
     }
-    // general shapes: gather the codes byte by byte (stalls, but correct)
+    // general shapes: gather the codes byte by byte; blocks past k get q = 0
+    uint32_t q = 0;
+    float s0 = 0.0f, s1 = 0.0f;
+    if (grow < n) {
+        const int64_t b0 = grow * kblocks + kb;
+        const int64_t nvalid = kblocks - kb;  // >= 1
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const int64_t grow = row0 + lane + 32 * u;
-        uint32_t q = 0;
-        float lo = 0.0f, hi = 0.0f;
-        if (grow < n) {
-            const int64_t b0 = grow * kblocks + kb0;
-            const int64_t nvalid = kblocks - kb0;  // >= 1
-#pragma unroll
-            for (int b = 0; b < 4; ++b)
-                if (b < nvalid)
-                    q |= static_cast<uint32_t>(static_cast<uint8_t>(__ldg(absmax_q + b0 + b))) << (8 * b);
-            const int64_t blast = b0 + (nvalid < 4 ? nvalid : 4) - 1;
-            lo = __ldg(absmax_scale + (b0 >> 8));
-            hi = __ldg(absmax_scale + (blast >> 8));
-        }
-        a.q[u] = q;
-        a.s_lo[u] = lo;
-        a.s_hi[u] = hi;
+        for (int b = 0; b < 4; ++b)
+            if (b < nvalid) q |= static_cast<uint32_t>(static_cast<uint8_t>(__ldg(absmax_q + b0 + b))) << (8 * b);
+        const int64_t last = b0 + (nvalid < 4 ? nvalid : 4) - 1;
+        const int64_t ba = b0 + 2 * half, bb = ba + 1;
+        s0 = __ldg(absmax_scale + ((ba < last ? ba : last) >> 8));
+        s1 = __ldg(absmax_scale + ((bb < last ? bb : last) >> 8));
     }
+    a.q = q;
+    a.s0 = s0;
+    a.s1 = s1;
 }
 
 // Keeps the compiler from hoisting work that uses `a` above the point where
 // this is called (the values pass through an opaque asm).
 __device__ __forceinline__ void pin(AbsmaxIn& a) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-        asm volatile("" : "+r"(a.q[u]), "+f"(a.s_lo[u]), "+f"(a.s_hi[u]));
+    asm volatile("" : "+r"(a.q), "+f"(a.s0), "+f"(a.s1));
 }
 
-constexpr int kPrefetch = 3;  // stages of absmax inputs in flight per producer lane
+// a = fp32(fp32(fp32(q / 127) * s) + mu) for the thread's two blocks, stored
+// to the stage's [row][block] table.
+__device__ __forceinline__ void store_ahat(uint32_t ahat_row, int half, const AbsmaxIn& a, float mu) {
+    const uint32_t qq = a.q >> (16 * half);
+    const float q0 = static_cast<float>(static_cast<int8_t>(qq & 0xffu));
+    const float q1 = static_cast<float>(static_cast<int8_t>((qq >> 8) & 0xffu));
+    const float a0 = __fadd_rn(__fmul_rn(div127(q0), a.s0), mu);
+    const float a1 = __fadd_rn(__fmul_rn(div127(q1), a.s1), mu);
+    asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(ahat_row + 8u * half), "f"(a0), "f"(a1) : "memory");
+}
+
+constexpr int kPrefetch = 3;  // stages of absmax inputs in flight per thread
+
+// Loads W (and, once allowed, X) of stage `st` into ring slot `slot`.
+__device__ __forceinline__ void issue_stage(uint8_t* stage, const CUtensorMap* tm_w, const CUtensorMap* tm_x,
+                                            uint64_t* tfull, int st, int64_t row0, bool with_x) {
+    mbar_arrive_expect_tx(tfull, kTmaBytes);
+    tma_load_2d(stage, tm_w, st * (kStageK / 2), static_cast<int32_t>(row0), tfull);
+    if (with_x) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) tma_load_2d(stage + kWBytes + b * kXBox, tm_x, st * kStageK + 64 * b, 0, tfull);
+    }
+}
 
 template <bool kBf16Out, bool kM16>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -186,12 +204,21 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
            const int8_t* __restrict__ absmax_q, const float* __restrict__ absmax_scale,
            const float* __restrict__ mu_ptr, int m, int64_t n, int64_t k, int cluster, int weights_early,
            void* __restrict__ Y, int32_t* __restrict__ dev_status) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* ring = smem;
-    float2* lut = reinterpret_cast<float2*>(smem + kRingBytes);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRingBytes + kLutBytes);
-    uint64_t* empty = full + kRing;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // The 128-byte swizzle needs 1 KiB-aligned stages.  The dynamic window is
+    // declared so aligned; should a platform place it otherwise, every CTA
+    // sees the same base and returns here, before any barrier, with an error.
+    if (smem_u32(smem_raw) & 1023u) {
+        if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && dev_status)
+            atomicExch(dev_status, -9 /* NF4_ERR_UNSUPPORTED_DEVICE */);
+        return;
+    }
+    uint8_t* ring = smem_raw;
+    float2* lut = reinterpret_cast<float2*>(smem_raw + kLutOff);
+    uint64_t* tfull = reinterpret_cast<uint64_t*>(smem_raw + kBarOff);  // TMA bytes of a stage landed
+    uint64_t* afull = tfull + kRing;                                     // absmax table of a stage written
+    uint32_t* done = reinterpret_cast<uint32_t*>(afull + kAring);        // warps finished, per ring slot
+    int* issued = reinterpret_cast<int*>(done + kRing);                  // last use issued, per ring slot
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -201,135 +228,104 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
     const int rank = static_cast<int>(blockIdx.y);
     const int s0 = static_cast<int>((static_cast<int64_t>(n_stages) * rank) / cluster);
     const int s1 = static_cast<int>((static_cast<int64_t>(n_stages) * (rank + 1)) / cluster);
+    const int nst = s1 - s0;  // >= 1
+    const int n_pre = nst < kRing ? nst : kRing;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kRing; ++s) {
-            mbar_init(&full[s], 2);   // the TMA bytes' arrive + the absmax-ready arrive
-            mbar_init(&empty[s], kConsumers);
+            mbar_init(&tfull[s], 1);
+            done[s] = 0;
+            issued[s] = -1;
         }
+        for (int s = 0; s < kAring; ++s) mbar_init(&afull[s], kConsumers);
         fence_mbar_init();
+        prefetch_tensormap(&tm_w);
+        prefetch_tensormap(&tm_x);
+        if (!weights_early) grid_dependency_wait();
+        // the weights of the first stages start streaming before anything else
+        for (int j = 0; j < n_pre; ++j) {
+            issue_stage(ring + j * kStageBytes, &tm_w, &tm_x, &tfull[j], s0 + j, row0, !weights_early);
+            issued[j] = 0;
+        }
     }
-    __syncthreads();
+
+    // absmax inputs of the first kPrefetch + 1 stages (rows past n clamped)
+    const int arow = threadIdx.x & (kRows - 1);
+    const int half = threadIdx.x >> 7;
+    const bool aligned4 = (kblocks & 3) == 0 && (reinterpret_cast<uintptr_t>(absmax_q) & 3) == 0;
+    const int64_t agrow = row0 + arow;
+    AbsmaxIn first;
+    AbsmaxIn pre[kPrefetch];
+    load_absmax_in(first, absmax_q, absmax_scale, agrow, half, s0, n, kblocks, aligned4);
+#pragma unroll
+    for (int d = 0; d < kPrefetch; ++d)
+        load_absmax_in(pre[d], absmax_q, absmax_scale, agrow, half, min(s0 + 1 + d, n_stages - 1), n, kblocks,
+                       aligned4);
+    const float mu = __ldg(mu_ptr);
+
+    // byte -> (level of high nibble, level of low nibble), 16 copies so that
+    // the 16 lanes of a half-warp always read distinct banks
+    // (consecutive threads write consecutive 16-byte chunks: 2 copies each)
+    for (int c = threadIdx.x; c < kLutBytes / 16; c += kThreads) {
+        const int b = c >> 3;
+        const uint32_t hi = __float_as_uint(kLevels[b >> 4]), lo = __float_as_uint(kLevels[b & 15]);
+        sts128(smem_u32(lut) + 16u * c, make_uint4(hi, lo, hi, lo));
+    }
+    __syncthreads();  // barriers initialised, LUT written
+
+    if (threadIdx.x == 0 && weights_early) {
+        // weights are in flight; X (the preceding kernel's output) only after it finished
+        grid_dependency_wait();
+        for (int j = 0; j < n_pre; ++j)
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                tma_load_2d(ring + j * kStageBytes + kWBytes + b * kXBox, &tm_x, (s0 + j) * kStageK + 64 * b, 0,
+                            &tfull[j]);
+    }
+    // the absmax table of the first stage
+    const uint32_t ahat_base = smem_u32(smem_raw + kAhatOff);
+    const uint32_t ahat_mine = ahat_base + arow * 16u;
+    pin(first);
+    store_ahat(ahat_mine, half, first, mu);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&afull[0]);
+    // Under a programmatic dependent launch, sleep here (rather than poll the
+    // ring) until the preceding kernel has finished; otherwise a no-op.
+    grid_dependency_wait();
+
+    const int g = lane >> 2;
+    const int i = lane & 3;
+    const int blk = warp & 3;            // 64-block of the stage
+    const int rbase = (warp >> 2) * 64;  // first of this warp's 64 rows
+    const uint32_t lut_lane = smem_u32(lut) + (lane & 15) * 8u;
+    float acc[kTiles][4];
+#pragma unroll
+    for (int t = 0; t < kTiles; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
 
     bool timed_out = false;
-    if (warp == kConsumers) {
-        // ------------------------------ producer ------------------------------
-        if (lane == 0) {
-            prefetch_tensormap(&tm_w);
-            prefetch_tensormap(&tm_x);
-        }
-        if (!weights_early) grid_dependency_wait();
-        const float mu = __ldg(mu_ptr);
-        int last_use[kRing];
+    for (int j0 = 0; j0 < nst && !timed_out; j0 += kPrefetch) {
 #pragma unroll
-        for (int s = 0; s < kRing; ++s) last_use[s] = -1;
-        bool x_ready = !weights_early;  // X (the previous kernel's output) may be read
-        const int n_pre = (s1 - s0) < kRing ? (s1 - s0) : kRing;
-        const bool aligned4 = (kblocks & 3) == 0 && (reinterpret_cast<uintptr_t>(absmax_q) & 3) == 0;
-        AbsmaxIn pre[kPrefetch];
-#pragma unroll
-        for (int d = 0; d < kPrefetch; ++d)
-            load_absmax_in(pre[d], absmax_q, absmax_scale, row0, lane, min(s0 + d, n_stages - 1), n, kblocks, aligned4);
-        for (int st0 = s0; st0 < s1 && !timed_out; st0 += kPrefetch) {
-#pragma unroll
-            for (int d = 0; d < kPrefetch; ++d) {
-                const int st = st0 + d;
-                if (st >= s1) break;
-                const int j = st - s0;
-                const int slot = j % kRing;
-                const int use = j / kRing;
-                if (j >= kRing && !__all_sync(kFull, mbar_wait(&empty[slot], (use - 1) & 1))) {
-                    timed_out = true;
-                    break;
-                }
-                uint8_t* stage = ring + slot * kStageBytes;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&full[slot], kTmaBytes);
-                    tma_load_2d(stage, &tm_w, st * (kStageK / 2), static_cast<int32_t>(row0), &full[slot]);
-                    if (x_ready) {
-#pragma unroll
-                        for (int b = 0; b < 4; ++b)
-                            tma_load_2d(stage + kWBytes + b * kXBox, &tm_x, st * kStageK + 64 * b, 0, &full[slot]);
-                    }
-                    last_use[slot] = use;
-                }
-                pin(pre[d]);  // the copies above are issued before the absmax work below
-                // reconstructed absmax a = fp32(fp32(fp32(q / 127) * s) + mu) of this stage.
-                // Blocks past k or rows past n get q = s = 0 (a = mu, finite): X is
-                // zero-filled there, so their products vanish.
-                const uint32_t ahat = smem_u32(stage + kTmaBytes);  // [row][block] floats
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int row = lane + 32 * u;
-                    const int64_t b0 = (row0 + row) * kblocks + static_cast<int64_t>(st) * 4;
-                    float a4[4];
-#pragma unroll
-                    for (int b = 0; b < 4; ++b) {
-                        const float sc = (((b0 + b) >> 8) == (b0 >> 8)) ? pre[d].s_lo[u] : pre[d].s_hi[u];
-                        const float qf = static_cast<float>(static_cast<int8_t>((pre[d].q[u] >> (8 * b)) & 0xffu));
-                        a4[b] = __fadd_rn(__fmul_rn(div127(qf), sc), mu);
-                    }
-                    sts128(ahat + row * 16u, make_uint4(__float_as_uint(a4[0]), __float_as_uint(a4[1]),
-                                                        __float_as_uint(a4[2]), __float_as_uint(a4[3])));
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&full[slot]);
-                // (unconditional, clamped to a valid stage, so no select waits on the loads)
-                load_absmax_in(pre[d], absmax_q, absmax_scale, row0, lane, min(st + kPrefetch, n_stages - 1), n,
-                               kblocks, aligned4);
-                if (!x_ready && j + 1 == n_pre) {
-                    // weights of the first stages are in flight; now wait for the
-                    // preceding kernel before touching X
-                    grid_dependency_wait();
-                    x_ready = true;
-                    if (lane == 0)
-                        for (int jj = 0; jj <= j; ++jj) {
-                            uint8_t* stg = ring + (jj % kRing) * kStageBytes;
-#pragma unroll
-                            for (int b = 0; b < 4; ++b)
-                                tma_load_2d(stg + kWBytes + b * kXBox, &tm_x, (s0 + jj) * kStageK + 64 * b, 0,
-                                            &full[jj % kRing]);
-                        }
-                }
-            }
-        }
-        if (!x_ready) grid_dependency_wait();
-        // every copy of this CTA is issued: the next kernel on the stream may
-        // start its prologue (its weight prefetch overlaps our last stages)
-        grid_launch_dependents();
-        // on a timeout leave no copy in flight: wait (bounded) for every stage issued
-        if (timed_out && lane == 0)
-            for (int s = 0; s < kRing; ++s)
-                if (last_use[s] >= 0) mbar_wait(&full[s], last_use[s] & 1);
-    } else {
-        // ------------------------------ consumers -----------------------------
-        // byte -> (level of high nibble, level of low nibble), 16 copies so that
-        // the 16 lanes of a half-warp always read distinct banks
-        // (consecutive threads write consecutive 16-byte chunks: 2 copies each)
-        for (int c = threadIdx.x; c < kLutBytes / 16; c += 32 * kConsumers) {
-            const int b = c >> 3;
-            const uint32_t hi = __float_as_uint(kLevels[b >> 4]), lo = __float_as_uint(kLevels[b & 15]);
-            sts128(smem_u32(lut) + 16u * c, make_uint4(hi, lo, hi, lo));
-        }
-        named_bar_sync(1, 32 * kConsumers);
-        // Under a programmatic dependent launch, sleep here (rather than poll
-        // the ring) until the preceding kernel has finished; otherwise a no-op.
-        grid_dependency_wait();
-
-        const int g = lane >> 2;
-        const int i = lane & 3;
-        const int blk = warp & 3;          // 64-block of the stage
-        const int rbase = (warp >> 2) * 64;  // first of this warp's 64 rows
-        const uint32_t lut_lane = smem_u32(lut) + (lane & 15) * 8u;
-        float acc[kTiles][4];
-#pragma unroll
-        for (int t = 0; t < kTiles; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-
-        for (int st = s0; st < s1; ++st) {
-            const int j = st - s0;
+        for (int d = 0; d < kPrefetch; ++d) {
+            const int j = j0 + d;
+            if (j >= nst) break;
             const int slot = j % kRing;
+            // absmax table of the next stage.  Its table slot held stage j - 3:
+            // this warp saw stage j - 1's table complete, so every warp has begun
+            // stage j - 2 and is done with stage j - 3.
+            if (j + 1 < nst) {
+                const int nslot = (j + 1) % kAring;
+                pin(pre[d]);
+                store_ahat(ahat_mine + nslot * kAhatBytes, half, pre[d], mu);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&afull[nslot]);
+                // (unconditional, clamped to a valid stage, so no select waits on the loads)
+                load_absmax_in(pre[d], absmax_q, absmax_scale, agrow, half,
+                               min(s0 + j + 1 + kPrefetch, n_stages - 1), n, kblocks, aligned4);
+            }
             // every lane polls; the warp proceeds only if all of them saw the stage
-            if (!__all_sync(kFull, mbar_wait(&full[slot], (j / kRing) & 1))) {
+            const int aslot = j % kAring;
+            if (!__all_sync(kFull, mbar_wait(&tfull[slot], (j / kRing) & 1) &&
+                                       mbar_wait(&afull[aslot], (j / kAring) & 1))) {
                 timed_out = true;
                 break;
             }
@@ -346,7 +342,7 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
             const uint32_t xa[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
             const uint32_t xc[8] = {xc0.x, xc0.y, xc0.z, xc0.w, xc1.x, xc1.y, xc1.z, xc1.w};
             const uint32_t wb = stage + (rbase + g) * 128 + ((((2 * blk + (i >> 1)) ^ g) << 4) + ((i & 1) << 3));
-            const uint32_t ab = stage + kTmaBytes + ((rbase + g) * 4 + blk) * 4;
+            const uint32_t ab = ahat_base + aslot * kAhatBytes + ((rbase + g) * 4 + blk) * 4;
 #pragma unroll
             for (int t = 0; t < kTiles; ++t) {
                 const uint2 raw = lds64(wb + t * 8 * 128);
@@ -362,24 +358,40 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
                 for (int s = 0; s < 4; ++s)
                     mma_16816(acc[t], xa[2 * s], xc[2 * s], xa[2 * s + 1], xc[2 * s + 1], bw[2 * s], bw[2 * s + 1]);
             }
+            // the last warp to finish the stage refills its slot
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[slot]);
+            if (lane == 0) {
+                const uint32_t prev = atomicAdd(&done[slot], 1u);
+                if (prev == static_cast<uint32_t>(kConsumers * (j / kRing + 1) - 1) && j + kRing < nst) {
+                    issue_stage(ring + slot * kStageBytes, &tm_w, &tm_x, &tfull[slot], s0 + j + kRing, row0, true);
+                    issued[slot] = j / kRing + 1;
+                }
+            }
         }
-
-        // fold the consumer warps: red[blk][token][row] (the two row halves of a
-        // block land in disjoint rows of the same buffer)
-        __syncwarp();
-        named_bar_sync(1, 32 * kConsumers);  // every consumer is done with the ring
-        float* red = reinterpret_cast<float*>(ring) + blk * 16 * kRedPitch;
-#pragma unroll
-        for (int t = 0; t < kTiles; ++t) {
-            const int r = rbase + 8 * t + 2 * i;
-            *reinterpret_cast<float2*>(&red[g * kRedPitch + r]) = make_float2(acc[t][0], acc[t][1]);
-            *reinterpret_cast<float2*>(&red[(g + 8) * kRedPitch + r]) = make_float2(acc[t][2], acc[t][3]);
-        }
-        grid_dependency_wait();  // Y may still be in use by the preceding kernel
     }
-    if (timed_out) record_timeout(dev_status);
+    // the next kernel on the stream may start its prologue (its weight
+    // prefetch overlaps our epilogue)
+    grid_launch_dependents();
+
+    // fold the warps: red[blk][token][row] (the two row halves of a block
+    // land in disjoint rows of the same buffer)
+    timed_out = __syncthreads_or(timed_out);  // every warp is done with the ring
+    if (timed_out) {
+        // leave no copy in flight: wait (bounded) for every stage issued
+        if (threadIdx.x == 0) {
+            record_timeout(dev_status);
+            for (int s = 0; s < kRing; ++s)
+                if (issued[s] >= 0) mbar_wait(&tfull[s], issued[s] & 1);
+        }
+        __syncthreads();
+    }
+    float* red = reinterpret_cast<float*>(ring) + blk * 16 * kRedPitch;
+#pragma unroll
+    for (int t = 0; t < kTiles; ++t) {
+        const int r = rbase + 8 * t + 2 * i;
+        *reinterpret_cast<float2*>(&red[g * kRedPitch + r]) = make_float2(acc[t][0], acc[t][1]);
+        *reinterpret_cast<float2*>(&red[(g + 8) * kRedPitch + r]) = make_float2(acc[t][2], acc[t][3]);
+    }
     __syncthreads();
     const float* redf = reinterpret_cast<const float*>(ring);
     float4* part4 = reinterpret_cast<float4*>(ring) + 4 * 16 * kRedPitch / 4;
