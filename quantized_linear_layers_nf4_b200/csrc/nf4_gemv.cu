@@ -10,27 +10,33 @@
 //   Y[t, r] = sum_c X[t, c] * What[r, c],   What[r, c] = bf16(fp32(level[idx] * a_block)).
 //
 // The operation is HBM-bound: per weight 0.5 B of codes plus 1/64 B of absmax
-// code must stream from HBM.  Design (one CTA = 128 weight rows x a slice of k):
+// code must stream from HBM.  Design (one CTA = 128 weight rows x a slice of k,
+// eight warps, two CTAs per SM):
 //
-// * A producer warp streams 256-wide k stages through a 3-deep shared-memory
-//   ring with TMA (no multicast): a [128 rows x 128 B] tile of packed codes and
-//   the matching [16 tokens x 256] tile of X, both 128-byte swizzled so the
-//   consumers' reads are bank-conflict free.  Its 32 lanes also reconstruct the
-//   stage's absmax values (loaded one stage ahead, so their latency hides behind
-//   the ring).  mbarriers carry full/empty state; every wait is bounded.
-// * Eight consumer warps: warp w owns 64-block (w % 4) of every stage for 64
-//   of the 128 rows, so one X fragment serves 8 MMAs.  The multiply-adds run on the tensor
-//   cores (mma.sync m16n8k16, bf16 in, fp32 accumulate) with the 16 token slots
-//   as the MMA's M side (zero-filled beyond m) and 8 weight rows as its N side.
-//   Each lane owns 16 consecutive weights of a block row; the MMA k order is a
-//   permutation of the true k order applied identically to X and the weights.
+// * Rings in shared memory, filled by TMA (no multicast): 3 slots of packed
+//   codes [128 rows x 128 B] and 3 slots of X [16 tokens x 256], both 128-byte
+//   swizzled so that the fragment reads are bank-conflict free.  A warp copies
+//   its codes of a stage into registers first and then leaves the codes slot;
+//   the last warp out refills it at once, so the next load overlaps the decode.
+//   X slots are refilled the same way after the stage is done.  mbarriers carry
+//   the TMA byte counts; every wait is bounded.
+// * Reconstructed absmax a = fp32(fp32(fp32(q / 127) * s) + mu): every thread
+//   computes two of the stage's 512 values one stage ahead (its inputs are
+//   loaded three stages ahead) into a 4-deep table ring.
+// * Warp w owns rows 32 (w mod 4) .. + 31 and 64-blocks 2 (w div 4) + {0, 1} of
+//   every stage.  The multiply-adds run on the tensor cores (mma.sync m16n8k16,
+//   bf16 in, fp32 accumulate) with the 16 token slots as the MMA's M side
+//   (zero-filled beyond m) and 8 weight rows as its N side.  Each lane owns 16
+//   consecutive weights of a block row; the MMA k order is a permutation of the
+//   true k order applied identically to X and the weights.
 // * Decode: a 256-entry table maps a packed byte to the two fp32 levels it
 //   encodes (replicated 16x so a half-warp's lookups never share a bank); each
 //   level is multiplied by the block's reconstructed absmax in fp32 and rounded
 //   to bf16 -- the same values nf4_dequantize produces.
-// * Split-k: the CTAs of a thread-block cluster share a row tile and split k;
-//   their fp32 partials are added through distributed shared memory in a fixed
-//   rank order, so results are deterministic and no global scratch is needed.
+// * Split-k: the CTAs of a thread-block cluster share a row tile and split k.
+//   Each rank pushes the partial sums of the rows another rank owns into that
+//   rank's shared memory; the owner adds them in rank order, so results are
+//   deterministic and no global scratch is needed.
 #include "nf4_common.cuh"
 #include "nf4_internal.h"
 #include "nf4_ptx.cuh"
@@ -43,28 +49,32 @@ constexpr int kRows = 128;                       // weight rows per CTA
 constexpr int kStageK = 256;                     // k per pipeline stage
 constexpr int kRing = 3;                         // stages in flight per CTA
 constexpr int kConsumers = 8;                    // consumer warps
-constexpr int kTiles = 8;                        // 8-row MMA tiles per consumer warp (64 rows)
+constexpr int kTiles = 4;                        // 8-row MMA tiles per warp (32 rows) and block
 constexpr int kThreads = 32 * kConsumers;        // no dedicated producer warp
 constexpr int kWBytes = kRows * kStageK / 2;     // 16384: packed codes of a stage
 constexpr int kXBox = 16 * 64 * 2;               // 2048: X box of 16 tokens x 64 k (bf16)
 constexpr int kXBytes = 4 * kXBox;               // 8192
-constexpr int kTmaBytes = kWBytes + kXBytes;     // bytes a stage receives by TMA
-constexpr int kStageBytes = kTmaBytes;           // 24576 (keeps 1 KiB alignment)
 constexpr int kAring = 4;                        // reconstructed-absmax tables in flight
 constexpr int kAhatBytes = 4 * kRows * 4;        // 2048: one stage's table, [row][block]
 constexpr int kLutBytes = 16 * 256 * 8;          // 32768
-constexpr int kRingBytes = kRing * kStageBytes;
+constexpr int kXRingOff = kRing * kWBytes;       // codes ring first, then the X ring
+constexpr int kRingBytes = kRing * (kWBytes + kXBytes);
 constexpr int kAhatOff = kRingBytes;
 constexpr int kLutOff = kAhatOff + kAring * kAhatBytes;
 constexpr int kBarOff = kLutOff + kLutBytes;
 // two CTAs per SM: (113 KiB + 1 KiB reserved) x 2 within the SM's 228 KiB
-constexpr int kSmemBytes = kBarOff + (kRing + kAring) * 8 + 2 * kRing * 4;
-static_assert(kStageBytes % 1024 == 0, "stages keep the 1 KiB alignment the 128-byte swizzle needs");
+constexpr int kSmemBytes = kBarOff + (2 * kRing + kAring + 1) * 8 + 4 * kRing * 4;
+static_assert(kWBytes % 1024 == 0 && kXBytes % 1024 == 0, "slots keep the 1 KiB alignment the 128-byte swizzle needs");
 static_assert(kSmemBytes + 1024 <= 228 * 1024 / 2, "two CTAs fit on an SM");
 // Per-block partial sums are stored [token][row] with a padded token pitch so
 // that the 8 row groups of a warp write distinct banks.
 constexpr int kRedPitch = kRows + 8;
-static_assert(4 * 16 * kRedPitch * 4 + 16 * kRows * 4 <= kRingBytes, "reduction fits in the ring");
+// Epilogue buffers, all inside the (then idle) ring: the two per-block-pair
+// partials, the CTA's folded partial [token][row], and the split-k receive
+// area [sender][token][rows of this rank].
+constexpr int kPartOff = 2 * 16 * kRedPitch * 4;
+constexpr int kRecvOff = kPartOff + 16 * kRows * 4;
+static_assert(kRecvOff + 16 * kRows * 4 <= kRingBytes, "reduction fits in the ring");
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
@@ -73,6 +83,13 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
         "{%0,%1,%2,%3};\n"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Byte `b` (0..3) of `word` in the low 8 bits, zeros above (one byte permute).
+__device__ __forceinline__ uint32_t byte_of(uint32_t word, uint32_t b) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(d) : "r"(word), "r"(0x4440u | b));
+    return d;
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -187,15 +204,25 @@ __device__ __forceinline__ void store_ahat(uint32_t ahat_row, int half, const Ab
 
 constexpr int kPrefetch = 3;  // stages of absmax inputs in flight per thread
 
-// Loads W (and, once allowed, X) of stage `st` into ring slot `slot`.
-__device__ __forceinline__ void issue_stage(uint8_t* stage, const CUtensorMap* tm_w, const CUtensorMap* tm_x,
-                                            uint64_t* tfull, int st, int64_t row0, bool with_x) {
-    mbar_arrive_expect_tx(tfull, kTmaBytes);
-    tma_load_2d(stage, tm_w, st * (kStageK / 2), static_cast<int32_t>(row0), tfull);
-    if (with_x) {
+// Codes [128 rows x 128 B] of stage `st` into a codes slot.
+__device__ __forceinline__ void issue_w(uint8_t* dst, const CUtensorMap* tm_w, uint64_t* bar, int st, int64_t row0) {
+    mbar_arrive_expect_tx(bar, kWBytes);
+    tma_load_2d(dst, tm_w, st * (kStageK / 2), static_cast<int32_t>(row0), bar);
+}
+
+// X [16 tokens x 256] of stage `st` (4 boxes of 64 columns) into an X slot.
+__device__ __forceinline__ void issue_x(uint8_t* dst, const CUtensorMap* tm_x, uint64_t* bar, int st) {
+    mbar_arrive_expect_tx(bar, kXBytes);
 #pragma unroll
-        for (int b = 0; b < 4; ++b) tma_load_2d(stage + kWBytes + b * kXBox, tm_x, st * kStageK + 64 * b, 0, tfull);
-    }
+    for (int b = 0; b < 4; ++b) tma_load_2d(dst + b * kXBox, tm_x, st * kStageK + 64 * b, 0, bar);
+}
+
+// Counts a warp out of a ring slot; acquire-release so that the warp's reads
+// of the slot are ordered before the refill that the last warp issues.
+__device__ __forceinline__ uint32_t slot_leave(uint32_t* counter) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;" : "=r"(old) : "r"(smem_u32(counter)) : "memory");
+    return old;
 }
 
 template <bool kBf16Out, bool kM16>
@@ -213,12 +240,17 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
             atomicExch(dev_status, -9 /* NF4_ERR_UNSUPPORTED_DEVICE */);
         return;
     }
-    uint8_t* ring = smem_raw;
+    uint8_t* ring = smem_raw;                 // codes slots, then X slots
+    uint8_t* xring = smem_raw + kXRingOff;
     float2* lut = reinterpret_cast<float2*>(smem_raw + kLutOff);
-    uint64_t* tfull = reinterpret_cast<uint64_t*>(smem_raw + kBarOff);  // TMA bytes of a stage landed
-    uint64_t* afull = tfull + kRing;                                     // absmax table of a stage written
-    uint32_t* done = reinterpret_cast<uint32_t*>(afull + kAring);        // warps finished, per ring slot
-    int* issued = reinterpret_cast<int*>(done + kRing);                  // last use issued, per ring slot
+    uint64_t* wfull = reinterpret_cast<uint64_t*>(smem_raw + kBarOff);  // codes of a stage landed
+    uint64_t* xfull = wfull + kRing;                                     // X of a stage landed
+    uint64_t* afull = xfull + kRing;                                     // absmax table of a stage written
+    uint64_t* rfull = afull + kAring;                                    // split-k partials received
+    uint32_t* wdone = reinterpret_cast<uint32_t*>(rfull + 1);            // warps out of a codes slot
+    uint32_t* xdone = wdone + kRing;                                     // warps out of an X slot
+    int* wissued = reinterpret_cast<int*>(xdone + kRing);                // last use issued per codes slot
+    int* xissued = wissued + kRing;                                      // last use issued per X slot
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -233,19 +265,25 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kRing; ++s) {
-            mbar_init(&tfull[s], 1);
-            done[s] = 0;
-            issued[s] = -1;
+            mbar_init(&wfull[s], 1);
+            mbar_init(&xfull[s], 1);
+            wdone[s] = xdone[s] = 0;
+            wissued[s] = xissued[s] = -1;
         }
         for (int s = 0; s < kAring; ++s) mbar_init(&afull[s], kConsumers);
+        mbar_init(rfull, cluster > 1 ? cluster - 1 : 1);
         fence_mbar_init();
         prefetch_tensormap(&tm_w);
         prefetch_tensormap(&tm_x);
         if (!weights_early) grid_dependency_wait();
         // the weights of the first stages start streaming before anything else
         for (int j = 0; j < n_pre; ++j) {
-            issue_stage(ring + j * kStageBytes, &tm_w, &tm_x, &tfull[j], s0 + j, row0, !weights_early);
-            issued[j] = 0;
+            issue_w(ring + j * kWBytes, &tm_w, &wfull[j], s0 + j, row0);
+            wissued[j] = 0;
+            if (!weights_early) {
+                issue_x(xring + j * kXBytes, &tm_x, &xfull[j], s0 + j);
+                xissued[j] = 0;
+            }
         }
     }
 
@@ -264,23 +302,34 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
     const float mu = __ldg(mu_ptr);
 
     // byte -> (level of high nibble, level of low nibble), 16 copies so that
-    // the 16 lanes of a half-warp always read distinct banks
-    // (consecutive threads write consecutive 16-byte chunks: 2 copies each)
-    for (int c = threadIdx.x; c < kLutBytes / 16; c += kThreads) {
-        const int b = c >> 3;
-        const uint32_t hi = __float_as_uint(kLevels[b >> 4]), lo = __float_as_uint(kLevels[b & 15]);
-        sts128(smem_u32(lut) + 16u * c, make_uint4(hi, lo, hi, lo));
+    // the 16 lanes of a half-warp always read distinct banks.  Thread t writes
+    // 16-byte chunks c = t + 256 it (two copies of byte c / 8): its low nibble
+    // (t / 8) mod 16 is fixed and its high nibble is 2 it + t / 128, so every
+    // level comes from an immediate and the build touches no memory but the table.
+    static_assert(kLutBytes / 16 == 8 * kThreads, "eight chunks per thread");
+    {
+        constexpr float kLv[16] = NF4_LEVELS_INIT;
+        const int lo_idx = (threadIdx.x >> 3) & 15;
+        float lo = kLv[0];
+#pragma unroll
+        for (int v = 1; v < 16; ++v) lo = (lo_idx == v) ? kLv[v] : lo;
+        const bool odd = (threadIdx.x >> 7) != 0;
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+            const float hi = odd ? kLv[2 * it + 1] : kLv[2 * it];
+            sts128(smem_u32(lut) + 16u * (threadIdx.x + kThreads * it),
+                   make_uint4(__float_as_uint(hi), __float_as_uint(lo), __float_as_uint(hi), __float_as_uint(lo)));
+        }
     }
     __syncthreads();  // barriers initialised, LUT written
 
     if (threadIdx.x == 0 && weights_early) {
         // weights are in flight; X (the preceding kernel's output) only after it finished
         grid_dependency_wait();
-        for (int j = 0; j < n_pre; ++j)
-#pragma unroll
-            for (int b = 0; b < 4; ++b)
-                tma_load_2d(ring + j * kStageBytes + kWBytes + b * kXBox, &tm_x, (s0 + j) * kStageK + 64 * b, 0,
-                            &tfull[j]);
+        for (int j = 0; j < n_pre; ++j) {
+            issue_x(xring + j * kXBytes, &tm_x, &xfull[j], s0 + j);
+            xissued[j] = 0;
+        }
     }
     // the absmax table of the first stage
     const uint32_t ahat_base = smem_u32(smem_raw + kAhatOff);
@@ -295,8 +344,8 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
 
     const int g = lane >> 2;
     const int i = lane & 3;
-    const int blk = warp & 3;            // 64-block of the stage
-    const int rbase = (warp >> 2) * 64;  // first of this warp's 64 rows
+    const int bpair = warp >> 2;         // the warp's two 64-blocks of the stage: 2 bpair, 2 bpair + 1
+    const int rbase = (warp & 3) * 32;   // first of this warp's 32 rows
     const uint32_t lut_lane = smem_u32(lut) + (lane & 15) * 8u;
     float acc[kTiles][4];
 #pragma unroll
@@ -324,48 +373,70 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
             }
             // every lane polls; the warp proceeds only if all of them saw the stage
             const int aslot = j % kAring;
-            if (!__all_sync(kFull, mbar_wait(&tfull[slot], (j / kRing) & 1) &&
-                                       mbar_wait(&afull[aslot], (j / kAring) & 1))) {
+            const uint32_t par = (j / kRing) & 1;
+            if (!__all_sync(kFull, mbar_wait(&wfull[slot], par) && mbar_wait(&afull[aslot], (j / kAring) & 1))) {
                 timed_out = true;
                 break;
             }
-            const uint32_t stage = smem_u32(ring + slot * kStageBytes);
-            // X fragments: tokens g and g + 8, k = 16 i .. 16 i + 15 of this warp's block
-            const uint32_t xb = stage + kWBytes + blk * kXBox;
-            const uint4 xa0 = lds128(xb + g * 128 + (((2 * i) ^ g) << 4));
-            const uint4 xa1 = lds128(xb + g * 128 + (((2 * i + 1) ^ g) << 4));
-            uint4 xc0 = make_uint4(0u, 0u, 0u, 0u), xc1 = xc0;
-            if (kM16) {
-                xc0 = lds128(xb + (g + 8) * 128 + (((2 * i) ^ g) << 4));
-                xc1 = lds128(xb + (g + 8) * 128 + (((2 * i + 1) ^ g) << 4));
+            // This warp's codes of the stage into registers (rows rbase + 8 t + g,
+            // 8 bytes per lane = 16 consecutive weights of a block), then leave the
+            // codes slot: the last warp out refills it while the decode runs.
+            const uint32_t wstage = smem_u32(ring + slot * kWBytes);
+            uint2 raw[2][kTiles];
+#pragma unroll
+            for (int bb = 0; bb < 2; ++bb) {
+                const uint32_t wb = wstage + (rbase + g) * 128 +
+                                    ((((2 * (2 * bpair + bb) + (i >> 1)) ^ g) << 4) + ((i & 1) << 3));
+#pragma unroll
+                for (int t = 0; t < kTiles; ++t) raw[bb][t] = lds64(wb + t * 8 * 128);
             }
-            const uint32_t xa[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
-            const uint32_t xc[8] = {xc0.x, xc0.y, xc0.z, xc0.w, xc1.x, xc1.y, xc1.z, xc1.w};
-            const uint32_t wb = stage + (rbase + g) * 128 + ((((2 * blk + (i >> 1)) ^ g) << 4) + ((i & 1) << 3));
-            const uint32_t ab = ahat_base + aslot * kAhatBytes + ((rbase + g) * 4 + blk) * 4;
-#pragma unroll
-            for (int t = 0; t < kTiles; ++t) {
-                const uint2 raw = lds64(wb + t * 8 * 128);
-                const uint64_t aa = dup_f32x2(lds_f32(ab + 128 * t));
-                uint32_t bw[8];
-#pragma unroll
-                for (int b = 0; b < 8; ++b) {
-                    const uint32_t word = (b < 4) ? raw.x : raw.y;
-                    const uint32_t byte = (word >> (8 * (b & 3))) & 0xffu;
-                    bw[b] = scale_pack(lds_b64(lut_lane + byte * 128u), aa);
-                }
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_16816(acc[t], xa[2 * s], xc[2 * s], xa[2 * s + 1], xc[2 * s + 1], bw[2 * s], bw[2 * s + 1]);
-            }
-            // the last warp to finish the stage refills its slot
             __syncwarp();
-            if (lane == 0) {
-                const uint32_t prev = atomicAdd(&done[slot], 1u);
-                if (prev == static_cast<uint32_t>(kConsumers * (j / kRing + 1) - 1) && j + kRing < nst) {
-                    issue_stage(ring + slot * kStageBytes, &tm_w, &tm_x, &tfull[slot], s0 + j + kRing, row0, true);
-                    issued[slot] = j / kRing + 1;
+            if (lane == 0 && slot_leave(&wdone[slot]) == static_cast<uint32_t>(kConsumers * (j / kRing + 1) - 1) &&
+                j + kRing < nst) {
+                issue_w(ring + slot * kWBytes, &tm_w, &wfull[slot], s0 + j + kRing, row0);
+                wissued[slot] = j / kRing + 1;
+            }
+            if (!__all_sync(kFull, mbar_wait(&xfull[slot], par))) {
+                timed_out = true;
+                break;
+            }
+            const uint32_t xstage = smem_u32(xring + slot * kXBytes);
+#pragma unroll
+            for (int bb = 0; bb < 2; ++bb) {
+                const int blk = 2 * bpair + bb;
+                // X fragments: tokens g and g + 8, k = 16 i .. 16 i + 15 of block blk
+                const uint32_t xb = xstage + blk * kXBox;
+                const uint4 xa0 = lds128(xb + g * 128 + (((2 * i) ^ g) << 4));
+                const uint4 xa1 = lds128(xb + g * 128 + (((2 * i + 1) ^ g) << 4));
+                uint4 xc0 = make_uint4(0u, 0u, 0u, 0u), xc1 = xc0;
+                if (kM16) {
+                    xc0 = lds128(xb + (g + 8) * 128 + (((2 * i) ^ g) << 4));
+                    xc1 = lds128(xb + (g + 8) * 128 + (((2 * i + 1) ^ g) << 4));
                 }
+                const uint32_t xa[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
+                const uint32_t xc[8] = {xc0.x, xc0.y, xc0.z, xc0.w, xc1.x, xc1.y, xc1.z, xc1.w};
+                const uint32_t ab = ahat_base + aslot * kAhatBytes + ((rbase + g) * 4 + blk) * 4;
+#pragma unroll
+                for (int t = 0; t < kTiles; ++t) {
+                    const uint64_t aa = dup_f32x2(lds_f32(ab + 128 * t));
+                    uint32_t bw[8];
+#pragma unroll
+                    for (int b = 0; b < 8; ++b) {
+                        const uint32_t word = (b < 4) ? raw[bb][t].x : raw[bb][t].y;
+                        bw[b] = scale_pack(lds_b64(lut_lane + (byte_of(word, b & 3) << 7)), aa);
+                    }
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        mma_16816(acc[t], xa[2 * s], xc[2 * s], xa[2 * s + 1], xc[2 * s + 1], bw[2 * s],
+                                  bw[2 * s + 1]);
+                }
+            }
+            // the last warp out of the X slot refills it
+            __syncwarp();
+            if (lane == 0 && slot_leave(&xdone[slot]) == static_cast<uint32_t>(kConsumers * (j / kRing + 1) - 1) &&
+                j + kRing < nst) {
+                issue_x(xring + slot * kXBytes, &tm_x, &xfull[slot], s0 + j + kRing);
+                xissued[slot] = j / kRing + 1;
             }
         }
     }
@@ -373,19 +444,21 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
     // prefetch overlaps our epilogue)
     grid_launch_dependents();
 
-    // fold the warps: red[blk][token][row] (the two row halves of a block
-    // land in disjoint rows of the same buffer)
+    // fold the warps: red[bpair][token][row] (the four row groups of a block
+    // pair land in disjoint rows of the same buffer)
     timed_out = __syncthreads_or(timed_out);  // every warp is done with the ring
     if (timed_out) {
         // leave no copy in flight: wait (bounded) for every stage issued
         if (threadIdx.x == 0) {
             record_timeout(dev_status);
-            for (int s = 0; s < kRing; ++s)
-                if (issued[s] >= 0) mbar_wait(&tfull[s], issued[s] & 1);
+            for (int s = 0; s < kRing; ++s) {
+                if (wissued[s] >= 0) mbar_wait(&wfull[s], wissued[s] & 1);
+                if (xissued[s] >= 0) mbar_wait(&xfull[s], xissued[s] & 1);
+            }
         }
         __syncthreads();
     }
-    float* red = reinterpret_cast<float*>(ring) + blk * 16 * kRedPitch;
+    float* red = reinterpret_cast<float*>(ring) + bpair * 16 * kRedPitch;
 #pragma unroll
     for (int t = 0; t < kTiles; ++t) {
         const int r = rbase + 8 * t + 2 * i;
@@ -394,41 +467,59 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
     }
     __syncthreads();
     const float* redf = reinterpret_cast<const float*>(ring);
-    float4* part4 = reinterpret_cast<float4*>(ring) + 4 * 16 * kRedPitch / 4;
+    float4* part4 = reinterpret_cast<float4*>(ring + kPartOff);
     constexpr int kQ = 16 * kRows / 4;  // float4s of partial sums per CTA
     constexpr int kB = 16 * kRedPitch;  // floats per block buffer
     for (int e = threadIdx.x; e < kQ; e += kThreads) {
         const int off = (e / (kRows / 4)) * kRedPitch + 4 * (e % (kRows / 4));
         const float4 a = *reinterpret_cast<const float4*>(redf + off);
         const float4 b = *reinterpret_cast<const float4*>(redf + kB + off);
-        const float4 c = *reinterpret_cast<const float4*>(redf + 2 * kB + off);
-        const float4 d = *reinterpret_cast<const float4*>(redf + 3 * kB + off);
-        part4[e] = make_float4(((a.x + b.x) + c.x) + d.x, ((a.y + b.y) + c.y) + d.y,
-                               ((a.z + b.z) + c.z) + d.z, ((a.w + b.w) + c.w) + d.w);
+        part4[e] = make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
     }
 
-    // cluster split-k: rank r adds rows [r * 128 / C, (r + 1) * 128 / C) over all ranks in rank order
-    cluster_sync();
+    // Cluster split-k: rank q owns rows [q * 128 / C, (q + 1) * 128 / C).  Every
+    // rank sends the partials of q's rows into q's receive area and arrives on
+    // q's barrier; q adds the C partials in rank order and writes Y.  Nothing
+    // reads another CTA's memory, so no rank waits for the others to finish.
     const int rows_per_rank = kRows / cluster;
     const int quads = rows_per_rank / 4;
     const int r_lo = rank * rows_per_rank;
-    const uint32_t part_addr = smem_u32(part4);
+    const uint32_t recv_addr = smem_u32(ring + kRecvOff);
+    if (cluster > 1) {
+        cluster_sync();  // every rank is done with its ring: receive areas are free
+        for (int e = threadIdx.x; e < m * (kRows / 4); e += kThreads) {
+            const int tok = e / (kRows / 4);
+            const int r = 4 * (e % (kRows / 4));
+            const int q = r / rows_per_rank;
+            if (q == rank) continue;
+            const uint32_t off =
+                static_cast<uint32_t>(((rank * 16 + tok) * rows_per_rank + (r - q * rows_per_rank)) * 4);
+            st_shared_cluster_f32x4(map_shared_rank(recv_addr + off, q), part4[tok * (kRows / 4) + r / 4]);
+        }
+        fence_acq_rel_cluster();
+        __syncthreads();
+        if (threadIdx.x < cluster && threadIdx.x != rank)
+            mbar_arrive_remote(map_shared_rank(smem_u32(rfull), threadIdx.x));
+        if (!mbar_wait_cluster(rfull, 0)) {
+            record_timeout(dev_status);
+            return;
+        }
+    }
     for (int e = threadIdx.x; e < m * quads; e += kThreads) {
         const int tok = e / quads;
-        const int r = r_lo + 4 * (e % quads);
-        const uint32_t off = static_cast<uint32_t>((tok * kRows + r) * 4);
-        float4 v[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-            if (q < cluster) v[q] = ld_shared_cluster_f32x4(map_shared_rank(part_addr + off, q));
-        float4 sum = v[0];
-#pragma unroll
-        for (int q = 1; q < 8; ++q)
-            if (q < cluster) sum = make_float4(sum.x + v[q].x, sum.y + v[q].y, sum.z + v[q].z, sum.w + v[q].w);
+        const int rr = 4 * (e % quads);
+        const float4 own = part4[tok * (kRows / 4) + (r_lo + rr) / 4];
+        float4 sum = own;
+        for (int q = 0; q < cluster; ++q) {
+            const float4 v = (q == rank) ? own
+                                         : *reinterpret_cast<const float4*>(
+                                               ring + kRecvOff + ((q * 16 + tok) * rows_per_rank + rr) * 4);
+            sum = (q == 0) ? v : make_float4(sum.x + v.x, sum.y + v.y, sum.z + v.z, sum.w + v.w);
+        }
         const float o[4] = {sum.x, sum.y, sum.z, sum.w};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            const int64_t grow = row0 + r + c;
+            const int64_t grow = row0 + r_lo + rr + c;
             if (grow >= n) break;
             if (kBf16Out)
                 reinterpret_cast<__nv_bfloat16*>(Y)[static_cast<int64_t>(tok) * n + grow] = __float2bfloat16_rn(o[c]);
@@ -436,7 +527,6 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
                 reinterpret_cast<float*>(Y)[static_cast<int64_t>(tok) * n + grow] = o[c];
         }
     }
-    cluster_sync();  // keep this CTA's partials alive until every rank has read them
 }
 
 }  // namespace gemv
