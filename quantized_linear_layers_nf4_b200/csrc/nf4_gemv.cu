@@ -10,33 +10,27 @@
 //   Y[t, r] = sum_c X[t, c] * What[r, c],   What[r, c] = bf16(fp32(level[idx] * a_block)).
 //
 // The operation is HBM-bound: per weight 0.5 B of codes plus 1/64 B of absmax
-// code must stream from HBM.  Design (one CTA = 128 weight rows x a slice of k,
-// eight warps, two CTAs per SM):
+// code must stream from HBM.  Design (one CTA = 128 weight rows x a slice of k):
 //
-// * Rings in shared memory, filled by TMA (no multicast): 3 slots of packed
-//   codes [128 rows x 128 B] and 3 slots of X [16 tokens x 256], both 128-byte
-//   swizzled so that the fragment reads are bank-conflict free.  A warp copies
-//   its codes of a stage into registers first and then leaves the codes slot;
-//   the last warp out refills it at once, so the next load overlaps the decode.
-//   X slots are refilled the same way after the stage is done.  mbarriers carry
-//   the TMA byte counts; every wait is bounded.
-// * Reconstructed absmax a = fp32(fp32(fp32(q / 127) * s) + mu): every thread
-//   computes two of the stage's 512 values one stage ahead (its inputs are
-//   loaded three stages ahead) into a 4-deep table ring.
-// * Warp w owns rows 32 (w mod 4) .. + 31 and 64-blocks 2 (w div 4) + {0, 1} of
-//   every stage.  The multiply-adds run on the tensor cores (mma.sync m16n8k16,
-//   bf16 in, fp32 accumulate) with the 16 token slots as the MMA's M side
-//   (zero-filled beyond m) and 8 weight rows as its N side.  Each lane owns 16
-//   consecutive weights of a block row; the MMA k order is a permutation of the
-//   true k order applied identically to X and the weights.
+// * A producer warp streams 256-wide k stages through a 3-deep shared-memory
+//   ring with TMA (no multicast): a [128 rows x 128 B] tile of packed codes and
+//   the matching [16 tokens x 256] tile of X, both 128-byte swizzled so the
+//   consumers' reads are bank-conflict free.  Its 32 lanes also reconstruct the
+//   stage's absmax values (loaded one stage ahead, so their latency hides behind
+//   the ring).  mbarriers carry full/empty state; every wait is bounded.
+// * Eight consumer warps: warp w owns 64-block (w % 4) of every stage for 64
+//   of the 128 rows, so one X fragment serves 8 MMAs.  The multiply-adds run on the tensor
+//   cores (mma.sync m16n8k16, bf16 in, fp32 accumulate) with the 16 token slots
+//   as the MMA's M side (zero-filled beyond m) and 8 weight rows as its N side.
+//   Each lane owns 16 consecutive weights of a block row; the MMA k order is a
+//   permutation of the true k order applied identically to X and the weights.
 // * Decode: a 256-entry table maps a packed byte to the two fp32 levels it
 //   encodes (replicated 16x so a half-warp's lookups never share a bank); each
 //   level is multiplied by the block's reconstructed absmax in fp32 and rounded
 //   to bf16 -- the same values nf4_dequantize produces.
-// * Split-k: the CTAs of a thread-block cluster share a row tile and split k.
-//   Each rank pushes the partial sums of the rows another rank owns into that
-//   rank's shared memory; the owner adds them in rank order, so results are
-//   deterministic and no global scratch is needed.
+// * Split-k: the CTAs of a thread-block cluster share a row tile and split k;
+//   their fp32 partials are added through distributed shared memory in a fixed
+//   rank order, so results are deterministic and no global scratch is needed.
 #include "nf4_common.cuh"
 #include "nf4_internal.h"
 #include "nf4_ptx.cuh"
@@ -49,32 +43,22 @@ constexpr int kRows = 128;                       // weight rows per CTA
 constexpr int kStageK = 256;                     // k per pipeline stage
 constexpr int kRing = 3;                         // stages in flight per CTA
 constexpr int kConsumers = 8;                    // consumer warps
-constexpr int kTiles = 4;                        // 8-row MMA tiles per warp (32 rows) and block
-constexpr int kThreads = 32 * kConsumers;        // no dedicated producer warp
+constexpr int kTiles = 8;                        // 8-row MMA tiles per consumer warp (64 rows)
+constexpr int kThreads = 32 * (kConsumers + 1);  // + one producer warp
 constexpr int kWBytes = kRows * kStageK / 2;     // 16384: packed codes of a stage
 constexpr int kXBox = 16 * 64 * 2;               // 2048: X box of 16 tokens x 64 k (bf16)
 constexpr int kXBytes = 4 * kXBox;               // 8192
-constexpr int kAring = 4;                        // reconstructed-absmax tables in flight
-constexpr int kAhatBytes = 4 * kRows * 4;        // 2048: one stage's table, [row][block]
+constexpr int kTmaBytes = kWBytes + kXBytes;     // bytes a stage receives by TMA
+constexpr int kAhatBytes = 4 * kRows * 4;        // 2048: reconstructed absmax, [row][block]
+constexpr int kStageBytes = kTmaBytes + kAhatBytes;  // 26624 = 26 KiB (keeps 1 KiB alignment)
 constexpr int kLutBytes = 16 * 256 * 8;          // 32768
-constexpr int kXRingOff = kRing * kWBytes;       // codes ring first, then the X ring
-constexpr int kRingBytes = kRing * (kWBytes + kXBytes);
-constexpr int kAhatOff = kRingBytes;
-constexpr int kLutOff = kAhatOff + kAring * kAhatBytes;
-constexpr int kBarOff = kLutOff + kLutBytes;
-// two CTAs per SM: (113 KiB + 1 KiB reserved) x 2 within the SM's 228 KiB
-constexpr int kSmemBytes = kBarOff + (2 * kRing + kAring + 1) * 8 + 4 * kRing * 4;
-static_assert(kWBytes % 1024 == 0 && kXBytes % 1024 == 0, "slots keep the 1 KiB alignment the 128-byte swizzle needs");
-static_assert(kSmemBytes + 1024 <= 228 * 1024 / 2, "two CTAs fit on an SM");
+constexpr int kRingBytes = kRing * kStageBytes;
+constexpr int kSmemBytes = 1024 /*alignment slack*/ + kRingBytes + kLutBytes + 2 * kRing * 8;
+static_assert(kStageBytes % 1024 == 0, "stages keep the 1 KiB alignment the 128-byte swizzle needs");
 // Per-block partial sums are stored [token][row] with a padded token pitch so
 // that the 8 row groups of a warp write distinct banks.
 constexpr int kRedPitch = kRows + 8;
-// Epilogue buffers, all inside the (then idle) ring: the two per-block-pair
-// partials, the CTA's folded partial [token][row], and the split-k receive
-// area [sender][token][rows of this rank].
-constexpr int kPartOff = 2 * 16 * kRedPitch * 4;
-constexpr int kRecvOff = kPartOff + 16 * kRows * 4;
-static_assert(kRecvOff + 16 * kRows * 4 <= kRingBytes, "reduction fits in the ring");
+static_assert(4 * 16 * kRedPitch * 4 + 16 * kRows * 4 <= kRingBytes, "reduction fits in the ring");
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
@@ -141,89 +125,67 @@ __device__ __forceinline__ uint32_t scale_pack(uint64_t levels, uint64_t aa) {
     return out;
 }
 
-// Reconstructed-absmax inputs of one stage for one thread.  Thread t owns row
-// (t mod 128) of the tile and blocks 2 (t div 128) + {0, 1} of the stage: the
-// row's 4 int8 codes of the stage packed in one word, and the
-// double-quantization scales of the thread's two blocks.
+// The producer's per-stage absmax inputs.  Lane l owns rows l + 32 u (u = 0..3)
+// and the stage's 4 blocks of each: the 4 int8 codes of a row packed in one
+// word, and the (at most two) double-quantization scales its 4 blocks use.
 struct AbsmaxIn {
-    uint32_t q;
-    float s0, s1;
+    uint32_t q[4];
+    float s_lo[4], s_hi[4];
 };
 
 __device__ __forceinline__ void load_absmax_in(AbsmaxIn& a, const int8_t* __restrict__ absmax_q,
-                                               const float* __restrict__ absmax_scale, int64_t grow, int half,
-                                               int st, int64_t n, int64_t kblocks, bool aligned4) {
-    const int64_t kb = static_cast<int64_t>(st) * 4;
+                                               const float* __restrict__ absmax_scale, int64_t row0,
+                                               int lane, int st, int64_t n, int64_t kblocks,
+                                               bool aligned4) {
+    const int64_t kb0 = static_cast<int64_t>(st) * 4;
     if (aligned4) {
         // k % 256 == 0 and an aligned code array: a row's 4 codes of a stage are
         // one aligned word.  Every load is unconditional (rows past n are
-        // clamped; their results are never stored), so nothing waits for it
-        // until the stage is used.
-        const int64_t r = grow < n ? grow : n - 1;
-        const int64_t b0 = r * kblocks + kb + 2 * half;
-        a.q = __ldg(reinterpret_cast<const uint32_t*>(absmax_q + (b0 - 2 * half)));
-        a.s0 = __ldg(absmax_scale + (b0 >> 8));
-        a.s1 = __ldg(absmax_scale + ((b0 + 1) >> 8));
+        // clamped; their results are never stored) and lands directly in its
+        // field, so nothing waits for it until the stage is used.
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            int64_t grow = row0 + lane + 32 * u;
+            grow = grow < n ? grow : n - 1;
+            const int64_t b0 = grow * kblocks + kb0;
+            a.q[u] = __ldg(reinterpret_cast<const uint32_t*>(absmax_q + b0));
+            a.s_lo[u] = __ldg(absmax_scale + (b0 >> 8));
+            a.s_hi[u] = __ldg(absmax_scale + ((b0 + 3) >> 8));
+        }
         return;
     }
-    // general shapes: gather the codes byte by byte; blocks past k get q = 0
-    uint32_t q = 0;
-    float s0 = 0.0f, s1 = 0.0f;
-    if (grow < n) {
-        const int64_t b0 = grow * kblocks + kb;
-        const int64_t nvalid = kblocks - kb;  // >= 1
+    // general shapes: gather the codes byte by byte (stalls, but correct)
 #pragma unroll
-        for (int b = 0; b < 4; ++b)
-            if (b < nvalid) q |= static_cast<uint32_t>(static_cast<uint8_t>(__ldg(absmax_q + b0 + b))) << (8 * b);
-        const int64_t last = b0 + (nvalid < 4 ? nvalid : 4) - 1;
-        const int64_t ba = b0 + 2 * half, bb = ba + 1;
-        s0 = __ldg(absmax_scale + ((ba < last ? ba : last) >> 8));
-        s1 = __ldg(absmax_scale + ((bb < last ? bb : last) >> 8));
+    for (int u = 0; u < 4; ++u) {
+        const int64_t grow = row0 + lane + 32 * u;
+        uint32_t q = 0;
+        float lo = 0.0f, hi = 0.0f;
+        if (grow < n) {
+            const int64_t b0 = grow * kblocks + kb0;
+            const int64_t nvalid = kblocks - kb0;  // >= 1
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                if (b < nvalid)
+                    q |= static_cast<uint32_t>(static_cast<uint8_t>(__ldg(absmax_q + b0 + b))) << (8 * b);
+            const int64_t blast = b0 + (nvalid < 4 ? nvalid : 4) - 1;
+            lo = __ldg(absmax_scale + (b0 >> 8));
+            hi = __ldg(absmax_scale + (blast >> 8));
+        }
+        a.q[u] = q;
+        a.s_lo[u] = lo;
+        a.s_hi[u] = hi;
     }
-    a.q = q;
-    a.s0 = s0;
-    a.s1 = s1;
 }
 
 // Keeps the compiler from hoisting work that uses `a` above the point where
 // this is called (the values pass through an opaque asm).
 __device__ __forceinline__ void pin(AbsmaxIn& a) {
-    asm volatile("" : "+r"(a.q), "+f"(a.s0), "+f"(a.s1));
-}
-
-// a = fp32(fp32(fp32(q / 127) * s) + mu) for the thread's two blocks, stored
-// to the stage's [row][block] table.
-__device__ __forceinline__ void store_ahat(uint32_t ahat_row, int half, const AbsmaxIn& a, float mu) {
-    const uint32_t qq = a.q >> (16 * half);
-    const float q0 = static_cast<float>(static_cast<int8_t>(qq & 0xffu));
-    const float q1 = static_cast<float>(static_cast<int8_t>((qq >> 8) & 0xffu));
-    const float a0 = __fadd_rn(__fmul_rn(div127(q0), a.s0), mu);
-    const float a1 = __fadd_rn(__fmul_rn(div127(q1), a.s1), mu);
-    asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(ahat_row + 8u * half), "f"(a0), "f"(a1) : "memory");
-}
-
-constexpr int kPrefetch = 3;  // stages of absmax inputs in flight per thread
-
-// Codes [128 rows x 128 B] of stage `st` into a codes slot.
-__device__ __forceinline__ void issue_w(uint8_t* dst, const CUtensorMap* tm_w, uint64_t* bar, int st, int64_t row0) {
-    mbar_arrive_expect_tx(bar, kWBytes);
-    tma_load_2d(dst, tm_w, st * (kStageK / 2), static_cast<int32_t>(row0), bar);
-}
-
-// X [16 tokens x 256] of stage `st` (4 boxes of 64 columns) into an X slot.
-__device__ __forceinline__ void issue_x(uint8_t* dst, const CUtensorMap* tm_x, uint64_t* bar, int st) {
-    mbar_arrive_expect_tx(bar, kXBytes);
 #pragma unroll
-    for (int b = 0; b < 4; ++b) tma_load_2d(dst + b * kXBox, tm_x, st * kStageK + 64 * b, 0, bar);
+    for (int u = 0; u < 4; ++u)
+        asm volatile("" : "+r"(a.q[u]), "+f"(a.s_lo[u]), "+f"(a.s_hi[u]));
 }
 
-// Counts a warp out of a ring slot; acquire-release so that the warp's reads
-// of the slot are ordered before the refill that the last warp issues.
-__device__ __forceinline__ uint32_t slot_leave(uint32_t* counter) {
-    uint32_t old;
-    asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;" : "=r"(old) : "r"(smem_u32(counter)) : "memory");
-    return old;
-}
+constexpr int kPrefetch = 3;  // stages of absmax inputs in flight per producer lane
 
 template <bool kBf16Out, bool kM16>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -231,26 +193,12 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
            const int8_t* __restrict__ absmax_q, const float* __restrict__ absmax_scale,
            const float* __restrict__ mu_ptr, int m, int64_t n, int64_t k, int cluster, int weights_early,
            void* __restrict__ Y, int32_t* __restrict__ dev_status) {
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    // The 128-byte swizzle needs 1 KiB-aligned stages.  The dynamic window is
-    // declared so aligned; should a platform place it otherwise, every CTA
-    // sees the same base and returns here, before any barrier, with an error.
-    if (smem_u32(smem_raw) & 1023u) {
-        if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && dev_status)
-            atomicExch(dev_status, -9 /* NF4_ERR_UNSUPPORTED_DEVICE */);
-        return;
-    }
-    uint8_t* ring = smem_raw;                 // codes slots, then X slots
-    uint8_t* xring = smem_raw + kXRingOff;
-    float2* lut = reinterpret_cast<float2*>(smem_raw + kLutOff);
-    uint64_t* wfull = reinterpret_cast<uint64_t*>(smem_raw + kBarOff);  // codes of a stage landed
-    uint64_t* xfull = wfull + kRing;                                     // X of a stage landed
-    uint64_t* afull = xfull + kRing;                                     // absmax table of a stage written
-    uint64_t* rfull = afull + kAring;                                    // split-k partials received
-    uint32_t* wdone = reinterpret_cast<uint32_t*>(rfull + 1);            // warps out of a codes slot
-    uint32_t* xdone = wdone + kRing;                                     // warps out of an X slot
-    int* wissued = reinterpret_cast<int*>(xdone + kRing);                // last use issued per codes slot
-    int* xissued = wissued + kRing;                                      // last use issued per X slot
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* ring = smem;
+    float2* lut = reinterpret_cast<float2*>(smem + kRingBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRingBytes + kLutBytes);
+    uint64_t* empty = full + kRing;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -260,266 +208,234 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
     const int rank = static_cast<int>(blockIdx.y);
     const int s0 = static_cast<int>((static_cast<int64_t>(n_stages) * rank) / cluster);
     const int s1 = static_cast<int>((static_cast<int64_t>(n_stages) * (rank + 1)) / cluster);
-    const int nst = s1 - s0;  // >= 1
-    const int n_pre = nst < kRing ? nst : kRing;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kRing; ++s) {
-            mbar_init(&wfull[s], 1);
-            mbar_init(&xfull[s], 1);
-            wdone[s] = xdone[s] = 0;
-            wissued[s] = xissued[s] = -1;
+            mbar_init(&full[s], 2);   // the TMA bytes' arrive + the absmax-ready arrive
+            mbar_init(&empty[s], kConsumers);
         }
-        for (int s = 0; s < kAring; ++s) mbar_init(&afull[s], kConsumers);
-        mbar_init(rfull, cluster > 1 ? cluster - 1 : 1);
         fence_mbar_init();
-        prefetch_tensormap(&tm_w);
-        prefetch_tensormap(&tm_x);
-        if (!weights_early) grid_dependency_wait();
-        // the weights of the first stages start streaming before anything else
-        for (int j = 0; j < n_pre; ++j) {
-            issue_w(ring + j * kWBytes, &tm_w, &wfull[j], s0 + j, row0);
-            wissued[j] = 0;
-            if (!weights_early) {
-                issue_x(xring + j * kXBytes, &tm_x, &xfull[j], s0 + j);
-                xissued[j] = 0;
-            }
-        }
-    }
-
-    // absmax inputs of the first kPrefetch + 1 stages (rows past n clamped)
-    const int arow = threadIdx.x & (kRows - 1);
-    const int half = threadIdx.x >> 7;
-    const bool aligned4 = (kblocks & 3) == 0 && (reinterpret_cast<uintptr_t>(absmax_q) & 3) == 0;
-    const int64_t agrow = row0 + arow;
-    AbsmaxIn first;
-    AbsmaxIn pre[kPrefetch];
-    load_absmax_in(first, absmax_q, absmax_scale, agrow, half, s0, n, kblocks, aligned4);
-#pragma unroll
-    for (int d = 0; d < kPrefetch; ++d)
-        load_absmax_in(pre[d], absmax_q, absmax_scale, agrow, half, min(s0 + 1 + d, n_stages - 1), n, kblocks,
-                       aligned4);
-    const float mu = __ldg(mu_ptr);
-
-    // byte -> (level of high nibble, level of low nibble), 16 copies so that
-    // the 16 lanes of a half-warp always read distinct banks.  Thread t writes
-    // 16-byte chunks c = t + 256 it (two copies of byte c / 8): its low nibble
-    // (t / 8) mod 16 is fixed and its high nibble is 2 it + t / 128, so every
-    // level comes from an immediate and the build touches no memory but the table.
-    static_assert(kLutBytes / 16 == 8 * kThreads, "eight chunks per thread");
-    {
-        constexpr float kLv[16] = NF4_LEVELS_INIT;
-        const int lo_idx = (threadIdx.x >> 3) & 15;
-        float lo = kLv[0];
-#pragma unroll
-        for (int v = 1; v < 16; ++v) lo = (lo_idx == v) ? kLv[v] : lo;
-        const bool odd = (threadIdx.x >> 7) != 0;
-#pragma unroll
-        for (int it = 0; it < 8; ++it) {
-            const float hi = odd ? kLv[2 * it + 1] : kLv[2 * it];
-            sts128(smem_u32(lut) + 16u * (threadIdx.x + kThreads * it),
-                   make_uint4(__float_as_uint(hi), __float_as_uint(lo), __float_as_uint(hi), __float_as_uint(lo)));
-        }
-    }
-    __syncthreads();  // barriers initialised, LUT written
-
-    if (threadIdx.x == 0 && weights_early) {
-        // weights are in flight; X (the preceding kernel's output) only after it finished
-        grid_dependency_wait();
-        for (int j = 0; j < n_pre; ++j) {
-            issue_x(xring + j * kXBytes, &tm_x, &xfull[j], s0 + j);
-            xissued[j] = 0;
-        }
-    }
-    // the absmax table of the first stage
-    const uint32_t ahat_base = smem_u32(smem_raw + kAhatOff);
-    const uint32_t ahat_mine = ahat_base + arow * 16u;
-    pin(first);
-    store_ahat(ahat_mine, half, first, mu);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&afull[0]);
-    // Under a programmatic dependent launch, sleep here (rather than poll the
-    // ring) until the preceding kernel has finished; otherwise a no-op.
-    grid_dependency_wait();
-
-    const int g = lane >> 2;
-    const int i = lane & 3;
-    const int bpair = warp >> 2;         // the warp's two 64-blocks of the stage: 2 bpair, 2 bpair + 1
-    const int rbase = (warp & 3) * 32;   // first of this warp's 32 rows
-    const uint32_t lut_lane = smem_u32(lut) + (lane & 15) * 8u;
-    float acc[kTiles][4];
-#pragma unroll
-    for (int t = 0; t < kTiles; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-
-    bool timed_out = false;
-    for (int j0 = 0; j0 < nst && !timed_out; j0 += kPrefetch) {
-#pragma unroll
-        for (int d = 0; d < kPrefetch; ++d) {
-            const int j = j0 + d;
-            if (j >= nst) break;
-            const int slot = j % kRing;
-            // absmax table of the next stage.  Its table slot held stage j - 3:
-            // this warp saw stage j - 1's table complete, so every warp has begun
-            // stage j - 2 and is done with stage j - 3.
-            if (j + 1 < nst) {
-                const int nslot = (j + 1) % kAring;
-                pin(pre[d]);
-                store_ahat(ahat_mine + nslot * kAhatBytes, half, pre[d], mu);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&afull[nslot]);
-                // (unconditional, clamped to a valid stage, so no select waits on the loads)
-                load_absmax_in(pre[d], absmax_q, absmax_scale, agrow, half,
-                               min(s0 + j + 1 + kPrefetch, n_stages - 1), n, kblocks, aligned4);
-            }
-            // every lane polls; the warp proceeds only if all of them saw the stage
-            const int aslot = j % kAring;
-            const uint32_t par = (j / kRing) & 1;
-            if (!__all_sync(kFull, mbar_wait(&wfull[slot], par) && mbar_wait(&afull[aslot], (j / kAring) & 1))) {
-                timed_out = true;
-                break;
-            }
-            // This warp's codes of the stage into registers (rows rbase + 8 t + g,
-            // 8 bytes per lane = 16 consecutive weights of a block), then leave the
-            // codes slot: the last warp out refills it while the decode runs.
-            const uint32_t wstage = smem_u32(ring + slot * kWBytes);
-            uint2 raw[2][kTiles];
-#pragma unroll
-            for (int bb = 0; bb < 2; ++bb) {
-                const uint32_t wb = wstage + (rbase + g) * 128 +
-                                    ((((2 * (2 * bpair + bb) + (i >> 1)) ^ g) << 4) + ((i & 1) << 3));
-#pragma unroll
-                for (int t = 0; t < kTiles; ++t) raw[bb][t] = lds64(wb + t * 8 * 128);
-            }
-            __syncwarp();
-            if (lane == 0 && slot_leave(&wdone[slot]) == static_cast<uint32_t>(kConsumers * (j / kRing + 1) - 1) &&
-                j + kRing < nst) {
-                issue_w(ring + slot * kWBytes, &tm_w, &wfull[slot], s0 + j + kRing, row0);
-                wissued[slot] = j / kRing + 1;
-            }
-            if (!__all_sync(kFull, mbar_wait(&xfull[slot], par))) {
-                timed_out = true;
-                break;
-            }
-            const uint32_t xstage = smem_u32(xring + slot * kXBytes);
-#pragma unroll
-            for (int bb = 0; bb < 2; ++bb) {
-                const int blk = 2 * bpair + bb;
-                // X fragments: tokens g and g + 8, k = 16 i .. 16 i + 15 of block blk
-                const uint32_t xb = xstage + blk * kXBox;
-                const uint4 xa0 = lds128(xb + g * 128 + (((2 * i) ^ g) << 4));
-                const uint4 xa1 = lds128(xb + g * 128 + (((2 * i + 1) ^ g) << 4));
-                uint4 xc0 = make_uint4(0u, 0u, 0u, 0u), xc1 = xc0;
-                if (kM16) {
-                    xc0 = lds128(xb + (g + 8) * 128 + (((2 * i) ^ g) << 4));
-                    xc1 = lds128(xb + (g + 8) * 128 + (((2 * i + 1) ^ g) << 4));
-                }
-                const uint32_t xa[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
-                const uint32_t xc[8] = {xc0.x, xc0.y, xc0.z, xc0.w, xc1.x, xc1.y, xc1.z, xc1.w};
-                const uint32_t ab = ahat_base + aslot * kAhatBytes + ((rbase + g) * 4 + blk) * 4;
-#pragma unroll
-                for (int t = 0; t < kTiles; ++t) {
-                    const uint64_t aa = dup_f32x2(lds_f32(ab + 128 * t));
-                    uint32_t bw[8];
-#pragma unroll
-                    for (int b = 0; b < 8; ++b) {
-                        const uint32_t word = (b < 4) ? raw[bb][t].x : raw[bb][t].y;
-                        bw[b] = scale_pack(lds_b64(lut_lane + (byte_of(word, b & 3) << 7)), aa);
-                    }
-#pragma unroll
-                    for (int s = 0; s < 4; ++s)
-                        mma_16816(acc[t], xa[2 * s], xc[2 * s], xa[2 * s + 1], xc[2 * s + 1], bw[2 * s],
-                                  bw[2 * s + 1]);
-                }
-            }
-            // the last warp out of the X slot refills it
-            __syncwarp();
-            if (lane == 0 && slot_leave(&xdone[slot]) == static_cast<uint32_t>(kConsumers * (j / kRing + 1) - 1) &&
-                j + kRing < nst) {
-                issue_x(xring + slot * kXBytes, &tm_x, &xfull[slot], s0 + j + kRing);
-                xissued[slot] = j / kRing + 1;
-            }
-        }
-    }
-    // the next kernel on the stream may start its prologue (its weight
-    // prefetch overlaps our epilogue)
-    grid_launch_dependents();
-
-    // fold the warps: red[bpair][token][row] (the four row groups of a block
-    // pair land in disjoint rows of the same buffer)
-    timed_out = __syncthreads_or(timed_out);  // every warp is done with the ring
-    if (timed_out) {
-        // leave no copy in flight: wait (bounded) for every stage issued
-        if (threadIdx.x == 0) {
-            record_timeout(dev_status);
-            for (int s = 0; s < kRing; ++s) {
-                if (wissued[s] >= 0) mbar_wait(&wfull[s], wissued[s] & 1);
-                if (xissued[s] >= 0) mbar_wait(&xfull[s], xissued[s] & 1);
-            }
-        }
-        __syncthreads();
-    }
-    float* red = reinterpret_cast<float*>(ring) + bpair * 16 * kRedPitch;
-#pragma unroll
-    for (int t = 0; t < kTiles; ++t) {
-        const int r = rbase + 8 * t + 2 * i;
-        *reinterpret_cast<float2*>(&red[g * kRedPitch + r]) = make_float2(acc[t][0], acc[t][1]);
-        *reinterpret_cast<float2*>(&red[(g + 8) * kRedPitch + r]) = make_float2(acc[t][2], acc[t][3]);
     }
     __syncthreads();
+
+    bool timed_out = false;
+    if (warp == kConsumers) {
+        // ------------------------------ producer ------------------------------
+        if (lane == 0) {
+            prefetch_tensormap(&tm_w);
+            prefetch_tensormap(&tm_x);
+        }
+        if (!weights_early) grid_dependency_wait();
+        const float mu = __ldg(mu_ptr);
+        int last_use[kRing];
+#pragma unroll
+        for (int s = 0; s < kRing; ++s) last_use[s] = -1;
+        bool x_ready = !weights_early;  // X (the previous kernel's output) may be read
+        const int n_pre = (s1 - s0) < kRing ? (s1 - s0) : kRing;
+        const bool aligned4 = (kblocks & 3) == 0 && (reinterpret_cast<uintptr_t>(absmax_q) & 3) == 0;
+        AbsmaxIn pre[kPrefetch];
+#pragma unroll
+        for (int d = 0; d < kPrefetch; ++d)
+            load_absmax_in(pre[d], absmax_q, absmax_scale, row0, lane, min(s0 + d, n_stages - 1), n, kblocks, aligned4);
+        for (int st0 = s0; st0 < s1 && !timed_out; st0 += kPrefetch) {
+#pragma unroll
+            for (int d = 0; d < kPrefetch; ++d) {
+                const int st = st0 + d;
+                if (st >= s1) break;
+                const int j = st - s0;
+                const int slot = j % kRing;
+                const int use = j / kRing;
+                if (j >= kRing && !__all_sync(kFull, mbar_wait(&empty[slot], (use - 1) & 1))) {
+                    timed_out = true;
+                    break;
+                }
+                uint8_t* stage = ring + slot * kStageBytes;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&full[slot], kTmaBytes);
+                    tma_load_2d(stage, &tm_w, st * (kStageK / 2), static_cast<int32_t>(row0), &full[slot]);
+                    if (x_ready) {
+#pragma unroll
+                        for (int b = 0; b < 4; ++b)
+                            tma_load_2d(stage + kWBytes + b * kXBox, &tm_x, st * kStageK + 64 * b, 0, &full[slot]);
+                    }
+                    last_use[slot] = use;
+                }
+                pin(pre[d]);  // the copies above are issued before the absmax work below
+                // reconstructed absmax a = fp32(fp32(fp32(q / 127) * s) + mu) of this stage.
+                // Blocks past k or rows past n get q = s = 0 (a = mu, finite): X is
+                // zero-filled there, so their products vanish.
+                const uint32_t ahat = smem_u32(stage + kTmaBytes);  // [row][block] floats
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int row = lane + 32 * u;
+                    const int64_t b0 = (row0 + row) * kblocks + static_cast<int64_t>(st) * 4;
+                    float a4[4];
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        const float sc = (((b0 + b) >> 8) == (b0 >> 8)) ? pre[d].s_lo[u] : pre[d].s_hi[u];
+                        const float qf = static_cast<float>(static_cast<int8_t>((pre[d].q[u] >> (8 * b)) & 0xffu));
+                        a4[b] = __fadd_rn(__fmul_rn(div127(qf), sc), mu);
+                    }
+                    sts128(ahat + row * 16u, make_uint4(__float_as_uint(a4[0]), __float_as_uint(a4[1]),
+                                                        __float_as_uint(a4[2]), __float_as_uint(a4[3])));
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full[slot]);
+                // (unconditional, clamped to a valid stage, so no select waits on the loads)
+                load_absmax_in(pre[d], absmax_q, absmax_scale, row0, lane, min(st + kPrefetch, n_stages - 1), n,
+                               kblocks, aligned4);
+                if (!x_ready && j + 1 == n_pre) {
+                    // weights of the first stages are in flight; now wait for the
+                    // preceding kernel before touching X
+                    grid_dependency_wait();
+                    x_ready = true;
+                    if (lane == 0)
+                        for (int jj = 0; jj <= j; ++jj) {
+                            uint8_t* stg = ring + (jj % kRing) * kStageBytes;
+#pragma unroll
+                            for (int b = 0; b < 4; ++b)
+                                tma_load_2d(stg + kWBytes + b * kXBox, &tm_x, (s0 + jj) * kStageK + 64 * b, 0,
+                                            &full[jj % kRing]);
+                        }
+                }
+            }
+        }
+        if (!x_ready) grid_dependency_wait();
+        // every copy of this CTA is issued: the next kernel on the stream may
+        // start its prologue (its weight prefetch overlaps our last stages)
+        grid_launch_dependents();
+        // on a timeout leave no copy in flight: wait (bounded) for every stage issued
+        if (timed_out && lane == 0)
+            for (int s = 0; s < kRing; ++s)
+                if (last_use[s] >= 0) mbar_wait(&full[s], last_use[s] & 1);
+    } else {
+        // ------------------------------ consumers -----------------------------
+        // byte -> (level of high nibble, level of low nibble), 16 copies so that
+        // the 16 lanes of a half-warp always read distinct banks.  Consumer
+        // thread t writes 16-byte chunks c = t + 256 it (two copies of byte
+        // c / 8): its low nibble (t / 8) mod 16 is fixed and its high nibble is
+        // 2 it + t / 128, so every level is an immediate and the build touches
+        // no memory but the table.
+        static_assert(kLutBytes / 16 == 8 * 32 * kConsumers, "eight chunks per consumer thread");
+        {
+            constexpr float kLv[16] = NF4_LEVELS_INIT;
+            const int lo_idx = (threadIdx.x >> 3) & 15;
+            float lo = kLv[0];
+#pragma unroll
+            for (int v = 1; v < 16; ++v) lo = (lo_idx == v) ? kLv[v] : lo;
+            const bool odd = (threadIdx.x >> 7) != 0;
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+                const float hi = odd ? kLv[2 * it + 1] : kLv[2 * it];
+                sts128(smem_u32(lut) + 16u * (threadIdx.x + 32 * kConsumers * it),
+                       make_uint4(__float_as_uint(hi), __float_as_uint(lo), __float_as_uint(hi), __float_as_uint(lo)));
+            }
+        }
+        named_bar_sync(1, 32 * kConsumers);
+        // Under a programmatic dependent launch, sleep here (rather than poll
+        // the ring) until the preceding kernel has finished; otherwise a no-op.
+        grid_dependency_wait();
+
+        const int g = lane >> 2;
+        const int i = lane & 3;
+        const int blk = warp & 3;          // 64-block of the stage
+        const int rbase = (warp >> 2) * 64;  // first of this warp's 64 rows
+        const uint32_t lut_lane = smem_u32(lut) + (lane & 15) * 8u;
+        float acc[kTiles][4];
+#pragma unroll
+        for (int t = 0; t < kTiles; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+
+        for (int st = s0; st < s1; ++st) {
+            const int j = st - s0;
+            const int slot = j % kRing;
+            // every lane polls; the warp proceeds only if all of them saw the stage
+            if (!__all_sync(kFull, mbar_wait(&full[slot], (j / kRing) & 1))) {
+                timed_out = true;
+                break;
+            }
+            const uint32_t stage = smem_u32(ring + slot * kStageBytes);
+            // X fragments: tokens g and g + 8, k = 16 i .. 16 i + 15 of this warp's block
+            const uint32_t xb = stage + kWBytes + blk * kXBox;
+            const uint4 xa0 = lds128(xb + g * 128 + (((2 * i) ^ g) << 4));
+            const uint4 xa1 = lds128(xb + g * 128 + (((2 * i + 1) ^ g) << 4));
+            uint4 xc0 = make_uint4(0u, 0u, 0u, 0u), xc1 = xc0;
+            if (kM16) {
+                xc0 = lds128(xb + (g + 8) * 128 + (((2 * i) ^ g) << 4));
+                xc1 = lds128(xb + (g + 8) * 128 + (((2 * i + 1) ^ g) << 4));
+            }
+            const uint32_t xa[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
+            const uint32_t xc[8] = {xc0.x, xc0.y, xc0.z, xc0.w, xc1.x, xc1.y, xc1.z, xc1.w};
+            const uint32_t wb = stage + (rbase + g) * 128 + ((((2 * blk + (i >> 1)) ^ g) << 4) + ((i & 1) << 3));
+            const uint32_t ab = stage + kTmaBytes + ((rbase + g) * 4 + blk) * 4;
+#pragma unroll
+            for (int t = 0; t < kTiles; ++t) {
+                const uint2 raw = lds64(wb + t * 8 * 128);
+                const uint64_t aa = dup_f32x2(lds_f32(ab + 128 * t));
+                uint32_t bw[8];
+#pragma unroll
+                for (int b = 0; b < 8; ++b) {
+                    const uint32_t word = (b < 4) ? raw.x : raw.y;
+                    bw[b] = scale_pack(lds_b64(lut_lane + (byte_of(word, b & 3) << 7)), aa);
+                }
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_16816(acc[t], xa[2 * s], xc[2 * s], xa[2 * s + 1], xc[2 * s + 1], bw[2 * s], bw[2 * s + 1]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
+        }
+
+        // fold the consumer warps: red[blk][token][row] (the two row halves of a
+        // block land in disjoint rows of the same buffer)
+        __syncwarp();
+        named_bar_sync(1, 32 * kConsumers);  // every consumer is done with the ring
+        float* red = reinterpret_cast<float*>(ring) + blk * 16 * kRedPitch;
+#pragma unroll
+        for (int t = 0; t < kTiles; ++t) {
+            const int r = rbase + 8 * t + 2 * i;
+            *reinterpret_cast<float2*>(&red[g * kRedPitch + r]) = make_float2(acc[t][0], acc[t][1]);
+            *reinterpret_cast<float2*>(&red[(g + 8) * kRedPitch + r]) = make_float2(acc[t][2], acc[t][3]);
+        }
+        grid_dependency_wait();  // Y may still be in use by the preceding kernel
+    }
+    if (timed_out) record_timeout(dev_status);
+    __syncthreads();
     const float* redf = reinterpret_cast<const float*>(ring);
-    float4* part4 = reinterpret_cast<float4*>(ring + kPartOff);
+    float4* part4 = reinterpret_cast<float4*>(ring) + 4 * 16 * kRedPitch / 4;
     constexpr int kQ = 16 * kRows / 4;  // float4s of partial sums per CTA
     constexpr int kB = 16 * kRedPitch;  // floats per block buffer
     for (int e = threadIdx.x; e < kQ; e += kThreads) {
         const int off = (e / (kRows / 4)) * kRedPitch + 4 * (e % (kRows / 4));
         const float4 a = *reinterpret_cast<const float4*>(redf + off);
         const float4 b = *reinterpret_cast<const float4*>(redf + kB + off);
-        part4[e] = make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+        const float4 c = *reinterpret_cast<const float4*>(redf + 2 * kB + off);
+        const float4 d = *reinterpret_cast<const float4*>(redf + 3 * kB + off);
+        part4[e] = make_float4(((a.x + b.x) + c.x) + d.x, ((a.y + b.y) + c.y) + d.y,
+                               ((a.z + b.z) + c.z) + d.z, ((a.w + b.w) + c.w) + d.w);
     }
 
-    // Cluster split-k: rank q owns rows [q * 128 / C, (q + 1) * 128 / C).  Every
-    // rank sends the partials of q's rows into q's receive area and arrives on
-    // q's barrier; q adds the C partials in rank order and writes Y.  Nothing
-    // reads another CTA's memory, so no rank waits for the others to finish.
+    // cluster split-k: rank r adds rows [r * 128 / C, (r + 1) * 128 / C) over all ranks in rank order
+    cluster_sync();
     const int rows_per_rank = kRows / cluster;
     const int quads = rows_per_rank / 4;
     const int r_lo = rank * rows_per_rank;
-    const uint32_t recv_addr = smem_u32(ring + kRecvOff);
-    if (cluster > 1) {
-        cluster_sync();  // every rank is done with its ring: receive areas are free
-        for (int e = threadIdx.x; e < m * (kRows / 4); e += kThreads) {
-            const int tok = e / (kRows / 4);
-            const int r = 4 * (e % (kRows / 4));
-            const int q = r / rows_per_rank;
-            if (q == rank) continue;
-            const uint32_t off =
-                static_cast<uint32_t>(((rank * 16 + tok) * rows_per_rank + (r - q * rows_per_rank)) * 4);
-            st_shared_cluster_f32x4(map_shared_rank(recv_addr + off, q), part4[tok * (kRows / 4) + r / 4]);
-        }
-        fence_acq_rel_cluster();
-        __syncthreads();
-        if (threadIdx.x < cluster && threadIdx.x != rank)
-            mbar_arrive_remote(map_shared_rank(smem_u32(rfull), threadIdx.x));
-        if (!mbar_wait_cluster(rfull, 0)) {
-            record_timeout(dev_status);
-            return;
-        }
-    }
+    const uint32_t part_addr = smem_u32(part4);
     for (int e = threadIdx.x; e < m * quads; e += kThreads) {
         const int tok = e / quads;
-        const int rr = 4 * (e % quads);
-        const float4 own = part4[tok * (kRows / 4) + (r_lo + rr) / 4];
-        float4 sum = own;
-        for (int q = 0; q < cluster; ++q) {
-            const float4 v = (q == rank) ? own
-                                         : *reinterpret_cast<const float4*>(
-                                               ring + kRecvOff + ((q * 16 + tok) * rows_per_rank + rr) * 4);
-            sum = (q == 0) ? v : make_float4(sum.x + v.x, sum.y + v.y, sum.z + v.z, sum.w + v.w);
-        }
+        const int r = r_lo + 4 * (e % quads);
+        const uint32_t off = static_cast<uint32_t>((tok * kRows + r) * 4);
+        float4 v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            if (q < cluster) v[q] = ld_shared_cluster_f32x4(map_shared_rank(part_addr + off, q));
+        float4 sum = v[0];
+#pragma unroll
+        for (int q = 1; q < 8; ++q)
+            if (q < cluster) sum = make_float4(sum.x + v[q].x, sum.y + v[q].y, sum.z + v[q].z, sum.w + v[q].w);
         const float o[4] = {sum.x, sum.y, sum.z, sum.w};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            const int64_t grow = row0 + r_lo + rr + c;
+            const int64_t grow = row0 + r + c;
             if (grow >= n) break;
             if (kBf16Out)
                 reinterpret_cast<__nv_bfloat16*>(Y)[static_cast<int64_t>(tok) * n + grow] = __float2bfloat16_rn(o[c]);
@@ -527,6 +443,7 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
                 reinterpret_cast<float*>(Y)[static_cast<int64_t>(tok) * n + grow] = o[c];
         }
     }
+    cluster_sync();  // keep this CTA's partials alive until every rank has read them
 }
 
 }  // namespace gemv
@@ -586,6 +503,8 @@ cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int
                             CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
     const int cluster = gemv_cluster(n, k, dev.sm_count);
+    // the split-k epilogue gives each rank 128 / C rows in groups of 4
+    if (cluster != 1 && cluster != 2 && cluster != 4 && cluster != 8) return cudaErrorInvalidConfiguration;
     const size_t ybytes = y_bf16 ? 2 : 4;
     const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
     for (int64_t t0 = 0; t0 < m; t0 += 16) {
