@@ -189,6 +189,17 @@ def test_linear_ragged_shapes(nf4, n, k):
     _check_linear(nf4, X, weight, orc)
 
 
+@pytest.mark.parametrize("m", [3, 16])
+def test_gemv_three_way_split_k(nf4, m):
+    """11000 x 2304 makes the GEMV split k three ways (258 CTAs, rank row ranges
+    of 42/43/43 rows, a partial last row tile): every output row is checked."""
+    n, k = 11000, 2304
+    W = synth.weight_normal(n, k, seed=700 + m, dtype=torch.bfloat16, device="cuda")
+    X = synth.activations(m, k, seed=710 + m, device="cuda")
+    weight, orc = _check_quant(nf4, W, full_dequant=False, rows=[0, 41, 42, 84, 85, 127, n - 1])
+    _check_linear(nf4, X, weight, orc)
+
+
 def test_deterministic_and_stream_aware(nf4):
     W = synth.weight_normal(512, 1024, seed=9, dtype=torch.bfloat16, device="cuda")
     X = synth.activations(16, 1024, seed=10, device="cuda")
