@@ -407,7 +407,41 @@ def run_ours(args, rank, world, local):
         gemm = {"m": 4096, "k": 4096, "n": 11008, "tflops": round(tflops, 2),
                 "ms": round(t_g * 1e3, 3), "peak_tflops": pk["bf16_tflops"],
                 "frac": round(tflops / pk["bf16_tflops"], 4), "peak_kind": pk_kind + " burst bf16"}
+        # the same weight over a sweep of token counts (m <= 16 runs the GEMV)
+        sweep = {}
+        for mm in (16, 128, 256, 512, 1024, 2048, 8192):
+            Xs = synth.activations(mm, 4096, seed=synth.seed_for(3, 2) + mm, device=dev)
+            Ys = torch.empty((mm, 11008), dtype=torch.bfloat16, device=dev)
+            fs = lambda: nf4.nf4_linear(Xs, wg, torch.bfloat16, out=Ys)
+            fs()
+            ts = _events_time(fs, 5 if mm < 8192 else 3, stream)
+            sweep[mm] = round(2.0 * mm * 4096 * 11008 / ts / 1e12, 1)
+            del Xs, Ys
+        sweep[4096] = gemm["tflops"]
+        gemm["tflops_by_m"] = dict(sorted(sweep.items()))
         del Xg, Yg, wg
+
+    # 70B-shaped stress layer: 28672 x 8192 Student-t(4) weight with outlier input
+    # columns, as GEMV (m = 1, 16) and GEMM (m = 512, 4096)
+    stress = None
+    if not args.skip_gemm:
+        n5, k5 = 28672, 8192
+        W5 = synth.weight_student_t(n5, k5, seed=synth.seed_for(5, 0), dtype=torch.bfloat16, device=dev)
+        w5 = nf4.quantize_weight(W5)
+        del W5
+        stress = {"n": n5, "k": k5, "gemv_gbs": {}, "gemm_tflops": {}}
+        for mm in (1, 16, 512, 4096):
+            X5 = synth.activations(mm, k5, seed=synth.seed_for(5, 1) + mm, device=dev)
+            Y5 = torch.empty((mm, n5), dtype=torch.bfloat16, device=dev)
+            f5 = lambda: nf4.nf4_linear(X5, w5, torch.bfloat16, out=Y5)
+            f5()
+            t5 = _events_time(f5, 5, stream)
+            if mm <= 16:
+                stress["gemv_gbs"][mm] = round(linear_bytes(n5, k5, mm, 2) / t5 / 1e9, 1)
+            else:
+                stress["gemm_tflops"][mm] = round(2.0 * mm * n5 * k5 / t5 / 1e12, 1)
+            del X5, Y5
+        del w5
 
     # quantize + double quant, and dequantize, over the stack
     qd = None
@@ -463,6 +497,7 @@ def run_ours(args, rank, world, local):
             "frac_of_peak": round(value / world / pk["hbm_gbs"], 4),
             "decode_gbs_by_m": by_m,
             "gemm": gemm,
+            "stress_70b_layer": stress,
             "quant": qd,
             "roofline": {"bound": "hbm", "kernel": "k_nf4_gemv", "achieved": round(achieved, 1),
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),

@@ -292,6 +292,11 @@ def test_cfg3_prefill_gemm(nf4):
     weight, orc = _check_quant(nf4, W, full_dequant=False, rows=_sample_rows(n, 16, 3))
     _check_linear(nf4, X, weight, orc, token_rows=_sample_rows(m, 48, 31),
                   weight_rows=_sample_rows(n, 160, 32))
+    # the token-count sweep that bench.py times on the same weight
+    for mm in (128, 256, 512, 1024, 2048, 8192):
+        Xs = synth.activations(mm, k, seed=synth.seed_for(3, 2) + mm, device="cuda")
+        _check_linear(nf4, Xs, weight, orc, token_rows=_sample_rows(mm, 16, mm),
+                      weight_rows=_sample_rows(n, 64, mm + 1))
 
 
 def test_cfg4_layer_stack_sample(nf4):
