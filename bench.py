@@ -322,10 +322,12 @@ def run_ours(args, rank, world, local):
         xs = {k: synth.activations(m, k, seed=synth.seed_for(2, 100 + m) + k, device=dev)
               for k in set(k for _, k in shapes)}
         ys = {n: torch.empty((m, n), dtype=torch.bfloat16, device=dev) for n in set(n for n, _ in shapes)}
+        # one split-k workspace serves every linear of the step (they run one after another)
+        ws = None if args.no_workspace else nf4.linear_workspace(shapes, m=m, device=dev)
 
         def step():
             for w in weights:
-                nf4.nf4_linear(xs[w.k], w, torch.bfloat16, out=ys[w.n], weights_early=early)
+                nf4.nf4_linear(xs[w.k], w, torch.bfloat16, out=ys[w.n], weights_early=early, workspace=ws)
         step()
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
@@ -491,9 +493,11 @@ def run_ours(args, rank, world, local):
                        "l2": "inputs larger than L2 (%.2f GB of NF4 weights per step vs 126 MB)"
                              % (sum(w.nbytes() for w in weights) / 1e9),
                        "y_dtype": "bf16", "parallelism": "replicas (weak scaling)",
-                       "launch": ("CUDA graph of nf4_linear_ex(NF4_LINEAR_WEIGHTS_EARLY): programmatic "
+                       "launch": ("CUDA graph of nf4_linear_ws(NF4_LINEAR_WEIGHTS_EARLY): programmatic "
                                   "dependent launches, weight loads overlap the previous layer") if early
-                                 else "CUDA graph of nf4_linear: each layer starts after the previous ends"},
+                                 else "CUDA graph of nf4_linear_ws: each layer starts after the previous ends",
+                       "split_k": "cluster (distributed shared memory)" if args.no_workspace
+                                  else "global workspace, last CTA of a tile reduces"},
             "frac_of_peak": round(value / world / pk["hbm_gbs"], 4),
             "decode_gbs_by_m": by_m,
             "gemm": gemm,
@@ -519,6 +523,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--m", type=int, default=16, help="tokens per decode step (1..16)")
     ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--no-workspace", action="store_true",
+                    help="split-k through thread-block clusters instead of a global workspace")
     ap.add_argument("--no-weights-early", action="store_true",
                     help="launch each linear without programmatic dependent launch")
     ap.add_argument("--skip-gemm", action="store_true")

@@ -231,6 +231,38 @@ nf4_status_t nf4_linear_ex(const void* X, int64_t m, const nf4_weight_t* w, void
                            nf4_dtype_t y_dtype, int32_t* dev_status, uint32_t flags,
                            nf4_stream_t stream);
 
+/*
+ * nf4_linear_workspace_bytes -- bytes of the optional split-k workspace that
+ * nf4_linear_ws can use for Y[m, n] = X[m, k] * What^T on the current device;
+ * 0 when that product splits no k range (then no workspace is needed).  The
+ * workspace holds one counter per 128-row tile and the fp32 partial sums of
+ * every CTA; one buffer serves every call whose requirement it meets.
+ * Returns 0 for invalid sizes.  Same source passages as nf4_linear.
+ */
+size_t nf4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k);
+
+/*
+ * nf4_linear_ws -- nf4_linear_ex with an optional caller-owned workspace; the
+ * results are bit-identical.  In the decode path (m <= 16) the k range of each
+ * 128-row tile is split across several CTAs.  Without a workspace those CTAs
+ * form a thread-block cluster and add their partial sums through distributed
+ * shared memory, each waiting for the others.  With a workspace they meet in
+ * global memory instead: every CTA stores its partial sums and counts itself in;
+ * the last one adds the partials in k order and writes Y, and the others exit at
+ * once.  (Same source passages as nf4_linear.)
+ *   workspace  device, 16-byte aligned, at least nf4_linear_workspace_bytes(m,
+ *              n, k) bytes, or NULL (the cluster path).  Its counters must be
+ *              zero before first use: zero-fill the buffer once; every call
+ *              leaves them zero again.  A workspace must not serve two calls
+ *              that can run at the same time (for example on two streams).
+ *   ws_bytes   size of workspace in bytes
+ * Errors: as nf4_linear_ex, plus NF4_ERR_WORKSPACE (workspace smaller than
+ * required) and NF4_ERR_ALIGN (workspace not 16-byte aligned).
+ */
+nf4_status_t nf4_linear_ws(const void* X, int64_t m, const nf4_weight_t* w, void* Y,
+                           nf4_dtype_t y_dtype, int32_t* dev_status, uint32_t flags,
+                           void* workspace, size_t ws_bytes, nf4_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -8,7 +8,8 @@ calls.  Functions carry the C names:
 * ``nf4_quantize(W)`` -> ``(wq, absmax)``
 * ``nf4_double_quant(absmax)`` -> ``(absmax_q, absmax_scale, absmax_offset)``
 * ``nf4_dequantize(weight, dtype)`` -> dense tensor
-* ``nf4_linear(X, weight, dtype)`` -> ``Y = X @ W_hat^T``
+* ``nf4_linear(X, weight, dtype)`` -> ``Y = X @ W_hat^T`` (optionally with a
+  split-k ``workspace`` from ``linear_workspace``)
 
 ``quantize_weight(W)`` runs the first two and returns an ``NF4Weight``.
 """
@@ -23,7 +24,8 @@ from . import _lib
 from ._lib import NF4_BF16, NF4_F32, NF4Error, nf4_weight_t
 
 __all__ = ["NF4Weight", "NF4Error", "nf4_quantize", "nf4_double_quant", "nf4_dequantize",
-           "nf4_linear", "nf4_linear_ex", "quantize_weight", "nf4_codebook", "library_path"]
+           "nf4_linear", "nf4_linear_ex", "nf4_linear_workspace_bytes", "linear_workspace",
+           "quantize_weight", "nf4_codebook", "library_path"]
 
 _DTYPES = {torch.float32: NF4_F32, torch.bfloat16: NF4_BF16}
 
@@ -142,14 +144,31 @@ def nf4_linear_ex(X, weight, dtype=torch.bfloat16, out=None, dev_status=None, st
                       weights_early=bool(flags & _lib.NF4_LINEAR_WEIGHTS_EARLY))
 
 
+def nf4_linear_workspace_bytes(m: int, n: int, k: int) -> int:
+    """Bytes of the optional split-k workspace of nf4_linear for these sizes on
+    the current device (0: none needed)."""
+    return int(_lib.lib().nf4_linear_workspace_bytes(m, n, k))
+
+
+def linear_workspace(shapes, m: int = 16, device=None) -> torch.Tensor:
+    """A zero-filled workspace large enough for nf4_linear at m tokens on every
+    (n, k) in ``shapes`` (one buffer serves them all)."""
+    nbytes = max([nf4_linear_workspace_bytes(m, n, k) for n, k in shapes] + [16])
+    return torch.zeros((nbytes + 15) // 16 * 16, dtype=torch.uint8, device=device or "cuda")
+
+
 def nf4_linear(X: torch.Tensor, weight: NF4Weight, dtype=torch.bfloat16,
                out: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
-               stream=None, weights_early: bool = False) -> torch.Tensor:
+               stream=None, weights_early: bool = False,
+               workspace: torch.Tensor | None = None) -> torch.Tensor:
     """Y = X @ W_hat^T for bf16 X [m, k]; Y [m, n] in ``dtype`` (bf16 or fp32).
 
-    ``weights_early=True`` calls ``nf4_linear_ex`` with NF4_LINEAR_WEIGHTS_EARLY:
-    the weight was not written by the work just before this call on the stream,
-    so its loads may overlap that work (programmatic dependent launch)."""
+    ``weights_early=True`` sets NF4_LINEAR_WEIGHTS_EARLY: the weight was not
+    written by the work just before this call on the stream, so its loads may
+    overlap that work (programmatic dependent launch).  ``workspace`` (from
+    ``linear_workspace``) lets the decode path's split-k CTAs meet in global
+    memory instead of waiting for each other in a cluster; the results are the
+    same bits.  The call goes to ``nf4_linear_ws``."""
     _need_cuda(X, "X")
     if X.dtype != torch.bfloat16 or X.dim() != 2:
         raise ValueError("X must be a 2-D bfloat16 tensor")
@@ -161,6 +180,11 @@ def nf4_linear(X: torch.Tensor, weight: NF4Weight, dtype=torch.bfloat16,
     st = weight.struct()
     ds = ctypes.c_void_p(0) if dev_status is None else _ptr(dev_status)
     flags = _lib.NF4_LINEAR_WEIGHTS_EARLY if weights_early else 0
-    _lib.check(_lib.lib().nf4_linear_ex(_ptr(X), m, ctypes.byref(st), _ptr(out), _DTYPES[dtype], ds,
-                                        flags, _stream(stream)), "nf4_linear_ex")
+    if workspace is None:
+        ws, ws_bytes = ctypes.c_void_p(0), 0
+    else:
+        _need_cuda(workspace, "workspace")
+        ws, ws_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+    _lib.check(_lib.lib().nf4_linear_ws(_ptr(X), m, ctypes.byref(st), _ptr(out), _DTYPES[dtype], ds,
+                                        flags, ws, ws_bytes, _stream(stream)), "nf4_linear_ws")
     return out

@@ -143,8 +143,9 @@ nf4_status_t nf4_dequantize(const nf4_weight_t* w, void* out, nf4_dtype_t out_dt
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
-nf4_status_t nf4_linear_ex(const void* X, int64_t m, const nf4_weight_t* w, void* Y,
-                           nf4_dtype_t y_dtype, int32_t* dev_status, uint32_t flags, nf4_stream_t stream) {
+nf4_status_t nf4_linear_ws(const void* X, int64_t m, const nf4_weight_t* w, void* Y,
+                           nf4_dtype_t y_dtype, int32_t* dev_status, uint32_t flags, void* workspace,
+                           size_t ws_bytes, nf4_stream_t stream) {
     nf4_status_t st = check_weight(w);
     if (st != NF4_OK) return st;
     if (!X || !Y) return NF4_ERR_NULL;
@@ -154,12 +155,26 @@ nf4_status_t nf4_linear_ex(const void* X, int64_t m, const nf4_weight_t* w, void
     if (m > INT64_MAX / w->k || m > INT64_MAX / w->n) return NF4_ERR_SHAPE;
     if (!aligned(X, 16) || !aligned(Y, 16) || (dev_status && !aligned(dev_status, 4)))
         return NF4_ERR_ALIGN;
+    if (workspace && !aligned(workspace, 16)) return NF4_ERR_ALIGN;
     nf4::DeviceInfo dev;
     if ((st = device_ok(&dev)) != NF4_OK) return st;
+    if (workspace && ws_bytes < nf4::linear_workspace_bytes(m, w->n, w->k, dev)) return NF4_ERR_WORKSPACE;
     return from_cuda(nf4::launch_linear(X, m, w->wq, w->absmax_q, w->absmax_scale, w->absmax_offset,
                                         w->n, w->k, Y, y_dtype == NF4_BF16, dev_status,
-                                        (flags & NF4_LINEAR_WEIGHTS_EARLY) != 0, dev,
+                                        (flags & NF4_LINEAR_WEIGHTS_EARLY) != 0, workspace, dev,
                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nf4_status_t nf4_linear_ex(const void* X, int64_t m, const nf4_weight_t* w, void* Y,
+                           nf4_dtype_t y_dtype, int32_t* dev_status, uint32_t flags, nf4_stream_t stream) {
+    return nf4_linear_ws(X, m, w, Y, y_dtype, dev_status, flags, nullptr, 0, stream);
+}
+
+size_t nf4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k) {
+    if (m < 1 || n < 1 || k < 1 || k % NF4_BLOCKSIZE != 0) return 0;
+    nf4::DeviceInfo dev;
+    if (device_ok(&dev) != NF4_OK) return 0;
+    return nf4::linear_workspace_bytes(m, n, k, dev);
 }
 
 nf4_status_t nf4_linear(const void* X, int64_t m, const nf4_weight_t* w, void* Y,

@@ -192,7 +192,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
            const int8_t* __restrict__ absmax_q, const float* __restrict__ absmax_scale,
            const float* __restrict__ mu_ptr, int m, int64_t n, int64_t k, int cluster, int weights_early,
-           void* __restrict__ Y, int32_t* __restrict__ dev_status) {
+           void* __restrict__ Y, int32_t* __restrict__ dev_status, uint32_t* __restrict__ ws_cnt,
+           float4* __restrict__ ws_part) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* ring = smem;
@@ -414,6 +415,48 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
                                ((a.z + b.z) + c.z) + d.z, ((a.w + b.w) + c.w) + d.w);
     }
 
+    if (ws_part != nullptr) {
+        // Split-k through the caller's workspace: each CTA stores its partial
+        // sums and counts itself in; the last of the tile's C CTAs adds the
+        // partials in rank order (the order the cluster path uses) and writes Y.
+        const int tile = static_cast<int>(blockIdx.x);
+        float4* part_g = ws_part + static_cast<int64_t>(tile) * cluster * kQ;
+        for (int e = threadIdx.x; e < m * (kRows / 4); e += kThreads) part_g[rank * kQ + e] = part4[e];
+        __syncthreads();
+        // One acquire-release add at GPU scope publishes the whole CTA's stores
+        // (ordered before it by the barrier) and, for the last CTA, makes every
+        // other CTA's partials visible to the loads below.
+        volatile int* last = reinterpret_cast<volatile int*>(part4 + kQ);  // a free word of the ring
+        if (threadIdx.x == 0) {
+            uint32_t old;
+            asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(ws_cnt + tile) : "memory");
+            *last = old == static_cast<uint32_t>(cluster - 1);
+        }
+        __syncthreads();
+        if (!*last) return;
+        for (int e = threadIdx.x; e < m * (kRows / 4); e += kThreads) {
+            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int q = 0; q < cluster; ++q) {
+                const float4 v = (q == rank) ? part4[e] : __ldcg(part_g + q * kQ + e);
+                sum = (q == 0) ? v : make_float4(sum.x + v.x, sum.y + v.y, sum.z + v.z, sum.w + v.w);
+            }
+            const int tok = e / (kRows / 4);
+            const int r = 4 * (e % (kRows / 4));
+            const float o[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int64_t grow = row0 + r + c;
+                if (grow >= n) break;
+                if (kBf16Out)
+                    reinterpret_cast<__nv_bfloat16*>(Y)[static_cast<int64_t>(tok) * n + grow] = __float2bfloat16_rn(o[c]);
+                else
+                    reinterpret_cast<float*>(Y)[static_cast<int64_t>(tok) * n + grow] = o[c];
+            }
+        }
+        if (threadIdx.x == 0) ws_cnt[tile] = 0;  // ready for the next call
+        return;
+    }
+
     // cluster split-k: rank r adds rows [r * 128 / C, (r + 1) * 128 / C) over all ranks in rank order
     cluster_sync();
     const int r_lo = (rank * kRows) / cluster;
@@ -500,11 +543,30 @@ static int gemv_cluster(int64_t n, int64_t k, int sm_count) {
     return best;
 }
 
+// Workspace layout, the same for every shape so that one buffer can serve a
+// sequence of different linears: kWsCounters 32-bit counters (one per 128-row
+// tile), then C fp32 partial tiles [16 tokens x 128 rows] per row tile.  A
+// split k only happens with at most one row tile per SM, far below kWsCounters.
+constexpr int64_t kWsCounters = 1024;
+constexpr size_t kWsCounterBytes = kWsCounters * 4;
+
+static bool gemv_ws_usable(int64_t n, int cluster) {
+    return cluster > 1 && (n + gemv::kRows - 1) / gemv::kRows <= kWsCounters;
+}
+
+size_t linear_workspace_bytes(int64_t m, int64_t n, int64_t k, const DeviceInfo& dev) {
+    if (m > kGemvMaxTokens) return 0;
+    const int cluster = gemv_cluster(n, k, dev.sm_count);
+    if (!gemv_ws_usable(n, cluster)) return 0;
+    const size_t tiles = static_cast<size_t>((n + gemv::kRows - 1) / gemv::kRows);
+    return kWsCounterBytes + tiles * cluster * 16 * gemv::kRows * sizeof(float);
+}
+
 template <bool kBf16Out, bool kM16>
 static cudaError_t launch_gemv(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const int8_t* absmax_q,
                                const float* absmax_scale, const float* absmax_offset, int mt, int64_t n,
                                int64_t k, int cluster, bool weights_early, void* Yt, int32_t* dev_status,
-                               int device, cudaStream_t stream) {
+                               void* ws, int device, cudaStream_t stream) {
     static bool attr_set[64] = {};
     if (!attr_set[device]) {
         const cudaError_t e = cudaFuncSetAttribute(gemv::k_nf4_gemv<kBf16Out, kM16>,
@@ -517,23 +579,35 @@ static cudaError_t launch_gemv(const CUtensorMap& tm_w, const CUtensorMap& tm_x,
     cfg.blockDim = dim3(gemv::kThreads, 1, 1);
     cfg.dynamicSmemBytes = gemv::kSmemBytes;
     cfg.stream = stream;
+    // With a workspace (and a split k) the CTAs of a tile need not be co-scheduled: no cluster.
+    const bool use_ws = ws != nullptr && gemv_ws_usable(n, cluster);
+    uint32_t* ws_cnt = use_ws ? static_cast<uint32_t*>(ws) : nullptr;
+    float4* ws_part = use_ws ? reinterpret_cast<float4*>(static_cast<char*>(ws) + kWsCounterBytes) : nullptr;
     cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = cluster;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    int na = 0;
+    if (!use_ws) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = 1;
+        attr[na].val.clusterDim.y = cluster;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (weights_early) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = weights_early ? 2 : 1;
+    cfg.numAttrs = na;
     return cudaLaunchKernelEx(&cfg, gemv::k_nf4_gemv<kBf16Out, kM16>, tm_w, tm_x, absmax_q, absmax_scale,
-                              absmax_offset, mt, n, k, cluster, weights_early ? 1 : 0, Yt, dev_status);
+                              absmax_offset, mt, n, k, cluster, weights_early ? 1 : 0, Yt, dev_status, ws_cnt,
+                              ws_part);
 }
 
 cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                           const float* absmax_scale, const float* absmax_offset, int64_t n,
                           int64_t k, void* Y, bool y_bf16, int32_t* dev_status, bool weights_early,
-                          const DeviceInfo& dev, cudaStream_t stream) {
+                          void* ws, const DeviceInfo& dev, cudaStream_t stream) {
     if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
     if (m > kGemvMaxTokens)
         return launch_gemm(X, m, wq, absmax_q, absmax_scale, absmax_offset, n, k, Y, y_bf16, dev_status, dev,
@@ -557,14 +631,14 @@ cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int
         void* Yt = static_cast<char*>(Y) + static_cast<size_t>(t0) * n * ybytes;
         if (y_bf16)
             e = (mt > 8) ? launch_gemv<true, true>(tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt, n, k,
-                                                   cluster, weights_early, Yt, dev_status, dev.device, stream)
+                                                   cluster, weights_early, Yt, dev_status, ws, dev.device, stream)
                          : launch_gemv<true, false>(tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt, n, k,
-                                                    cluster, weights_early, Yt, dev_status, dev.device, stream);
+                                                    cluster, weights_early, Yt, dev_status, ws, dev.device, stream);
         else
             e = (mt > 8) ? launch_gemv<false, true>(tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt, n, k,
-                                                    cluster, weights_early, Yt, dev_status, dev.device, stream)
+                                                    cluster, weights_early, Yt, dev_status, ws, dev.device, stream)
                          : launch_gemv<false, false>(tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt, n,
-                                                     k, cluster, weights_early, Yt, dev_status, dev.device, stream);
+                                                     k, cluster, weights_early, Yt, dev_status, ws, dev.device, stream);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

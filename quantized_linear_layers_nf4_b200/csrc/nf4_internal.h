@@ -33,10 +33,14 @@ cudaError_t launch_dequantize(const uint8_t* wq, const int8_t* absmax_q, const f
                               const float* absmax_offset, int64_t n_elem, void* out, bool out_bf16,
                               const DeviceInfo& dev, cudaStream_t stream);
 
+// Bytes of the split-k workspace the decode path needs for (m, n, k); 0 if none.
+size_t linear_workspace_bytes(int64_t m, int64_t n, int64_t k, const DeviceInfo& dev);
+
+// `ws` (nullable) must hold linear_workspace_bytes(m, n, k, dev) bytes, 16-byte aligned.
 cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                           const float* absmax_scale, const float* absmax_offset, int64_t n,
                           int64_t k, void* Y, bool y_bf16, int32_t* dev_status, bool weights_early,
-                          const DeviceInfo& dev, cudaStream_t stream);
+                          void* ws, const DeviceInfo& dev, cudaStream_t stream);
 
 cudaError_t launch_gemm(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                         const float* absmax_scale, const float* absmax_offset, int64_t n, int64_t k, void* Y,

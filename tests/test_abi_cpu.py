@@ -133,6 +133,19 @@ def test_weight_struct_validation(L):
     assert lex(FAKE, 0, ctypes.byref(_weight()), FAKE, 1, None, 1, None) == -2
 
 
+def test_linear_workspace_validation(L):
+    lws = L.nf4_linear_ws
+    w = ctypes.byref(_weight())
+    # a misaligned workspace is rejected before any device query
+    assert lws(FAKE, 4, w, FAKE, 1, None, 0, ODD, 1 << 20, None) == -3
+    assert lws(FAKE, 4, w, FAKE, 1, None, 4, FAKE, 1 << 20, None) == -4    # unknown flag bit
+    assert lws(FAKE, 0, w, FAKE, 1, None, 0, FAKE, 1 << 20, None) == -2
+    assert lws(None, 4, w, FAKE, 1, None, 0, None, 0, None) == -1
+    # sizes that are not a valid product need no workspace
+    assert L.nf4_linear_workspace_bytes(0, 4096, 4096) == 0
+    assert L.nf4_linear_workspace_bytes(16, 4096, 100) == 0
+
+
 def test_valid_call_without_a_gpu_reports_instead_of_crashing(L):
     """On a host without a usable B200 a fully valid call must come back with a
     status (no device / unsupported device), never crash or launch."""

@@ -200,6 +200,69 @@ def test_gemv_three_way_split_k(nf4, m):
     _check_linear(nf4, X, weight, orc)
 
 
+@pytest.mark.parametrize("n,k,m", [(4096, 4096, 16), (11008, 4096, 16), (11000, 2304, 3), (1000, 1024, 7),
+                                   (4096, 11008, 1), (300, 576, 16), (64, 128, 5)])
+def test_workspace_split_k_is_bit_identical(nf4, n, k, m):
+    """nf4_linear_ws with a workspace (CTAs meet in global memory, the last one
+    reduces) gives the same bits as the cluster path, for split-k factors
+    1, 2, 3, 4 and 8, and leaves every counter at zero."""
+    W = synth.weight_normal(n, k, seed=1200 + n + k, dtype=torch.bfloat16, device="cuda")
+    X = synth.activations(m, k, seed=1300 + m, device="cuda")
+    weight = nf4.quantize_weight(W)
+    nb = nf4.nf4_linear_workspace_bytes(m, n, k)
+    ws = nf4.linear_workspace([(n, k)], m=m)
+    ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for dtype in (torch.float32, torch.bfloat16):
+        ref = nf4.nf4_linear(X, weight, dtype)
+        for _ in range(2):   # twice: the counters must have been reset by the first call
+            got = nf4.nf4_linear(X, weight, dtype, workspace=ws, dev_status=ds)
+            torch.cuda.synchronize()
+            assert torch.equal(got.view(torch.int16) if dtype == torch.bfloat16 else got.view(torch.int32),
+                               ref.view(torch.int16) if dtype == torch.bfloat16 else ref.view(torch.int32))
+    tiles = (n + 127) // 128
+    if nb:
+        assert int(ws[: 4 * tiles].view(torch.int32).abs().sum()) == 0, "split-k counters not reset"
+    assert ds.item() == 0
+
+
+def test_workspace_errors_and_graph_reuse(nf4):
+    n, k, m = 4096, 4096, 16
+    W = synth.weight_normal(n, k, seed=1400, dtype=torch.bfloat16, device="cuda")
+    weight = nf4.quantize_weight(W)
+    X = synth.activations(m, k, seed=1401, device="cuda")
+    need = nf4.nf4_linear_workspace_bytes(m, n, k)
+    assert need > 0
+    small = torch.zeros(need // 2, dtype=torch.uint8, device="cuda")
+    with pytest.raises(nf4.NF4Error) as e:
+        nf4.nf4_linear(X, weight, torch.float32, workspace=small)
+    assert "WORKSPACE" in str(e.value)
+    # one workspace shared by a chain of launches inside a CUDA graph, with
+    # programmatic dependent launch, gives the cluster path's bits every replay
+    W2 = synth.weight_normal(11008, k, seed=1402, dtype=torch.bfloat16, device="cuda")
+    w2 = nf4.quantize_weight(W2)
+    ws = nf4.linear_workspace([(n, k), (11008, k)], m=m)
+    y1 = torch.empty(m, n, dtype=torch.bfloat16, device="cuda")
+    y2 = torch.empty(m, 11008, dtype=torch.bfloat16, device="cuda")
+    r1 = nf4.nf4_linear(X, weight, torch.bfloat16)
+    r2 = nf4.nf4_linear(X, w2, torch.bfloat16)
+
+    def step():
+        for _ in range(3):
+            nf4.nf4_linear(X, weight, torch.bfloat16, out=y1, workspace=ws, weights_early=True)
+            nf4.nf4_linear(X, w2, torch.bfloat16, out=y2, workspace=ws, weights_early=True)
+    step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for _ in range(3):
+        y1.zero_(); y2.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y1.view(torch.int16), r1.view(torch.int16))
+        assert torch.equal(y2.view(torch.int16), r2.view(torch.int16))
+
+
 def test_deterministic_and_stream_aware(nf4):
     W = synth.weight_normal(512, 1024, seed=9, dtype=torch.bfloat16, device="cuda")
     X = synth.activations(16, 1024, seed=10, device="cuda")
