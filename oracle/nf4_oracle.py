@@ -11,7 +11,7 @@ from .build_oracle import build
 
 __all__ = [
     "norm_ppf", "codebook", "quantize", "dq_sum", "dq_mean", "double_quant", "absmax_hat",
-    "dequantize", "dequantize_range", "f32_to_bf16", "bf16_to_f32", "linear_bf16", "unpack",
+    "dequantize", "dequantize_range", "f32_to_bf16", "bf16_to_f32", "linear_bf16", "linear_dx_bf16", "unpack",
     "use_library",
 ]
 
@@ -166,6 +166,20 @@ def linear_bf16(x_bf16: np.ndarray, w_bf16: np.ndarray) -> np.ndarray:
     y = np.zeros((m, n), dtype=np.float64)
     lib().orc_linear_bf16(_ptr(x), m, _ptr(w), n, k, _ptr(y))
     return y
+
+
+def linear_dx_bf16(dy_bf16: np.ndarray, w_bf16: np.ndarray) -> np.ndarray:
+    """Backward through the frozen quantized base: dX = dY * What.
+
+    Page "Tim Dettmers 如何用 bitsandbytes 與 QLoRA 降低 LLM 訓練門檻？", section
+    "QLoRA 把 frozen 4-bit base 與可訓練 adapter 分開": the 4-bit base is dequantized
+    to the compute dtype in the backward pass as in the forward one, and never
+    updated.  dy_bf16 [m, n] and w_bf16 [n, k] (the bf16 dequantized weight,
+    row-major) as uint16 bit patterns -> dX float64 [m, k] with
+    dX[i, c] = sum_r dY[i, r] * What[r, c], exact products and fp64 sums (the
+    forward linear applied to the transposed weight)."""
+    w = np.ascontiguousarray(w_bf16, dtype=np.uint16)
+    return linear_bf16(dy_bf16, np.ascontiguousarray(w.T))
 
 
 def unpack(wq: np.ndarray) -> np.ndarray:

@@ -361,3 +361,43 @@ def test_normalisation_is_a_true_division():
             assert idx[i] == _exact_argmin(f32(blk[i]) / a, c)
         found += len(cases)
     assert found > 0, "no weight distinguishes division from reciprocal multiply"
+
+
+# ---------------------------------------------------------------------------
+# Backward through the frozen base: dX = dY * What (yololab page, section
+# "QLoRA 把 frozen 4-bit base 與可訓練 adapter 分開": the base is dequantized in the
+# backward pass too).  Pinned by the adjoint identity of the forward linear and
+# by brute force on exact integer inputs.
+# ---------------------------------------------------------------------------
+
+def _bf16_bits(a):
+    return (np.asarray(a, dtype=np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def test_linear_dx_adjoint_identity():
+    """<dY, X What^T> = <dY What, X> for every X, dY: the backward product is the
+    adjoint of the forward one (a transposed or mis-indexed weight breaks it)."""
+    rng = np.random.default_rng(21)
+    for (m, n, k) in [(3, 5, 7), (4, 64, 64), (2, 96, 128)]:
+        W = _bf16_bits(rng.standard_normal((n, k)).astype(np.float32))
+        X = _bf16_bits(rng.standard_normal((m, k)).astype(np.float32))
+        dY = _bf16_bits(rng.standard_normal((m, n)).astype(np.float32))
+        y = O.linear_bf16(X, W)
+        dx = O.linear_dx_bf16(dY, W)
+        assert dx.shape == (m, k)
+        lhs = float(np.sum(O.bf16_to_f32(dY).astype(np.float64) * y))
+        rhs = float(np.sum(dx * O.bf16_to_f32(X).astype(np.float64)))
+        assert abs(lhs - rhs) <= 1e-12 * max(1.0, abs(lhs)), (lhs, rhs)
+
+
+def test_linear_dx_exact_small_integers():
+    """Small integers are exact in bf16 and their products and sums exact in
+    fp64, so dX must equal the integer matrix product computed by loops."""
+    rng = np.random.default_rng(22)
+    m, n, k = 3, 5, 4
+    Wi = rng.integers(-8, 9, size=(n, k))
+    dYi = rng.integers(-8, 9, size=(m, n))
+    dx = O.linear_dx_bf16(_bf16_bits(dYi), _bf16_bits(Wi))
+    for i in range(m):
+        for c in range(k):
+            assert dx[i, c] == sum(int(dYi[i, r]) * int(Wi[r, c]) for r in range(n))
