@@ -421,6 +421,15 @@ def run_ours(args, rank, world, local):
             del Xs, Ys
         sweep[4096] = gemm["tflops"]
         gemm["tflops_by_m"] = dict(sorted(sweep.items()))
+        # backward through the frozen base on the same weight: dX [4096, 4096] = dY [4096, 11008] * What
+        dYg = synth.activations(4096, 11008, seed=synth.seed_for(3, 7), device=dev)
+        dXg = torch.empty((4096, 4096), dtype=torch.bfloat16, device=dev)
+        fdx = lambda: nf4.nf4_linear_dx(dYg, wg, torch.bfloat16, out=dXg)
+        fdx()
+        t_dx = _events_time(fdx, 3, stream)
+        gemm["dx"] = {"m": 4096, "n": 11008, "k": 4096, "tflops": round(2.0 * 4096 * 11008 * 4096 / t_dx / 1e12, 2),
+                      "ms": round(t_dx * 1e3, 3), "frac": round(2.0 * 4096 * 11008 * 4096 / t_dx / 1e12 / pk["bf16_tflops"], 4)}
+        del dYg, dXg
         del Xg, Yg, wg
 
     # 70B-shaped stress layer: 28672 x 8192 Student-t(4) weight with outlier input

@@ -232,6 +232,26 @@ nf4_status_t nf4_linear_ex(const void* X, int64_t m, const nf4_weight_t* w, void
                            nf4_stream_t stream);
 
 /*
+ * nf4_linear_dx -- backward through the frozen quantized base:
+ * dX = dY * What, with What the bf16 dequantized weight, fused like nf4_linear:
+ * the weight is dequantized tile by tile on chip and never written out ([P1]
+ * "QLoRA 把 frozen 4-bit base 與可訓練 adapter 分開": the 4-bit base is dequantized
+ * to the compute dtype in the backward pass as in the forward one and is not
+ * updated; the gradient reaches the adapters through it).  The products
+ * dY[i][r] * What[r][c] are accumulated in fp32 in an unspecified order.  Runs
+ * a tcgen05 dequant-GEMM that contracts over the rows of W.
+ *   dY         device, bf16 [m, n], 16-byte aligned rows (n % 8 == 0 required)
+ *   m          rows of dY (tokens), >= 1
+ *   w          host struct describing the [n, k] quantized weight
+ *   dX         device, [m, k] of dx_dtype (NF4_F32 or NF4_BF16), 16-byte aligned (output)
+ *   dev_status as for nf4_linear
+ * Errors: NF4_ERR_NULL, NF4_ERR_STATE, NF4_ERR_SHAPE (m < 1, k % 64 != 0,
+ * n % 8 != 0), NF4_ERR_ALIGN, NF4_ERR_DTYPE, NF4_ERR_UNSUPPORTED, NF4_ERR_CUDA.
+ */
+nf4_status_t nf4_linear_dx(const void* dY, int64_t m, const nf4_weight_t* w, void* dX,
+                           nf4_dtype_t dx_dtype, int32_t* dev_status, nf4_stream_t stream);
+
+/*
  * nf4_linear_workspace_bytes -- bytes of the optional split-k workspace that
  * nf4_linear_ws can use for Y[m, n] = X[m, k] * What^T on the current device;
  * 0 when that product splits no k range (then no workspace is needed).  The

@@ -10,6 +10,8 @@ calls.  Functions carry the C names:
 * ``nf4_dequantize(weight, dtype)`` -> dense tensor
 * ``nf4_linear(X, weight, dtype)`` -> ``Y = X @ W_hat^T`` (optionally with a
   split-k ``workspace`` from ``linear_workspace``)
+* ``nf4_linear_dx(dY, weight, dtype)`` -> ``dX = dY @ W_hat`` (backward through
+  the frozen base)
 
 ``quantize_weight(W)`` runs the first two and returns an ``NF4Weight``.
 """
@@ -24,7 +26,7 @@ from . import _lib
 from ._lib import NF4_BF16, NF4_F32, NF4Error, nf4_weight_t
 
 __all__ = ["NF4Weight", "NF4Error", "nf4_quantize", "nf4_double_quant", "nf4_dequantize",
-           "nf4_linear", "nf4_linear_ex", "nf4_linear_workspace_bytes", "linear_workspace",
+           "nf4_linear", "nf4_linear_ex", "nf4_linear_dx", "nf4_linear_workspace_bytes", "linear_workspace",
            "quantize_weight", "nf4_codebook", "library_path"]
 
 _DTYPES = {torch.float32: NF4_F32, torch.bfloat16: NF4_BF16}
@@ -187,4 +189,23 @@ def nf4_linear(X: torch.Tensor, weight: NF4Weight, dtype=torch.bfloat16,
         ws, ws_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
     _lib.check(_lib.lib().nf4_linear_ws(_ptr(X), m, ctypes.byref(st), _ptr(out), _DTYPES[dtype], ds,
                                         flags, ws, ws_bytes, _stream(stream)), "nf4_linear_ws")
+    return out
+
+
+def nf4_linear_dx(dY: torch.Tensor, weight: NF4Weight, dtype=torch.bfloat16,
+                  out: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+                  stream=None) -> torch.Tensor:
+    """dX = dY @ W_hat for bf16 dY [m, n] (n % 8 == 0); dX [m, k] in ``dtype``."""
+    _need_cuda(dY, "dY")
+    if dY.dtype != torch.bfloat16 or dY.dim() != 2 or dY.shape[1] != weight.n:
+        raise ValueError("dY must be a 2-D bfloat16 tensor with n columns")
+    if dtype not in _DTYPES:
+        raise ValueError("dtype must be float32 or bfloat16")
+    m = dY.shape[0]
+    if out is None:
+        out = torch.empty((m, weight.k), dtype=dtype, device=dY.device)
+    st = weight.struct()
+    ds = ctypes.c_void_p(0) if dev_status is None else _ptr(dev_status)
+    _lib.check(_lib.lib().nf4_linear_dx(_ptr(dY), m, ctypes.byref(st), _ptr(out), _DTYPES[dtype], ds,
+                                        _stream(stream)), "nf4_linear_dx")
     return out

@@ -48,6 +48,7 @@ SIGNATURES = {
     "nf4_linear_ex": (ctypes.c_int, [_p, _i64, ctypes.POINTER(nf4_weight_t), _p, ctypes.c_int, _p,
                                      ctypes.c_uint32, _p]),
     "nf4_linear_workspace_bytes": (ctypes.c_size_t, [_i64, _i64, _i64]),
+    "nf4_linear_dx": (ctypes.c_int, [_p, _i64, ctypes.POINTER(nf4_weight_t), _p, ctypes.c_int, _p, _p]),
     "nf4_linear_ws": (ctypes.c_int, [_p, _i64, ctypes.POINTER(nf4_weight_t), _p, ctypes.c_int, _p,
                                      ctypes.c_uint32, _p, ctypes.c_size_t, _p]),
 }

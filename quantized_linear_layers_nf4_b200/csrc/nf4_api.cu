@@ -170,6 +170,22 @@ nf4_status_t nf4_linear_ex(const void* X, int64_t m, const nf4_weight_t* w, void
     return nf4_linear_ws(X, m, w, Y, y_dtype, dev_status, flags, nullptr, 0, stream);
 }
 
+nf4_status_t nf4_linear_dx(const void* dY, int64_t m, const nf4_weight_t* w, void* dX,
+                           nf4_dtype_t dx_dtype, int32_t* dev_status, nf4_stream_t stream) {
+    nf4_status_t st = check_weight(w);
+    if (st != NF4_OK) return st;
+    if (!dY || !dX) return NF4_ERR_NULL;
+    if (dx_dtype != NF4_F32 && dx_dtype != NF4_BF16) return NF4_ERR_DTYPE;
+    if (m < 1 || w->k % NF4_BLOCKSIZE != 0 || w->n % 8 != 0) return NF4_ERR_SHAPE;
+    if (m > INT64_MAX / w->k || m > INT64_MAX / w->n) return NF4_ERR_SHAPE;
+    if (!aligned(dY, 16) || !aligned(dX, 16) || (dev_status && !aligned(dev_status, 4))) return NF4_ERR_ALIGN;
+    nf4::DeviceInfo dev;
+    if ((st = device_ok(&dev)) != NF4_OK) return st;
+    return from_cuda(nf4::launch_gemm_dx(dY, m, w->wq, w->absmax_q, w->absmax_scale, w->absmax_offset, w->n,
+                                         w->k, dX, dx_dtype == NF4_BF16, dev_status, dev,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t nf4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k) {
     if (m < 1 || n < 1 || k < 1 || k % NF4_BLOCKSIZE != 0) return 0;
     nf4::DeviceInfo dev;

@@ -369,6 +369,257 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+// ---------------------------------------------------------------------------
+// Backward through the frozen base: dX[m, k] = dY[m, n] * What[n, k] (page "Tim
+// Dettmers 如何用 bitsandbytes 與 QLoRA 降低 LLM 訓練門檻？", section "QLoRA 把 frozen
+// 4-bit base 與可訓練 adapter 分開": the base is dequantized to the compute dtype in
+// the backward pass as in the forward one).
+//
+// One CTA computes a 256 (tokens) x 256 (columns of W) tile of dX and loops over
+// the rows of W, the contraction, 64 per stage.  The decoded tile is laid out
+// like the forward's -- rows of 64 consecutive columns, 128-byte swizzled --
+// which is the MN-major operand layout with N = columns (contiguous) and K =
+// rows: four 64-column blocks of 64 rows, 8 KB each.  Warp 0 streams dY tiles
+// [256 x 64] (K-major, like X in the forward), warp 2 the packed codes
+// [64 rows x 128 B] (swizzled, so each dequant warp's reads hit distinct
+// banks), warps 4..11 decode one (row, 64-column block) per thread per stage,
+// warp 1 issues the MMAs with the weight as the MN-major B operand.
+// ---------------------------------------------------------------------------
+constexpr int kBKX = 64;                            // rows of W per stage (MMA K)
+constexpr uint32_t kIdescDx = kIdesc | (1u << 16);  // B (the weight) MN-major
+
+// MN-major, 128-byte swizzle: the leading byte offset is the stride between
+// 64-column blocks (8 KB), the stride byte offset between 8-row groups (1 KB).
+__device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>(8192 >> 4) << 16;
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
+}
+
+template <bool kBf16Out>
+__global__ void __launch_bounds__(kThreads, 1)
+k_nf4_gemm_dx(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_w,
+              const int8_t* __restrict__ absmax_q, const float* __restrict__ absmax_scale,
+              const float* __restrict__ mu_ptr, int64_t m, int64_t n, int64_t k, void* __restrict__ dX,
+              int32_t* __restrict__ dev_status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+    uint64_t* full_a = bars;
+    uint64_t* empty_a = full_a + kStagesA;
+    uint64_t* full_b = empty_a + kStagesA;
+    uint64_t* empty_b = full_b + kStagesB;
+    uint64_t* full_p = empty_b + kStagesB;
+    uint64_t* empty_p = full_p + kStagesP;
+    uint64_t* acc_ready = empty_p + kStagesP;
+    uint64_t* drained = acc_ready + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kBN;  // first column of W (and of dX)
+    const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kBM;
+    const int nr = static_cast<int>((n + kBKX - 1) / kBKX);
+    const uint32_t sbase = smem_u32(smem);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStagesA; ++s) {
+            mbar_init(&full_a[s], 1);
+            mbar_init(&empty_a[s], 1);
+        }
+        for (int s = 0; s < kStagesB; ++s) {
+            mbar_init(&full_b[s], kDequantWarps);
+            mbar_init(&empty_b[s], 1);
+        }
+        for (int s = 0; s < kStagesP; ++s) {
+            mbar_init(&full_p[s], 1);
+            mbar_init(&empty_p[s], kDequantWarps);
+        }
+        mbar_init(acc_ready, 1);
+        mbar_init(drained, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    bool timed_out = false;
+    if (warp == 0) {
+        // ---------------------------- dY producer ----------------------------
+        if (lane == 0) {
+            prefetch_tensormap(&tm_dy);
+            int issued = 0;
+            for (int rt = 0; rt < nr; ++rt) {
+                const int s = rt % kStagesA;
+                if (rt >= kStagesA && !mbar_wait(&empty_a[s], ((rt / kStagesA) - 1) & 1)) {
+                    timed_out = true;
+                    break;
+                }
+                mbar_arrive_expect_tx(&full_a[s], kABytes);
+                tma_load_2d(smem + s * kABytes, &tm_dy, rt * kBKX, static_cast<int32_t>(m0), &full_a[s]);
+                issued = rt + 1;
+            }
+            if (timed_out)  // leave no copy in flight
+                for (int rt = (issued > kStagesA ? issued - kStagesA : 0); rt < issued; ++rt)
+                    mbar_wait(&full_a[rt % kStagesA], (rt / kStagesA) & 1);
+        }
+    } else if (warp == 2) {
+        // ------------------------ packed-weight producer ----------------------
+        if (lane == 0) {
+            prefetch_tensormap(&tm_w);
+            int issued = 0;
+            for (int rt = 0; rt < nr; ++rt) {
+                const int s = rt % kStagesP;
+                if (rt >= kStagesP && !mbar_wait(&empty_p[s], ((rt / kStagesP) - 1) & 1)) {
+                    timed_out = true;
+                    break;
+                }
+                mbar_arrive_expect_tx(&full_p[s], kPBytes);
+                tma_load_2d(smem + kOffP + s * kPBytes, &tm_w, static_cast<int32_t>(c0 / 2), rt * kBKX, &full_p[s]);
+                issued = rt + 1;
+            }
+            if (timed_out)
+                for (int rt = (issued > kStagesP ? issued - kStagesP : 0); rt < issued; ++rt)
+                    mbar_wait(&full_p[rt % kStagesP], (rt / kStagesP) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------ MMA issuer ----------------------------
+        if (lane == 0) {
+            for (int rt = 0; rt < nr; ++rt) {
+                const int sa = rt % kStagesA;
+                const int sb = rt % kStagesB;
+                if (!mbar_wait(&full_a[sa], (rt / kStagesA) & 1) || !mbar_wait(&full_b[sb], (rt / kStagesB) & 1)) {
+                    timed_out = true;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a_addr = sbase + sa * kABytes;
+                const uint32_t b_addr = sbase + kOffB + sb * kBBytes;
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int j = 0; j < kBKX / 16; ++j)
+                        tc_mma_bf16(tmem + h * 256, smem_desc_sw128(a_addr + h * (128 * 128) + 32 * j),
+                                    smem_desc_sw128_mn(b_addr + 2048 * j), kIdescDx, (rt > 0 || j > 0) ? 1u : 0u);
+                tc_commit(&empty_a[sa]);
+                tc_commit(&empty_b[sb]);
+            }
+            tc_commit(timed_out ? drained : acc_ready);
+            if (timed_out) mbar_wait(drained, 0);  // issued MMAs finish before TMEM is freed
+        }
+    } else if (warp >= 4) {
+        // ------------------------ dequantize, then epilogue --------------------
+        const int t = threadIdx.x - 128;
+        const int r = t & (kBKX - 1);  // row of the stage
+        const int cb = t >> 6;         // 64-column block of the tile
+        const int64_t kblocks = k / 64;
+        int64_t colblk = c0 / 64 + cb;  // blocks past k: computed, never stored
+        if (colblk > kblocks - 1) colblk = kblocks - 1;
+        const float mu = __ldg(mu_ptr);
+        uint64_t cpair[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) cpair[j] = pack_f32x2(kLevels[2 * j], kLevels[2 * j + 1]);
+        const uint32_t swz = static_cast<uint32_t>(r & 7);
+        const uint32_t prow = sbase + kOffP + r * 128;
+        const uint32_t brow = sbase + kOffB + cb * (kBKX * 128) + r * 128;
+        // absmax inputs of (row rt * 64 + r, colblk), one stage ahead; rows past
+        // n are clamped (their codes and dY are zero-filled, so they add nothing)
+        auto row_of = [&](int rt) {
+            const int64_t row = static_cast<int64_t>(rt) * kBKX + r;
+            return row < n ? row : n - 1;
+        };
+        int64_t bidx = row_of(0) * kblocks + colblk;
+        int q_next = __ldg(absmax_q + bidx);
+        float s_next = __ldg(absmax_scale + (bidx >> 8));
+        for (int rt = 0; rt < nr; ++rt) {
+            const int sp = rt % kStagesP;
+            const int sb = rt % kStagesB;
+            const int q = q_next;
+            const float sc = s_next;
+            bidx = row_of(rt + 1 < nr ? rt + 1 : rt) * kblocks + colblk;
+            q_next = __ldg(absmax_q + bidx);
+            s_next = __ldg(absmax_scale + (bidx >> 8));
+            if (!__all_sync(kFull, mbar_wait(&full_p[sp], (rt / kStagesP) & 1))) {
+                timed_out = true;
+                break;
+            }
+            const uint4 r0 = lds128(prow + sp * kPBytes + ((((2 * cb) ^ static_cast<int>(swz))) << 4));
+            const uint4 r1 = lds128(prow + sp * kPBytes + ((((2 * cb + 1) ^ static_cast<int>(swz))) << 4));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty_p[sp]);
+            Planes P;
+            build_planes(cpair, absmax_hat(q, sc, mu), P);
+            if (rt >= kStagesB && !__all_sync(kFull, mbar_wait(&empty_b[sb], ((rt / kStagesB) - 1) & 1))) {
+                timed_out = true;
+                break;
+            }
+            const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+            const uint32_t bst = brow + sb * kBBytes;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint32_t x = w[c] ^ 0x88888888u;
+                uint32_t o0, o1, o2, o3;
+                decode4(w[c], x, P, o0, o1);
+                decode4(w[c] >> 16, x >> 16, P, o2, o3);
+                sts128(bst + ((c ^ swz) << 4), o0, o1, o2, o3);
+            }
+            fence_proxy_async_shared();  // generic-proxy writes -> tensor-core reads
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full_b[sb]);
+        }
+        // epilogue: accumulators -> dX
+        const bool ok = !timed_out && __all_sync(kFull, mbar_wait(acc_ready, 0));
+        if (!ok) timed_out = true;
+        tc_fence_after();
+        const int wd = warp - 4;
+        const int half = wd >> 2;
+        const int quarter = warp & 3;  // tensor-memory lanes this warp may access
+        const int64_t tok = m0 + half * 128 + quarter * 32 + lane;
+        const bool vec = kBf16Out ? (k % 8 == 0) : (k % 4 == 0);
+#pragma unroll 1
+        for (int cc = 0; cc < kBN / 32; ++cc) {
+            uint32_t rr[32];
+            if (ok) tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * 256 + cc * 32, rr);
+            const int64_t col0 = c0 + cc * 32;
+            if (!ok || tok >= m || col0 >= k) continue;
+            if (kBf16Out) {
+                __nv_bfloat16* drow = reinterpret_cast<__nv_bfloat16*>(dX) + tok * k;
+                if (vec && col0 + 32 <= k) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = pack_bf16x2(__uint_as_float(rr[2 * e]), __uint_as_float(rr[2 * e + 1]));
+                    uint4* dst = reinterpret_cast<uint4*>(drow + col0);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                } else {
+                    for (int e = 0; e < 32 && col0 + e < k; ++e) drow[col0 + e] = __float2bfloat16_rn(__uint_as_float(rr[e]));
+                }
+            } else {
+                float* drow = reinterpret_cast<float*>(dX) + tok * k;
+                if (vec && col0 + 32 <= k) {
+                    uint4* dst = reinterpret_cast<uint4*>(drow + col0);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) dst[e] = make_uint4(rr[4 * e], rr[4 * e + 1], rr[4 * e + 2], rr[4 * e + 3]);
+                } else {
+                    for (int e = 0; e < 32 && col0 + e < k; ++e) drow[col0 + e] = __uint_as_float(rr[e]);
+                }
+            }
+        }
+    }
+    if (timed_out) record_timeout(dev_status);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
 }  // namespace gemm
 
 cudaError_t launch_gemm(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
@@ -399,6 +650,39 @@ cudaError_t launch_gemm(const void* X, int64_t m, const uint8_t* wq, const int8_
     else
         gemm::k_nf4_gemm<false><<<grid, gemm::kThreads, gemm::kSmemBytes, stream>>>(
             tm_x, tm_w, absmax_q, absmax_scale, absmax_offset, m, n, k, Y, dev_status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_dx(const void* dY, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
+                           const float* absmax_scale, const float* absmax_offset, int64_t n, int64_t k, void* dX,
+                           bool dx_bf16, int32_t* dev_status, const DeviceInfo& dev, cudaStream_t stream) {
+    static bool attr_set[64][2] = {};
+    if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
+    const void* fn = dx_bf16 ? reinterpret_cast<const void*>(&gemm::k_nf4_gemm_dx<true>)
+                             : reinterpret_cast<const void*>(&gemm::k_nf4_gemm_dx<false>);
+    if (!attr_set[dev.device][dx_bf16]) {
+        const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set[dev.device][dx_bf16] = true;
+    }
+    CUtensorMap tm_dy, tm_w;
+    // dY [m, n] bf16, K-major boxes [256 tokens x 64 rows of W]
+    cudaError_t e = tmap_2d(&tm_dy, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, static_cast<uint64_t>(n),
+                            static_cast<uint64_t>(m), static_cast<uint64_t>(n * 2), gemm::kBKX, gemm::kBM,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    // codes [n, k/2] bytes, boxes [64 rows x 128 B] (256 columns), 128-byte swizzled
+    e = tmap_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n),
+                static_cast<uint64_t>(k / 2), gemm::kBN / 2, gemm::kBKX, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    const dim3 grid(static_cast<unsigned>((k + gemm::kBN - 1) / gemm::kBN),
+                    static_cast<unsigned>((m + gemm::kBM - 1) / gemm::kBM));
+    if (dx_bf16)
+        gemm::k_nf4_gemm_dx<true><<<grid, gemm::kThreads, gemm::kSmemBytes, stream>>>(
+            tm_dy, tm_w, absmax_q, absmax_scale, absmax_offset, m, n, k, dX, dev_status);
+    else
+        gemm::k_nf4_gemm_dx<false><<<grid, gemm::kThreads, gemm::kSmemBytes, stream>>>(
+            tm_dy, tm_w, absmax_q, absmax_scale, absmax_offset, m, n, k, dX, dev_status);
     return cudaGetLastError();
 }
 

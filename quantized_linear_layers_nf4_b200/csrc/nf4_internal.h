@@ -42,6 +42,10 @@ cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int
                           int64_t k, void* Y, bool y_bf16, int32_t* dev_status, bool weights_early,
                           void* ws, const DeviceInfo& dev, cudaStream_t stream);
 
+cudaError_t launch_gemm_dx(const void* dY, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
+                           const float* absmax_scale, const float* absmax_offset, int64_t n, int64_t k, void* dX,
+                           bool dx_bf16, int32_t* dev_status, const DeviceInfo& dev, cudaStream_t stream);
+
 cudaError_t launch_gemm(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                         const float* absmax_scale, const float* absmax_offset, int64_t n, int64_t k, void* Y,
                         bool y_bf16, int32_t* dev_status, const DeviceInfo& dev, cudaStream_t stream);

@@ -146,6 +146,16 @@ def test_linear_workspace_validation(L):
     assert L.nf4_linear_workspace_bytes(16, 4096, 100) == 0
 
 
+def test_linear_dx_validation(L):
+    dx = L.nf4_linear_dx
+    assert dx(None, 4, ctypes.byref(_weight()), FAKE, 1, None, None) == -1
+    assert dx(FAKE, 0, ctypes.byref(_weight()), FAKE, 1, None, None) == -2
+    assert dx(FAKE, 4, ctypes.byref(_weight(n=100, k=64)), FAKE, 1, None, None) == -2   # n % 8 != 0
+    assert dx(FAKE, 4, ctypes.byref(_weight()), FAKE, 9, None, None) == -4
+    assert dx(ODD, 4, ctypes.byref(_weight()), FAKE, 1, None, None) == -3
+    assert dx(FAKE, 4, ctypes.byref(_weight(magic=7)), FAKE, 1, None, None) == -5
+
+
 def test_valid_call_without_a_gpu_reports_instead_of_crashing(L):
     """On a host without a usable B200 a fully valid call must come back with a
     status (no device / unsupported device), never crash or launch."""

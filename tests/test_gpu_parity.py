@@ -263,6 +263,55 @@ def test_workspace_errors_and_graph_reuse(nf4):
         assert torch.equal(y2.view(torch.int16), r2.view(torch.int16))
 
 
+def _check_dx(nf4, dY, weight, orc, token_rows=None, tol=LINEAR_TOL):
+    """nf4_linear_dx vs the oracle's fp64 dX = dY * What on the bf16-dequantized
+    weight (every column, the sampled token rows)."""
+    owq, oq, os_, omu = orc
+    m, n = dY.shape
+    k = weight.k
+    T = np.arange(m) if token_rows is None else np.asarray(token_rows)
+    D32 = nf4.nf4_linear_dx(dY, weight, torch.float32)
+    D16 = nf4.nf4_linear_dx(dY, weight, torch.bfloat16)
+    torch.cuda.synchronize()
+    what = O.f32_to_bf16(O.dequantize_range(owq, oq, os_, omu, 0, n * k)).reshape(n, k)
+    ref = O.linear_dx_bf16(np.ascontiguousarray(_bits(dY).reshape(m, n)[T]), what)
+    d32 = D32.cpu().numpy()[T]
+    e32 = _rel_fro(d32, ref)
+    assert e32 <= tol, "dX fp32 rel-Frobenius %.3g > %.3g" % (e32, tol)
+    d16 = D16.float().cpu().numpy()[T]
+    d32r = torch.from_numpy(np.ascontiguousarray(d32)).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(d16, d32r), "bf16 dX is not the rounded fp32 dX"
+    return e32
+
+
+@pytest.mark.parametrize("m,n,k", [(17, 64, 64), (257, 136, 320), (300, 520, 640), (64, 8, 128),
+                                   (513, 2048, 256), (1, 200, 576)])
+def test_linear_dx_ragged(nf4, m, n, k):
+    """Backward through the frozen base, dX = dY * What: ragged token, row
+    (contraction) and column tiles."""
+    W = synth.weight_normal(n, k, seed=1500 + n + k, dtype=torch.bfloat16, device="cuda")
+    dY = synth.activations(m, n, seed=1600 + m, device="cuda")
+    weight, orc = _check_quant(nf4, W, full_dequant=False, rows=[0, n - 1])
+    _check_dx(nf4, dY, weight, orc)
+
+
+def test_linear_dx_prefill_shape(nf4):
+    """dX for the MLP down/up shapes at 4096 tokens: W 11008 x 4096, dY 4096 x 11008."""
+    m, n, k = 4096, 11008, 4096
+    W = synth.weight_normal(n, k, seed=synth.seed_for(3, 0), dtype=torch.bfloat16, device="cuda")
+    dY = synth.activations(m, n, seed=synth.seed_for(3, 7), device="cuda")
+    weight, orc = _check_quant(nf4, W, full_dequant=False, rows=_sample_rows(n, 16, 3))
+    _check_dx(nf4, dY, weight, orc, token_rows=_sample_rows(m, 12, 41))
+
+
+def test_linear_dx_errors(nf4):
+    W = synth.weight_normal(100, 64, seed=1700, dtype=torch.bfloat16, device="cuda")   # n % 8 != 0
+    weight = nf4.quantize_weight(W)
+    dY = synth.activations(4, 100, seed=1701, device="cuda")
+    with pytest.raises(nf4.NF4Error):
+        nf4.nf4_linear_dx(dY, weight, torch.float32)
+
+
 def test_deterministic_and_stream_aware(nf4):
     W = synth.weight_normal(512, 1024, seed=9, dtype=torch.bfloat16, device="cuda")
     X = synth.activations(16, 1024, seed=10, device="cuda")
