@@ -11,7 +11,7 @@ from .build_oracle import build
 
 __all__ = [
     "norm_ppf", "codebook", "quantize", "dq_sum", "dq_mean", "double_quant", "absmax_hat",
-    "dequantize", "dequantize_range", "f32_to_bf16", "bf16_to_f32", "linear_bf16", "linear_dx_bf16", "unpack",
+    "dequantize", "dequantize_range", "f32_to_bf16", "bf16_to_f32", "linear_bf16", "linear_dx_bf16", "linear_lora_bf16", "unpack",
     "use_library",
 ]
 
@@ -180,6 +180,26 @@ def linear_dx_bf16(dy_bf16: np.ndarray, w_bf16: np.ndarray) -> np.ndarray:
     forward linear applied to the transposed weight)."""
     w = np.ascontiguousarray(w_bf16, dtype=np.uint16)
     return linear_bf16(dy_bf16, np.ascontiguousarray(w.T))
+
+
+def linear_lora_bf16(x_bf16: np.ndarray, w_bf16: np.ndarray, down_bf16: np.ndarray, up_bf16: np.ndarray,
+                     scale: float) -> np.ndarray:
+    """The QLoRA layer: the frozen quantized base plus a low-rank update.
+
+    Page "LLM 相關知識" (technicalnotes), section "2-2. LoRA（低秩適應）": the
+    frozen W is used as W + dW with dW = A x B of rank r (A: out x r, B: r x in),
+    trained in bf16; section 4: the base is frozen INT4, the LoRA matrices bf16.
+    With W [n, k] (rows = outputs): dW = up [n, r] * down [r, k], and
+        Y = X What^T + scale * (X down^T) up^T
+    in fp64 with exact products (scale as given, e.g. lora_alpha / r).
+    x_bf16 [m, k], w_bf16 [n, k], down_bf16 [r, k], up_bf16 [n, r] as uint16 bit
+    patterns -> Y float64 [m, n]."""
+    base = linear_bf16(x_bf16, w_bf16)
+    x = bf16_to_f32(x_bf16).astype(np.float64)
+    down = bf16_to_f32(down_bf16).astype(np.float64)
+    up = bf16_to_f32(up_bf16).astype(np.float64)
+    t = x @ down.T                       # [m, r]: the low-rank projection of X
+    return base + float(scale) * (t @ up.T)
 
 
 def unpack(wq: np.ndarray) -> np.ndarray:

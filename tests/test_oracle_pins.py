@@ -401,3 +401,48 @@ def test_linear_dx_exact_small_integers():
     for i in range(m):
         for c in range(k):
             assert dx[i, c] == sum(int(dYi[i, r]) * int(Wi[r, c]) for r in range(n))
+
+
+# ---------------------------------------------------------------------------
+# LoRA layer: Y = X What^T + s (X down^T) up^T (technicalnotes page, sections
+# "2-2. LoRA" and 4).  Pinned by the zero-scale case, by the merged-weight
+# identity W' = What + s up down, and by integer brute force.
+# ---------------------------------------------------------------------------
+
+def test_linear_lora_zero_scale_is_the_base_linear():
+    rng = np.random.default_rng(31)
+    m, n, k, r = 3, 40, 64, 4
+    X = _bf16_bits(rng.standard_normal((m, k)))
+    W = _bf16_bits(rng.standard_normal((n, k)))
+    D = _bf16_bits(rng.standard_normal((r, k)))
+    U = _bf16_bits(rng.standard_normal((n, r)))
+    assert np.array_equal(O.linear_lora_bf16(X, W, D, U, 0.0), O.linear_bf16(X, W))
+
+
+def test_linear_lora_equals_the_merged_weight():
+    """X (What + s up down)^T computed directly (merge first, then multiply)
+    agrees with the layer's low-rank path to fp64 rounding."""
+    rng = np.random.default_rng(32)
+    for (m, n, k, r, s) in [(2, 24, 64, 3, 2.0), (4, 64, 128, 16, 0.5)]:
+        X = _bf16_bits(rng.standard_normal((m, k)))
+        W = _bf16_bits(rng.standard_normal((n, k)))
+        D = _bf16_bits(rng.standard_normal((r, k)))
+        U = _bf16_bits(rng.standard_normal((n, r)))
+        y = O.linear_lora_bf16(X, W, D, U, s)
+        wm = O.bf16_to_f32(W).astype(np.float64) + s * (O.bf16_to_f32(U).astype(np.float64)
+                                                         @ O.bf16_to_f32(D).astype(np.float64))
+        ym = O.bf16_to_f32(X).astype(np.float64) @ wm.T
+        assert np.allclose(y, ym, rtol=1e-12, atol=1e-12)
+
+
+def test_linear_lora_exact_small_integers():
+    rng = np.random.default_rng(33)
+    m, n, k, r = 2, 3, 5, 2
+    Xi, Wi = rng.integers(-4, 5, size=(m, k)), rng.integers(-4, 5, size=(n, k))
+    Di, Ui = rng.integers(-4, 5, size=(r, k)), rng.integers(-4, 5, size=(n, r))
+    y = O.linear_lora_bf16(_bf16_bits(Xi), _bf16_bits(Wi), _bf16_bits(Di), _bf16_bits(Ui), 3.0)
+    for i in range(m):
+        for o in range(n):
+            base = sum(int(Xi[i, c]) * int(Wi[o, c]) for c in range(k))
+            low = sum(sum(int(Xi[i, c]) * int(Di[j, c]) for c in range(k)) * int(Ui[o, j]) for j in range(r))
+            assert y[i, o] == base + 3 * low
