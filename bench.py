@@ -430,6 +430,26 @@ def run_ours(args, rank, world, local):
         gemm["dx"] = {"m": 4096, "n": 11008, "k": 4096, "tflops": round(2.0 * 4096 * 11008 * 4096 / t_dx / 1e12, 2),
                       "ms": round(t_dx * 1e3, 3), "frac": round(2.0 * 4096 * 11008 * 4096 / t_dx / 1e12 / pk["bf16_tflops"], 4)}
         del dYg, dXg
+        # the QLoRA layer (r = 16, scale = lora_alpha / r = 32 / 16) against the plain linear:
+        # decode on a q_proj-shaped weight at m = 16, prefill on this weight at m = 4096
+        rl = 16
+        lora = {"r": rl, "scale": 2.0}
+        for tag, wl, ml in (("decode_4096x4096_m16", weights[0], 16), ("prefill_11008x4096_m4096", wg, 4096)):
+            Xl = synth.activations(ml, wl.k, seed=synth.seed_for(3, 8) + ml, device=dev)
+            Yl = torch.empty((ml, wl.n), dtype=torch.bfloat16, device=dev)
+            dl = (synth.activations(rl, wl.k, seed=synth.seed_for(3, 9), device=dev).float() * 0.02).to(torch.bfloat16)
+            ul = (synth.activations(wl.n, rl, seed=synth.seed_for(3, 10), device=dev).float() * 0.02).to(torch.bfloat16)
+            wsl = nf4.lora_workspace(ml, [(wl.n, wl.k)], rl, device=dev)
+            wsp = nf4.linear_workspace([(wl.n, wl.k)], m=ml, device=dev)
+            f_l = lambda: nf4.nf4_linear_lora(Xl, wl, dl, ul, 2.0, wsl, out=Yl)
+            f_p = lambda: nf4.nf4_linear(Xl, wl, torch.bfloat16, out=Yl, workspace=wsp)
+            f_l(); f_p()
+            t_l = _events_time(f_l, 20, stream)
+            t_p = _events_time(f_p, 20, stream)
+            lora[tag] = {"us_lora": round(t_l * 1e6, 2), "us_plain": round(t_p * 1e6, 2),
+                         "overhead": round(t_l / t_p - 1.0, 4)}
+            del Xl, Yl, dl, ul, wsl, wsp
+        gemm["lora"] = lora
         del Xg, Yg, wg
 
     # 70B-shaped stress layer: 28672 x 8192 Student-t(4) weight with outlier input

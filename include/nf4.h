@@ -252,6 +252,39 @@ nf4_status_t nf4_linear_dx(const void* dY, int64_t m, const nf4_weight_t* w, voi
                            nf4_dtype_t dx_dtype, int32_t* dev_status, nf4_stream_t stream);
 
 /*
+ * nf4_linear_lora_workspace_bytes -- bytes of the workspace nf4_linear_lora
+ * needs for m tokens, an [n, k] weight and rank r: the low-rank projection
+ * t [m, r] (fp32), then the split-k area of nf4_linear_ws.  0 for invalid sizes.
+ */
+size_t nf4_linear_lora_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t r);
+
+/*
+ * nf4_linear_lora -- the QLoRA layer: the frozen quantized base plus a trained
+ * low-rank update, Y = X * What^T + scale * (X * down^T) * up^T ([P4] "2-2. LoRA
+ * （低秩適應）": W acts as W + dW with dW = A x B of rank r; section 4: base frozen
+ * INT4, LoRA matrices bf16).  With W stored [n, k], dW = up * down.
+ * t = scale * X down^T is computed first (fp32, fixed summation order); the
+ * linear then adds sum_j t[i][j] * up[o][j] (j in order, fp32) to each fp32
+ * output before rounding it to y_dtype.  Same path and flags as nf4_linear_ws.
+ *   X          device, bf16 [m, k], 16-byte aligned
+ *   w          the [n, k] quantized weight
+ *   lora_down  device, bf16 [r, k] row-major (PEFT's lora_A.weight), 16-byte aligned
+ *   lora_up    device, bf16 [n, r] row-major (PEFT's lora_B.weight), 16-byte aligned
+ *   r          rank, 1 .. 256
+ *   scale      e.g. lora_alpha / r
+ *   Y          device, [m, n] of y_dtype, 16-byte aligned (output)
+ *   dev_status, flags  as for nf4_linear_ex
+ *   workspace  device, 16-byte aligned, >= nf4_linear_lora_workspace_bytes(m, n,
+ *              k, r) bytes, zero-filled before first use (as for nf4_linear_ws)
+ * Errors: as nf4_linear_ws; NF4_ERR_NULL also for a missing LoRA matrix or
+ * workspace; NF4_ERR_SHAPE for r out of range.
+ */
+nf4_status_t nf4_linear_lora(const void* X, int64_t m, const nf4_weight_t* w, const void* lora_down,
+                             const void* lora_up, int32_t r, float scale, void* Y, nf4_dtype_t y_dtype,
+                             int32_t* dev_status, uint32_t flags, void* workspace, size_t ws_bytes,
+                             nf4_stream_t stream);
+
+/*
  * nf4_linear_workspace_bytes -- bytes of the optional split-k workspace that
  * nf4_linear_ws can use for Y[m, n] = X[m, k] * What^T on the current device;
  * 0 when that product splits no k range (then no workspace is needed).  The

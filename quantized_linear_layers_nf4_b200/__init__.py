@@ -12,6 +12,8 @@ calls.  Functions carry the C names:
   split-k ``workspace`` from ``linear_workspace``)
 * ``nf4_linear_dx(dY, weight, dtype)`` -> ``dX = dY @ W_hat`` (backward through
   the frozen base)
+* ``nf4_linear_lora(X, weight, down, up, scale, workspace=...)`` -> the QLoRA
+  layer ``X @ W_hat^T + scale * (X @ down^T) @ up^T``
 
 ``quantize_weight(W)`` runs the first two and returns an ``NF4Weight``.
 """
@@ -26,7 +28,8 @@ from . import _lib
 from ._lib import NF4_BF16, NF4_F32, NF4Error, nf4_weight_t
 
 __all__ = ["NF4Weight", "NF4Error", "nf4_quantize", "nf4_double_quant", "nf4_dequantize",
-           "nf4_linear", "nf4_linear_ex", "nf4_linear_dx", "nf4_linear_workspace_bytes", "linear_workspace",
+           "nf4_linear", "nf4_linear_ex", "nf4_linear_dx", "nf4_linear_lora", "lora_workspace",
+           "nf4_linear_workspace_bytes", "linear_workspace",
            "quantize_weight", "nf4_codebook", "library_path"]
 
 _DTYPES = {torch.float32: NF4_F32, torch.bfloat16: NF4_BF16}
@@ -208,4 +211,40 @@ def nf4_linear_dx(dY: torch.Tensor, weight: NF4Weight, dtype=torch.bfloat16,
     ds = ctypes.c_void_p(0) if dev_status is None else _ptr(dev_status)
     _lib.check(_lib.lib().nf4_linear_dx(_ptr(dY), m, ctypes.byref(st), _ptr(out), _DTYPES[dtype], ds,
                                         _stream(stream)), "nf4_linear_dx")
+    return out
+
+
+def lora_workspace(m: int, shapes, r: int, device=None) -> torch.Tensor:
+    """A zero-filled workspace for nf4_linear_lora at m tokens and rank r on every
+    (n, k) in ``shapes``."""
+    L = _lib.lib()
+    nbytes = max([int(L.nf4_linear_lora_workspace_bytes(m, n, k, r)) for n, k in shapes] + [16])
+    return torch.zeros((nbytes + 15) // 16 * 16, dtype=torch.uint8, device=device or "cuda")
+
+
+def nf4_linear_lora(X: torch.Tensor, weight: NF4Weight, down: torch.Tensor, up: torch.Tensor, scale: float,
+                    workspace: torch.Tensor, dtype=torch.bfloat16, out: torch.Tensor | None = None,
+                    dev_status: torch.Tensor | None = None, stream=None,
+                    weights_early: bool = False) -> torch.Tensor:
+    """Y = X @ W_hat^T + scale * (X @ down^T) @ up^T with down bf16 [r, k] and up
+    bf16 [n, r]; ``workspace`` from ``lora_workspace``."""
+    for t, name in ((X, "X"), (down, "down"), (up, "up"), (workspace, "workspace")):
+        _need_cuda(t, name)
+    if X.dtype != torch.bfloat16 or down.dtype != torch.bfloat16 or up.dtype != torch.bfloat16:
+        raise ValueError("X, down and up must be bfloat16")
+    r = down.shape[0]
+    if down.shape != (r, weight.k) or up.shape != (weight.n, r) or X.shape[1] != weight.k:
+        raise ValueError("shapes: X [m, k], down [r, k], up [n, r]")
+    if dtype not in _DTYPES:
+        raise ValueError("dtype must be float32 or bfloat16")
+    m = X.shape[0]
+    if out is None:
+        out = torch.empty((m, weight.n), dtype=dtype, device=X.device)
+    st = weight.struct()
+    ds = ctypes.c_void_p(0) if dev_status is None else _ptr(dev_status)
+    flags = _lib.NF4_LINEAR_WEIGHTS_EARLY if weights_early else 0
+    _lib.check(_lib.lib().nf4_linear_lora(_ptr(X), m, ctypes.byref(st), _ptr(down), _ptr(up), r, float(scale),
+                                          _ptr(out), _DTYPES[dtype], ds, flags, _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _stream(stream)),
+               "nf4_linear_lora")
     return out

@@ -49,6 +49,10 @@ SIGNATURES = {
                                      ctypes.c_uint32, _p]),
     "nf4_linear_workspace_bytes": (ctypes.c_size_t, [_i64, _i64, _i64]),
     "nf4_linear_dx": (ctypes.c_int, [_p, _i64, ctypes.POINTER(nf4_weight_t), _p, ctypes.c_int, _p, _p]),
+    "nf4_linear_lora_workspace_bytes": (ctypes.c_size_t, [_i64, _i64, _i64, ctypes.c_int32]),
+    "nf4_linear_lora": (ctypes.c_int, [_p, _i64, ctypes.POINTER(nf4_weight_t), _p, _p, ctypes.c_int32,
+                                       ctypes.c_float, _p, ctypes.c_int, _p, ctypes.c_uint32, _p, ctypes.c_size_t,
+                                       _p]),
     "nf4_linear_ws": (ctypes.c_int, [_p, _i64, ctypes.POINTER(nf4_weight_t), _p, ctypes.c_int, _p,
                                      ctypes.c_uint32, _p, ctypes.c_size_t, _p]),
 }

@@ -143,6 +143,48 @@ nf4_status_t nf4_dequantize(const nf4_weight_t* w, void* out, nf4_dtype_t out_dt
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
+static size_t lora_t_bytes(int64_t m, int32_t r) {
+    return (static_cast<size_t>(m) * static_cast<size_t>(r) * sizeof(float) + 255) / 256 * 256;
+}
+
+nf4_status_t nf4_linear_lora(const void* X, int64_t m, const nf4_weight_t* w, const void* lora_down,
+                             const void* lora_up, int32_t r, float scale, void* Y, nf4_dtype_t y_dtype,
+                             int32_t* dev_status, uint32_t flags, void* workspace, size_t ws_bytes,
+                             nf4_stream_t stream) {
+    nf4_status_t st = check_weight(w);
+    if (st != NF4_OK) return st;
+    if (!X || !Y || !lora_down || !lora_up || !workspace) return NF4_ERR_NULL;
+    if (y_dtype != NF4_F32 && y_dtype != NF4_BF16) return NF4_ERR_DTYPE;
+    if ((flags & ~static_cast<uint32_t>(NF4_LINEAR_WEIGHTS_EARLY)) != 0) return NF4_ERR_DTYPE;
+    if (m < 1 || w->k % NF4_BLOCKSIZE != 0 || r < 1 || r > 256) return NF4_ERR_SHAPE;
+    if (m > INT64_MAX / w->k || m > INT64_MAX / w->n || m > INT64_MAX / 1024) return NF4_ERR_SHAPE;
+    if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(lora_down, 16) || !aligned(lora_up, 16) ||
+        !aligned(workspace, 16) || (dev_status && !aligned(dev_status, 4)))
+        return NF4_ERR_ALIGN;
+    nf4::DeviceInfo dev;
+    if ((st = device_ok(&dev)) != NF4_OK) return st;
+    const size_t tb = lora_t_bytes(m, r);
+    if (ws_bytes < tb + nf4::linear_workspace_bytes(m, w->n, w->k, dev)) return NF4_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    float* t = static_cast<float*>(workspace);
+    st = from_cuda(nf4::launch_lora_down(X, m, w->k, lora_down, r, scale, t, s));
+    if (st != NF4_OK) return st;
+    nf4::LoraArgs lora;
+    lora.t = t;
+    lora.up = static_cast<const __nv_bfloat16*>(lora_up);
+    lora.r = r;
+    return from_cuda(nf4::launch_linear(X, m, w->wq, w->absmax_q, w->absmax_scale, w->absmax_offset, w->n, w->k,
+                                        Y, y_dtype == NF4_BF16, dev_status, (flags & NF4_LINEAR_WEIGHTS_EARLY) != 0,
+                                        static_cast<char*>(workspace) + tb, lora, dev, s));
+}
+
+size_t nf4_linear_lora_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t r) {
+    if (m < 1 || n < 1 || k < 1 || k % NF4_BLOCKSIZE != 0 || r < 1 || r > 256) return 0;
+    nf4::DeviceInfo dev;
+    if (device_ok(&dev) != NF4_OK) return 0;
+    return lora_t_bytes(m, r) + nf4::linear_workspace_bytes(m, n, k, dev);
+}
+
 nf4_status_t nf4_linear_ws(const void* X, int64_t m, const nf4_weight_t* w, void* Y,
                            nf4_dtype_t y_dtype, int32_t* dev_status, uint32_t flags, void* workspace,
                            size_t ws_bytes, nf4_stream_t stream) {
@@ -161,7 +203,7 @@ nf4_status_t nf4_linear_ws(const void* X, int64_t m, const nf4_weight_t* w, void
     if (workspace && ws_bytes < nf4::linear_workspace_bytes(m, w->n, w->k, dev)) return NF4_ERR_WORKSPACE;
     return from_cuda(nf4::launch_linear(X, m, w->wq, w->absmax_q, w->absmax_scale, w->absmax_offset,
                                         w->n, w->k, Y, y_dtype == NF4_BF16, dev_status,
-                                        (flags & NF4_LINEAR_WEIGHTS_EARLY) != 0, workspace, dev,
+                                        (flags & NF4_LINEAR_WEIGHTS_EARLY) != 0, workspace, nf4::LoraArgs(), dev,
                                         reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -136,12 +136,13 @@ __device__ __forceinline__ void decode4(uint32_t s, uint32_t sx, const Planes& P
     o1 = prmt(l, h, 0x6273);
 }
 
-template <bool kBf16Out>
+template <bool kBf16Out, bool kLora>
 __global__ void __launch_bounds__(kThreads, 1)
 k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
            const int8_t* __restrict__ absmax_q, const float* __restrict__ absmax_scale,
            const float* __restrict__ mu_ptr, int64_t m, int64_t n, int64_t k, void* __restrict__ Y,
-           int32_t* __restrict__ dev_status) {
+           int32_t* __restrict__ dev_status, const float* __restrict__ lora_t,
+           const __nv_bfloat16* __restrict__ lora_up, int lora_r) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -337,6 +338,40 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             if (ok) tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * 256 + cc * 32, r);
             const int64_t col0 = n0 + cc * 32;
             if (!ok || tok >= m || col0 >= n) continue;
+            if (kLora) {
+                // low-rank term: + sum_j t[tok, j] * up[col, j], j ascending for every column
+                const float* tr = lora_t + tok * lora_r;
+                if ((lora_r & 7) == 0) {  // 16-byte aligned rows: 8 ranks per load
+                    for (int j = 0; j < lora_r; j += 8) {
+                        const float4 t0 = __ldg(reinterpret_cast<const float4*>(tr + j));
+                        const float4 t1 = __ldg(reinterpret_cast<const float4*>(tr + j + 4));
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            if (col0 + e >= n) continue;
+                            const uint4 u = __ldg(reinterpret_cast<const uint4*>(lora_up + (col0 + e) * lora_r + j));
+                            float v = __uint_as_float(r[e]);
+                            v = __fmaf_rn(t0.x, bf16_bits_to_float(u.x & 0xffffu), v);
+                            v = __fmaf_rn(t0.y, bf16_bits_to_float(u.x >> 16), v);
+                            v = __fmaf_rn(t0.z, bf16_bits_to_float(u.y & 0xffffu), v);
+                            v = __fmaf_rn(t0.w, bf16_bits_to_float(u.y >> 16), v);
+                            v = __fmaf_rn(t1.x, bf16_bits_to_float(u.z & 0xffffu), v);
+                            v = __fmaf_rn(t1.y, bf16_bits_to_float(u.z >> 16), v);
+                            v = __fmaf_rn(t1.z, bf16_bits_to_float(u.w & 0xffffu), v);
+                            v = __fmaf_rn(t1.w, bf16_bits_to_float(u.w >> 16), v);
+                            r[e] = __float_as_uint(v);
+                        }
+                    }
+                } else {
+                    for (int j = 0; j < lora_r; ++j) {
+                        const float tv = __ldg(tr + j);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (col0 + e < n)
+                                r[e] = __float_as_uint(__fmaf_rn(tv, __bfloat162float(lora_up[(col0 + e) * lora_r + j]),
+                                                                 __uint_as_float(r[e])));
+                    }
+                }
+            }
             if (kBf16Out) {
                 __nv_bfloat16* yrow = reinterpret_cast<__nv_bfloat16*>(Y) + tok * n;
                 if (vec && col0 + 32 <= n) {
@@ -624,15 +659,20 @@ k_nf4_gemm_dx(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
 
 cudaError_t launch_gemm(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                         const float* absmax_scale, const float* absmax_offset, int64_t n, int64_t k, void* Y,
-                        bool y_bf16, int32_t* dev_status, const DeviceInfo& dev, cudaStream_t stream) {
-    static bool attr_set[64][2] = {};
+                        bool y_bf16, int32_t* dev_status, const LoraArgs& lora, const DeviceInfo& dev,
+                        cudaStream_t stream) {
+    static bool attr_set[64][4] = {};
     if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
-    const void* fn = y_bf16 ? reinterpret_cast<const void*>(&gemm::k_nf4_gemm<true>)
-                            : reinterpret_cast<const void*>(&gemm::k_nf4_gemm<false>);
-    if (!attr_set[dev.device][y_bf16]) {
+    const bool lo = lora.t != nullptr;
+    const void* fn = y_bf16 ? (lo ? reinterpret_cast<const void*>(&gemm::k_nf4_gemm<true, true>)
+                                  : reinterpret_cast<const void*>(&gemm::k_nf4_gemm<true, false>))
+                            : (lo ? reinterpret_cast<const void*>(&gemm::k_nf4_gemm<false, true>)
+                                  : reinterpret_cast<const void*>(&gemm::k_nf4_gemm<false, false>));
+    const int vi = (y_bf16 ? 1 : 0) + (lo ? 2 : 0);
+    if (!attr_set[dev.device][vi]) {
         const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::kSmemBytes);
         if (e != cudaSuccess) return e;
-        attr_set[dev.device][y_bf16] = true;
+        attr_set[dev.device][vi] = true;
     }
     CUtensorMap tm_x, tm_w;
     cudaError_t e = tmap_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, static_cast<uint64_t>(k),
@@ -644,12 +684,15 @@ cudaError_t launch_gemm(const void* X, int64_t m, const uint8_t* wq, const int8_
     if (e != cudaSuccess) return e;
     const dim3 grid(static_cast<unsigned>((n + gemm::kBN - 1) / gemm::kBN),
                     static_cast<unsigned>((m + gemm::kBM - 1) / gemm::kBM));
-    if (y_bf16)
-        gemm::k_nf4_gemm<true><<<grid, gemm::kThreads, gemm::kSmemBytes, stream>>>(
-            tm_x, tm_w, absmax_q, absmax_scale, absmax_offset, m, n, k, Y, dev_status);
-    else
-        gemm::k_nf4_gemm<false><<<grid, gemm::kThreads, gemm::kSmemBytes, stream>>>(
-            tm_x, tm_w, absmax_q, absmax_scale, absmax_offset, m, n, k, Y, dev_status);
+#define NF4_GEMM_LAUNCH(B, L)                                                                               \
+    gemm::k_nf4_gemm<B, L><<<grid, gemm::kThreads, gemm::kSmemBytes, stream>>>(                              \
+        tm_x, tm_w, absmax_q, absmax_scale, absmax_offset, m, n, k, Y, dev_status, lora.t, lora.up, lora.r)
+    if (y_bf16) {
+        if (lo) NF4_GEMM_LAUNCH(true, true); else NF4_GEMM_LAUNCH(true, false);
+    } else {
+        if (lo) NF4_GEMM_LAUNCH(false, true); else NF4_GEMM_LAUNCH(false, false);
+    }
+#undef NF4_GEMM_LAUNCH
     return cudaGetLastError();
 }
 

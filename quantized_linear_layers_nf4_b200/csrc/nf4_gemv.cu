@@ -69,6 +69,32 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// v + sum_j t[tok * r + j] * up[row * r + j], in j order (the low-rank term of
+// a LoRA layer, added to the fp32 result before it is stored).
+__device__ __forceinline__ float lora_term(float v, const float* __restrict__ lt, const __nv_bfloat16* __restrict__ up,
+                                           int r, int tok, int64_t row) {
+    const float* tr = lt + static_cast<int64_t>(tok) * r;
+    const __nv_bfloat16* ur = up + row * r;
+    int j = 0;
+    if ((r & 7) == 0) {  // rows of up and t are 16-byte aligned: 8 ranks per load pair
+        for (; j < r; j += 8) {
+            const uint4 u = __ldg(reinterpret_cast<const uint4*>(ur + j));
+            const float4 t0 = __ldg(reinterpret_cast<const float4*>(tr + j));
+            const float4 t1 = __ldg(reinterpret_cast<const float4*>(tr + j + 4));
+            v = __fmaf_rn(t0.x, bf16_bits_to_float(u.x & 0xffffu), v);
+            v = __fmaf_rn(t0.y, bf16_bits_to_float(u.x >> 16), v);
+            v = __fmaf_rn(t0.z, bf16_bits_to_float(u.y & 0xffffu), v);
+            v = __fmaf_rn(t0.w, bf16_bits_to_float(u.y >> 16), v);
+            v = __fmaf_rn(t1.x, bf16_bits_to_float(u.z & 0xffffu), v);
+            v = __fmaf_rn(t1.y, bf16_bits_to_float(u.z >> 16), v);
+            v = __fmaf_rn(t1.z, bf16_bits_to_float(u.w & 0xffffu), v);
+            v = __fmaf_rn(t1.w, bf16_bits_to_float(u.w >> 16), v);
+        }
+    }
+    for (; j < r; ++j) v = __fmaf_rn(__ldg(tr + j), __bfloat162float(ur[j]), v);
+    return v;
+}
+
 // Byte `b` (0..3) of `word` in the low 8 bits, zeros above (one byte permute).
 __device__ __forceinline__ uint32_t byte_of(uint32_t word, uint32_t b) {
     uint32_t d;
@@ -187,13 +213,14 @@ __device__ __forceinline__ void pin(AbsmaxIn& a) {
 
 constexpr int kPrefetch = 3;  // stages of absmax inputs in flight per producer lane
 
-template <bool kBf16Out, bool kM16>
+template <bool kBf16Out, bool kM16, bool kLora>
 __global__ void __launch_bounds__(kThreads, 2)
 k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
            const int8_t* __restrict__ absmax_q, const float* __restrict__ absmax_scale,
            const float* __restrict__ mu_ptr, int m, int64_t n, int64_t k, int cluster, int weights_early,
            void* __restrict__ Y, int32_t* __restrict__ dev_status, uint32_t* __restrict__ ws_cnt,
-           float4* __restrict__ ws_part) {
+           float4* __restrict__ ws_part, const float* __restrict__ lora_t, const __nv_bfloat16* __restrict__ lora_up,
+           int lora_r) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* ring = smem;
@@ -442,11 +469,12 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
             }
             const int tok = e / (kRows / 4);
             const int r = 4 * (e % (kRows / 4));
-            const float o[4] = {sum.x, sum.y, sum.z, sum.w};
+            float o[4] = {sum.x, sum.y, sum.z, sum.w};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const int64_t grow = row0 + r + c;
                 if (grow >= n) break;
+                if (kLora) o[c] = lora_term(o[c], lora_t, lora_up, lora_r, tok, grow);
                 if (kBf16Out)
                     reinterpret_cast<__nv_bfloat16*>(Y)[static_cast<int64_t>(tok) * n + grow] = __float2bfloat16_rn(o[c]);
                 else
@@ -479,6 +507,7 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
                 if (q < cluster) sum = sum + v[q];
             const int64_t grow = row0 + r;
             if (grow < n) {
+                if (kLora) sum = lora_term(sum, lora_t, lora_up, lora_r, tok, grow);
                 if (kBf16Out)
                     reinterpret_cast<__nv_bfloat16*>(Y)[static_cast<int64_t>(tok) * n + grow] = __float2bfloat16_rn(sum);
                 else
@@ -498,11 +527,12 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
 #pragma unroll
         for (int q = 1; q < 8; ++q)
             if (q < cluster) sum = make_float4(sum.x + v[q].x, sum.y + v[q].y, sum.z + v[q].z, sum.w + v[q].w);
-        const float o[4] = {sum.x, sum.y, sum.z, sum.w};
+        float o[4] = {sum.x, sum.y, sum.z, sum.w};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             const int64_t grow = row0 + r + c;
             if (grow >= n) break;
+            if (kLora) o[c] = lora_term(o[c], lora_t, lora_up, lora_r, tok, grow);
             if (kBf16Out)
                 reinterpret_cast<__nv_bfloat16*>(Y)[static_cast<int64_t>(tok) * n + grow] = __float2bfloat16_rn(o[c]);
             else
@@ -562,14 +592,14 @@ size_t linear_workspace_bytes(int64_t m, int64_t n, int64_t k, const DeviceInfo&
     return kWsCounterBytes + tiles * cluster * 16 * gemv::kRows * sizeof(float);
 }
 
-template <bool kBf16Out, bool kM16>
+template <bool kBf16Out, bool kM16, bool kLora>
 static cudaError_t launch_gemv(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const int8_t* absmax_q,
                                const float* absmax_scale, const float* absmax_offset, int mt, int64_t n,
                                int64_t k, int cluster, bool weights_early, void* Yt, int32_t* dev_status,
-                               void* ws, int device, cudaStream_t stream) {
+                               void* ws, const LoraArgs& lora, int device, cudaStream_t stream) {
     static bool attr_set[64] = {};
     if (!attr_set[device]) {
-        const cudaError_t e = cudaFuncSetAttribute(gemv::k_nf4_gemv<kBf16Out, kM16>,
+        const cudaError_t e = cudaFuncSetAttribute(gemv::k_nf4_gemv<kBf16Out, kM16, kLora>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, gemv::kSmemBytes);
         if (e != cudaSuccess) return e;
         attr_set[device] = true;
@@ -599,18 +629,39 @@ static cudaError_t launch_gemv(const CUtensorMap& tm_w, const CUtensorMap& tm_x,
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    return cudaLaunchKernelEx(&cfg, gemv::k_nf4_gemv<kBf16Out, kM16>, tm_w, tm_x, absmax_q, absmax_scale,
+    return cudaLaunchKernelEx(&cfg, gemv::k_nf4_gemv<kBf16Out, kM16, kLora>, tm_w, tm_x, absmax_q, absmax_scale,
                               absmax_offset, mt, n, k, cluster, weights_early ? 1 : 0, Yt, dev_status, ws_cnt,
-                              ws_part);
+                              ws_part, lora.t, lora.up, lora.r);
+}
+
+// One of the eight instantiations: output type, more than 8 tokens, LoRA term.
+static cudaError_t dispatch_gemv(bool bf16, bool m16, bool lora_on, const CUtensorMap& tm_w, const CUtensorMap& tm_x,
+                                 const int8_t* absmax_q, const float* absmax_scale, const float* absmax_offset,
+                                 int mt, int64_t n, int64_t k, int cluster, bool early, void* Yt, int32_t* ds,
+                                 void* ws, const LoraArgs& lora, int device, cudaStream_t stream) {
+#define NF4_GEMV_CASE(B, M, L)                                                                                   \
+    if (bf16 == B && m16 == M && lora_on == L)                                                                  \
+        return launch_gemv<B, M, L>(tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt, n, k, cluster, early, \
+                                    Yt, ds, ws, lora, device, stream);
+    NF4_GEMV_CASE(true, true, false)
+    NF4_GEMV_CASE(true, false, false)
+    NF4_GEMV_CASE(false, true, false)
+    NF4_GEMV_CASE(false, false, false)
+    NF4_GEMV_CASE(true, true, true)
+    NF4_GEMV_CASE(true, false, true)
+    NF4_GEMV_CASE(false, true, true)
+    NF4_GEMV_CASE(false, false, true)
+#undef NF4_GEMV_CASE
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                           const float* absmax_scale, const float* absmax_offset, int64_t n,
                           int64_t k, void* Y, bool y_bf16, int32_t* dev_status, bool weights_early,
-                          void* ws, const DeviceInfo& dev, cudaStream_t stream) {
+                          void* ws, const LoraArgs& lora, const DeviceInfo& dev, cudaStream_t stream) {
     if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
     if (m > kGemvMaxTokens)
-        return launch_gemm(X, m, wq, absmax_q, absmax_scale, absmax_offset, n, k, Y, y_bf16, dev_status, dev,
+        return launch_gemm(X, m, wq, absmax_q, absmax_scale, absmax_offset, n, k, Y, y_bf16, dev_status, lora, dev,
                            stream);
     CUtensorMap tm_w;
     cudaError_t e = tmap_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, static_cast<uint64_t>(k / 2),
@@ -629,16 +680,8 @@ cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int
                     static_cast<uint64_t>(mt), static_cast<uint64_t>(k * 2), 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
         if (e != cudaSuccess) return e;
         void* Yt = static_cast<char*>(Y) + static_cast<size_t>(t0) * n * ybytes;
-        if (y_bf16)
-            e = (mt > 8) ? launch_gemv<true, true>(tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt, n, k,
-                                                   cluster, weights_early, Yt, dev_status, ws, dev.device, stream)
-                         : launch_gemv<true, false>(tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt, n, k,
-                                                    cluster, weights_early, Yt, dev_status, ws, dev.device, stream);
-        else
-            e = (mt > 8) ? launch_gemv<false, true>(tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt, n, k,
-                                                    cluster, weights_early, Yt, dev_status, ws, dev.device, stream)
-                         : launch_gemv<false, false>(tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt, n,
-                                                     k, cluster, weights_early, Yt, dev_status, ws, dev.device, stream);
+        e = dispatch_gemv(y_bf16, mt > 8, lora.t != nullptr, tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt,
+                          n, k, cluster, weights_early, Yt, dev_status, ws, lora, dev.device, stream);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 namespace nf4 {
@@ -14,6 +15,14 @@ struct DeviceInfo {
     int major = 0;
     int minor = 0;
     size_t smem_optin = 0;
+};
+
+// Low-rank (LoRA) term added in a linear's epilogue: Y[t, o] += sum_j t[t * r + j] * up[o * r + j]
+// (t = scale * X down^T, fp32 [m, r]; up bf16 [n, r]).  t == nullptr: none.
+struct LoraArgs {
+    const float* t = nullptr;
+    const __nv_bfloat16* up = nullptr;
+    int r = 0;
 };
 
 // Properties of the current device (cached per device).
@@ -40,7 +49,11 @@ size_t linear_workspace_bytes(int64_t m, int64_t n, int64_t k, const DeviceInfo&
 cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                           const float* absmax_scale, const float* absmax_offset, int64_t n,
                           int64_t k, void* Y, bool y_bf16, int32_t* dev_status, bool weights_early,
-                          void* ws, const DeviceInfo& dev, cudaStream_t stream);
+                          void* ws, const LoraArgs& lora, const DeviceInfo& dev, cudaStream_t stream);
+
+// t[m, r] = scale * X[m, k] down[r, k]^T in fp32 (one block per token, fixed order).
+cudaError_t launch_lora_down(const void* X, int64_t m, int64_t k, const void* down, int r, float scale, float* t,
+                             cudaStream_t stream);
 
 cudaError_t launch_gemm_dx(const void* dY, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                            const float* absmax_scale, const float* absmax_offset, int64_t n, int64_t k, void* dX,
@@ -48,7 +61,8 @@ cudaError_t launch_gemm_dx(const void* dY, int64_t m, const uint8_t* wq, const i
 
 cudaError_t launch_gemm(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                         const float* absmax_scale, const float* absmax_offset, int64_t n, int64_t k, void* Y,
-                        bool y_bf16, int32_t* dev_status, const DeviceInfo& dev, cudaStream_t stream);
+                        bool y_bf16, int32_t* dev_status, const LoraArgs& lora, const DeviceInfo& dev,
+                        cudaStream_t stream);
 
 // Token counts up to this run the decode GEMV; larger ones the tcgen05 GEMM.
 constexpr int64_t kGemvMaxTokens = 16;

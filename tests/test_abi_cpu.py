@@ -156,6 +156,17 @@ def test_linear_dx_validation(L):
     assert dx(FAKE, 4, ctypes.byref(_weight(magic=7)), FAKE, 1, None, None) == -5
 
 
+def test_linear_lora_validation(L):
+    lo = L.nf4_linear_lora
+    w = ctypes.byref(_weight())
+    assert lo(FAKE, 4, w, None, FAKE, 16, 2.0, FAKE, 1, None, 0, FAKE, 1 << 20, None) == -1   # no down
+    assert lo(FAKE, 4, w, FAKE, FAKE, 16, 2.0, FAKE, 1, None, 0, None, 0, None) == -1        # no workspace
+    assert lo(FAKE, 4, w, FAKE, FAKE, 0, 2.0, FAKE, 1, None, 0, FAKE, 1 << 20, None) == -2   # rank 0
+    assert lo(FAKE, 4, w, FAKE, FAKE, 300, 2.0, FAKE, 1, None, 0, FAKE, 1 << 20, None) == -2
+    assert lo(FAKE, 4, w, FAKE, ODD, 16, 2.0, FAKE, 1, None, 0, FAKE, 1 << 20, None) == -3
+    assert L.nf4_linear_lora_workspace_bytes(4, 4096, 4096, 0) == 0
+
+
 def test_valid_call_without_a_gpu_reports_instead_of_crashing(L):
     """On a host without a usable B200 a fully valid call must come back with a
     status (no device / unsupported device), never crash or launch."""

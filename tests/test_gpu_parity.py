@@ -312,6 +312,38 @@ def test_linear_dx_errors(nf4):
         nf4.nf4_linear_dx(dY, weight, torch.float32)
 
 
+@pytest.mark.parametrize("m,n,k,r,scale", [(16, 4096, 4096, 16, 2.0), (3, 11000, 2304, 64, 0.5),
+                                           (16, 64, 128, 1, 2.0), (7, 1000, 1024, 8, 1.0),
+                                           (300, 520, 640, 16, 2.0), (1024, 1024, 1024, 64, 0.25)])
+def test_linear_lora(nf4, m, n, k, r, scale):
+    """The QLoRA layer Y = X What^T + s (X down^T) up^T: decode path (k split 8, 3
+    and 1) and prefill path, against the oracle; the bf16 output is the rounded
+    fp32 output."""
+    W = synth.weight_normal(n, k, seed=1800 + n + r, dtype=torch.bfloat16, device="cuda")
+    X = synth.activations(m, k, seed=1810 + m, device="cuda")
+    down = (synth.activations(r, k, seed=1820 + r, device="cuda").float() * 0.02).to(torch.bfloat16)
+    up = (synth.activations(n, r, seed=1830 + r, device="cuda").float() * 0.02).to(torch.bfloat16)
+    weight, orc = _check_quant(nf4, W, full_dequant=False, rows=[0, n - 1])
+    owq, oq, os_, omu = orc
+    ws = nf4.lora_workspace(m, [(n, k)], r)
+    T = np.arange(m) if m <= 64 else _sample_rows(m, 24, m)
+    R = np.arange(n) if n <= 4096 else _sample_rows(n, 256, n)
+    Y32 = nf4.nf4_linear_lora(X, weight, down, up, scale, ws, dtype=torch.float32)
+    Y16 = nf4.nf4_linear_lora(X, weight, down, up, scale, ws, dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    wrows = np.stack([O.f32_to_bf16(O.dequantize_range(owq, oq, os_, omu, int(rr) * k, k)) for rr in R])
+    ref = O.linear_lora_bf16(np.ascontiguousarray(_bits(X).reshape(m, k)[T]), wrows, _bits(down).reshape(r, k),
+                             np.ascontiguousarray(_bits(up).reshape(n, r)[R]), scale)
+    y32 = Y32.cpu().numpy()[np.ix_(T, R)]
+    e32 = _rel_fro(y32, ref)
+    assert e32 <= LINEAR_TOL, "LoRA layer fp32 rel-Frobenius %.3g" % e32
+    y16 = Y16.float().cpu().numpy()[np.ix_(T, R)]
+    assert np.array_equal(y16, torch.from_numpy(np.ascontiguousarray(y32)).to(torch.bfloat16).float().numpy())
+    # a zero scale leaves the base linear
+    Y0 = nf4.nf4_linear_lora(X, weight, down, up, 0.0, ws, dtype=torch.float32)
+    assert torch.equal(Y0, nf4.nf4_linear(X, weight, torch.float32))
+
+
 def test_deterministic_and_stream_aware(nf4):
     W = synth.weight_normal(512, 1024, seed=9, dtype=torch.bfloat16, device="cuda")
     X = synth.activations(16, 1024, seed=10, device="cuda")
