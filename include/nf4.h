@@ -254,7 +254,8 @@ nf4_status_t nf4_linear_dx(const void* dY, int64_t m, const nf4_weight_t* w, voi
 /*
  * nf4_linear_lora_workspace_bytes -- bytes of the workspace nf4_linear_lora
  * needs for m tokens, an [n, k] weight and rank r: the low-rank projection
- * t [m, r] (fp32), then the split-k area of nf4_linear_ws.  0 for invalid sizes.
+ * t [m, r] in fp32 and as two bf16 halves, then the split-k area of
+ * nf4_linear_ws.  0 for invalid sizes.
  */
 size_t nf4_linear_lora_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t r);
 
@@ -263,9 +264,13 @@ size_t nf4_linear_lora_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t 
  * low-rank update, Y = X * What^T + scale * (X * down^T) * up^T ([P4] "2-2. LoRA
  * （低秩適應）": W acts as W + dW with dW = A x B of rank r; section 4: base frozen
  * INT4, LoRA matrices bf16).  With W stored [n, k], dW = up * down.
- * t = scale * X down^T is computed first (fp32, fixed summation order); the
- * linear then adds sum_j t[i][j] * up[o][j] (j in order, fp32) to each fp32
- * output before rounding it to y_dtype.  Same path and flags as nf4_linear_ws.
+ * t = scale * X down^T is computed first (fp32, fixed summation order).  For
+ * m <= 16 the linear then adds sum_j t[i][j] * up[o][j] (j in order, fp32) to
+ * each fp32 output before rounding it to y_dtype.  For larger m with r % 8 == 0
+ * the term runs on the tensor cores as extra K steps, t_hi up^T + t_lo up^T
+ * with t = t_hi + t_lo split into bf16 halves (t kept to about 16 bits) and
+ * accumulated in fp32; other ranks use the fp32 epilogue.  Same path and flags
+ * as nf4_linear_ws.
  *   X          device, bf16 [m, k], 16-byte aligned
  *   w          the [n, k] quantized weight
  *   lora_down  device, bf16 [r, k] row-major (PEFT's lora_A.weight), 16-byte aligned

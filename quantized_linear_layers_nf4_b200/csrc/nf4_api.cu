@@ -143,8 +143,13 @@ nf4_status_t nf4_dequantize(const nf4_weight_t* w, void* out, nf4_dtype_t out_dt
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// LoRA workspace: t fp32 [m, r], then its bf16 halves t_hi, t_lo [m, r] (each
+// region padded to 256 bytes), then the split-k area of the decode path.
+static size_t lora_t_region(int64_t m, int32_t r, size_t elem) {
+    return (static_cast<size_t>(m) * static_cast<size_t>(r) * elem + 255) / 256 * 256;
+}
 static size_t lora_t_bytes(int64_t m, int32_t r) {
-    return (static_cast<size_t>(m) * static_cast<size_t>(r) * sizeof(float) + 255) / 256 * 256;
+    return lora_t_region(m, r, sizeof(float)) + 2 * lora_t_region(m, r, 2);
 }
 
 nf4_status_t nf4_linear_lora(const void* X, int64_t m, const nf4_weight_t* w, const void* lora_down,
@@ -167,12 +172,16 @@ nf4_status_t nf4_linear_lora(const void* X, int64_t m, const nf4_weight_t* w, co
     if (ws_bytes < tb + nf4::linear_workspace_bytes(m, w->n, w->k, dev)) return NF4_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     float* t = static_cast<float*>(workspace);
-    st = from_cuda(nf4::launch_lora_down(X, m, w->k, lora_down, r, scale, t, s));
+    __nv_bfloat16* t_hi = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(workspace) + lora_t_region(m, r, 4));
+    __nv_bfloat16* t_lo = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<char*>(t_hi) + lora_t_region(m, r, 2));
+    st = from_cuda(nf4::launch_lora_down(X, m, w->k, lora_down, r, scale, t, t_hi, t_lo, s));
     if (st != NF4_OK) return st;
     nf4::LoraArgs lora;
     lora.t = t;
     lora.up = static_cast<const __nv_bfloat16*>(lora_up);
     lora.r = r;
+    lora.t_hi = t_hi;
+    lora.t_lo = t_lo;
     return from_cuda(nf4::launch_linear(X, m, w->wq, w->absmax_q, w->absmax_scale, w->absmax_offset, w->n, w->k,
                                         Y, y_dtype == NF4_BF16, dev_status, (flags & NF4_LINEAR_WEIGHTS_EARLY) != 0,
                                         static_cast<char*>(workspace) + tb, lora, dev, s));

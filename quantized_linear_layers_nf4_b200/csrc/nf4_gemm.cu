@@ -54,7 +54,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kOffB = kStagesA * kABytes;
 constexpr int kOffP = kOffB + kStagesB * kBBytes;
 constexpr int kOffBar = kOffP + kStagesP * kPBytes;
-constexpr int kNumBars = 2 * kStagesA + 2 * kStagesB + 2 * kStagesP + 2;
+constexpr int kNumBars = 2 * kStagesA + 2 * kStagesB + 2 * kStagesP + 4;  // + low-rank tiles, MMA drain
 constexpr int kSmemBytes = 1024 + kOffBar + kNumBars * 8 + 16;
 
 // Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major,
@@ -142,7 +142,9 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
            const int8_t* __restrict__ absmax_q, const float* __restrict__ absmax_scale,
            const float* __restrict__ mu_ptr, int64_t m, int64_t n, int64_t k, void* __restrict__ Y,
            int32_t* __restrict__ dev_status, const float* __restrict__ lora_t,
-           const __nv_bfloat16* __restrict__ lora_up, int lora_r) {
+           const __nv_bfloat16* __restrict__ lora_up, int lora_r, int lora_tc,
+           const __grid_constant__ CUtensorMap tm_thi, const __grid_constant__ CUtensorMap tm_tlo,
+           const __grid_constant__ CUtensorMap tm_up) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -154,6 +156,8 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     uint64_t* empty_p = full_p + kStagesP;
     uint64_t* acc_ready = empty_p + kStagesP;
     uint64_t* drained = acc_ready + 1;
+    uint64_t* lora_full = drained + 1;   // low-rank tiles landed
+    uint64_t* mma_done = lora_full + 1;   // every MMA issued so far has completed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
 
     const int warp = threadIdx.x >> 5;
@@ -178,6 +182,8 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         }
         mbar_init(acc_ready, 1);
         mbar_init(drained, 1);
+        mbar_init(lora_full, 1);
+        mbar_init(mma_done, 1);
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
@@ -247,6 +253,37 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                                     smem_desc_sw128(b_addr + 32 * j), kIdesc, (kt > 0 || j > 0) ? 1u : 0u);
                 tc_commit(&empty_a[sa]);
                 tc_commit(&empty_b[sb]);
+            }
+            if (kLora && lora_tc && !timed_out) {
+                // Low-rank term on the tensor cores: Y += t_hi up^T + t_lo up^T, with
+                // t = t_hi + t_lo (two bf16 halves) and up as the B operand, in K
+                // tiles of 64 ranks (zero-filled past r) loaded into the stage
+                // buffers once every main-loop MMA has read them.
+                const int nlt = (lora_r + 63) / 64;
+                for (int lt = 0; lt < nlt && !timed_out; ++lt) {
+                    tc_commit(mma_done);
+                    if (!mbar_wait(mma_done, lt & 1)) {
+                        timed_out = true;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(lora_full, 3 * kABytes);
+                    tma_load_2d(smem, &tm_thi, lt * 64, static_cast<int32_t>(m0), lora_full);
+                    tma_load_2d(smem + kABytes, &tm_tlo, lt * 64, static_cast<int32_t>(m0), lora_full);
+                    tma_load_2d(smem + 2 * kABytes, &tm_up, lt * 64, static_cast<int32_t>(n0), lora_full);
+                    if (!mbar_wait(lora_full, lt & 1)) {
+                        timed_out = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int ks = ((lora_r - lt * 64 < 64 ? lora_r - lt * 64 : 64) + 15) / 16;
+                    for (int h = 0; h < 2; ++h)
+                        for (int j = 0; j < ks; ++j) {
+                            const uint64_t bd = smem_desc_sw128(sbase + 2 * kABytes + 32 * j);
+                            tc_mma_bf16(tmem + h * 256, smem_desc_sw128(sbase + h * (128 * 128) + 32 * j), bd, kIdesc, 1u);
+                            tc_mma_bf16(tmem + h * 256, smem_desc_sw128(sbase + kABytes + h * (128 * 128) + 32 * j), bd,
+                                        kIdesc, 1u);
+                        }
+                }
             }
             tc_commit(timed_out ? drained : acc_ready);
             if (timed_out) mbar_wait(drained, 0);  // issued MMAs finish before TMEM is freed
@@ -338,8 +375,9 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             if (ok) tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * 256 + cc * 32, r);
             const int64_t col0 = n0 + cc * 32;
             if (!ok || tok >= m || col0 >= n) continue;
-            if (kLora) {
-                // low-rank term: + sum_j t[tok, j] * up[col, j], j ascending for every column
+            if (kLora && !lora_tc) {
+                // low-rank term on the CUDA cores (rank not a multiple of 8):
+                // + sum_j t[tok, j] * up[col, j], j ascending for every column
                 const float* tr = lora_t + tok * lora_r;
                 if ((lora_r & 7) == 0) {  // 16-byte aligned rows: 8 ranks per load
                     for (int j = 0; j < lora_r; j += 8) {
@@ -684,9 +722,26 @@ cudaError_t launch_gemm(const void* X, int64_t m, const uint8_t* wq, const int8_
     if (e != cudaSuccess) return e;
     const dim3 grid(static_cast<unsigned>((n + gemm::kBN - 1) / gemm::kBN),
                     static_cast<unsigned>((m + gemm::kBM - 1) / gemm::kBM));
+    // the low-rank term on the tensor cores needs 16-byte rows of t_hi / t_lo / up (r % 8 == 0)
+    int lora_tc = 0;
+    CUtensorMap tm_thi = tm_x, tm_tlo = tm_x, tm_up = tm_x;  // unused unless lora_tc
+    if (lo && lora.t_hi && lora.t_lo && lora.r % 8 == 0) {
+        const uint64_t rr = static_cast<uint64_t>(lora.r);
+        e = tmap_2d(&tm_thi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora.t_hi, rr, static_cast<uint64_t>(m), rr * 2,
+                    64, gemm::kBM, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (e != cudaSuccess) return e;
+        e = tmap_2d(&tm_tlo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora.t_lo, rr, static_cast<uint64_t>(m), rr * 2,
+                    64, gemm::kBM, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (e != cudaSuccess) return e;
+        e = tmap_2d(&tm_up, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora.up, rr, static_cast<uint64_t>(n), rr * 2,
+                    64, gemm::kBN, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (e != cudaSuccess) return e;
+        lora_tc = 1;
+    }
 #define NF4_GEMM_LAUNCH(B, L)                                                                               \
     gemm::k_nf4_gemm<B, L><<<grid, gemm::kThreads, gemm::kSmemBytes, stream>>>(                              \
-        tm_x, tm_w, absmax_q, absmax_scale, absmax_offset, m, n, k, Y, dev_status, lora.t, lora.up, lora.r)
+        tm_x, tm_w, absmax_q, absmax_scale, absmax_offset, m, n, k, Y, dev_status, lora.t, lora.up, lora.r,  \
+        lora_tc, tm_thi, tm_tlo, tm_up)
     if (y_bf16) {
         if (lo) NF4_GEMM_LAUNCH(true, true); else NF4_GEMM_LAUNCH(true, false);
     } else {

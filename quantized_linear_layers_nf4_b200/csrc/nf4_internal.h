@@ -19,10 +19,14 @@ struct DeviceInfo {
 
 // Low-rank (LoRA) term added in a linear's epilogue: Y[t, o] += sum_j t[t * r + j] * up[o * r + j]
 // (t = scale * X down^T, fp32 [m, r]; up bf16 [n, r]).  t == nullptr: none.
+// t_hi / t_lo: t split into two bf16 halves (t_hi = bf16(t), t_lo = bf16(t - t_hi)),
+// [m, r] each, for the tensor-core form of the term in the large-m GEMM.
 struct LoraArgs {
     const float* t = nullptr;
     const __nv_bfloat16* up = nullptr;
     int r = 0;
+    const __nv_bfloat16* t_hi = nullptr;
+    const __nv_bfloat16* t_lo = nullptr;
 };
 
 // Properties of the current device (cached per device).
@@ -51,9 +55,10 @@ cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int
                           int64_t k, void* Y, bool y_bf16, int32_t* dev_status, bool weights_early,
                           void* ws, const LoraArgs& lora, const DeviceInfo& dev, cudaStream_t stream);
 
-// t[m, r] = scale * X[m, k] down[r, k]^T in fp32 (one block per token, fixed order).
+// t[m, r] = scale * X[m, k] down[r, k]^T in fp32 (fixed order); also its two bf16
+// halves when t_hi / t_lo are given.
 cudaError_t launch_lora_down(const void* X, int64_t m, int64_t k, const void* down, int r, float scale, float* t,
-                             cudaStream_t stream);
+                             __nv_bfloat16* t_hi, __nv_bfloat16* t_lo, cudaStream_t stream);
 
 cudaError_t launch_gemm_dx(const void* dY, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                            const float* absmax_scale, const float* absmax_offset, int64_t n, int64_t k, void* dX,

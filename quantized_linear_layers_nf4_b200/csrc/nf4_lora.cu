@@ -19,7 +19,8 @@ namespace lora {
 
 __global__ void __launch_bounds__(256) k_lora_down(const __nv_bfloat16* __restrict__ X, int64_t k,
                                                    const __nv_bfloat16* __restrict__ down, int r, float scale,
-                                                   float* __restrict__ t) {
+                                                   float* __restrict__ t, __nv_bfloat16* __restrict__ t_hi,
+                                                   __nv_bfloat16* __restrict__ t_lo) {
     // block (token, group of 8 ranks); warp w computes rank 8 * blockIdx.y + w
     const int64_t tok = blockIdx.x;
     const int j = static_cast<int>(blockIdx.y) * 8 + (threadIdx.x >> 5);
@@ -50,17 +51,25 @@ __global__ void __launch_bounds__(256) k_lora_down(const __nv_bfloat16* __restri
     float v = __fadd_rn(__fadd_rn(acc[0], acc[1]), __fadd_rn(acc[2], acc[3]));
 #pragma unroll
     for (int h = 16; h >= 1; h >>= 1) v = __fadd_rn(v, __shfl_xor_sync(kFull, v, h));
-    if (lane == 0) t[tok * r + j] = __fmul_rn(v, scale);
+    if (lane == 0) {
+        const float tv = __fmul_rn(v, scale);
+        t[tok * r + j] = tv;
+        if (t_hi) {
+            const __nv_bfloat16 h = __float2bfloat16_rn(tv);
+            t_hi[tok * r + j] = h;
+            t_lo[tok * r + j] = __float2bfloat16_rn(__fsub_rn(tv, __bfloat162float(h)));
+        }
+    }
 }
 
 }  // namespace lora
 
 cudaError_t launch_lora_down(const void* X, int64_t m, int64_t k, const void* down, int r, float scale, float* t,
-                             cudaStream_t stream) {
+                             __nv_bfloat16* t_hi, __nv_bfloat16* t_lo, cudaStream_t stream) {
     const dim3 grid(static_cast<unsigned>(m), static_cast<unsigned>((r + 7) / 8));
     lora::k_lora_down<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), k,
                                                                       static_cast<const __nv_bfloat16*>(down), r,
-                                                                      scale, t);
+                                                                      scale, t, t_hi, t_lo);
     return cudaGetLastError();
 }
 
