@@ -441,8 +441,9 @@ def run_ours(args, rank, world, local):
             ul = (synth.activations(wl.n, rl, seed=synth.seed_for(3, 10), device=dev).float() * 0.02).to(torch.bfloat16)
             wsl = nf4.lora_workspace(ml, [(wl.n, wl.k)], rl, device=dev)
             wsp = nf4.linear_workspace([(wl.n, wl.k)], m=ml, device=dev)
-            f_l = lambda: nf4.nf4_linear_lora(Xl, wl, dl, ul, 2.0, wsl, out=Yl)
-            f_p = lambda: nf4.nf4_linear(Xl, wl, torch.bfloat16, out=Yl, workspace=wsp)
+            early = ml <= 16   # the decode path runs with programmatic dependent launch
+            f_l = lambda: nf4.nf4_linear_lora(Xl, wl, dl, ul, 2.0, wsl, out=Yl, weights_early=early)
+            f_p = lambda: nf4.nf4_linear(Xl, wl, torch.bfloat16, out=Yl, workspace=wsp, weights_early=early)
             f_l(); f_p()
             t_l = _events_time(f_l, 20, stream)
             t_p = _events_time(f_p, 20, stream)
