@@ -283,6 +283,16 @@ void orc_f32_to_bf16(const float* x, int64_t n, uint16_t* out) {
  * dtype feeds the matmul ([P4] §5: weights are restored to BF16 before the
  * matrix multiply).  Every bf16 x bf16 product is exact in fp64; the sum runs
  * over k in order. */
+void orc_lora_delta(const uint16_t* up, const uint16_t* down, int64_t n, int64_t r, int64_t k, float* delta) {
+    for (int64_t o = 0; o < n; ++o)
+        for (int64_t c = 0; c < k; ++c) {
+            float acc = 0.0f;
+            for (int64_t j = 0; j < r; ++j)
+                acc = fmaf(bf16_bits_to_f32(up[o * r + j]), bf16_bits_to_f32(down[j * k + c]), acc);
+            delta[o * k + c] = acc;
+        }
+}
+
 void orc_linear_bf16(const uint16_t* x, int64_t m, const uint16_t* w, int64_t n, int64_t k,
                      double* y) {
     for (int64_t i = 0; i < m; ++i)

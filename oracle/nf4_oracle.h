@@ -84,6 +84,12 @@ void orc_f32_to_bf16(const float* x, int64_t n, uint16_t* out);
 
 /* y[m][n] = sum_k x[m][k] * w[n][k] in fp64, x and w given as bf16 bit patterns,
  * x [m,k] and w [n,k] row-major, y [m,n] row-major. */
+/* LoRA merge delta ("LLM 相關知識", section "8. LoRA 的合併（Merge）": W_new = W + A x B
+ * in BF16 after dequantizing): delta[o][c] = sum_j up[o][j] * down[j][c] as an fp32
+ * fused multiply-add chain in j order starting from +0 (fmaf, one rounding per
+ * step).  up bf16 [n, r], down bf16 [r, k] as bit patterns -> delta fp32 [n, k]. */
+void orc_lora_delta(const uint16_t* up, const uint16_t* down, int64_t n, int64_t r, int64_t k, float* delta);
+
 void orc_linear_bf16(const uint16_t* x, int64_t m, const uint16_t* w, int64_t n, int64_t k,
                      double* y);
 

@@ -11,7 +11,7 @@ from .build_oracle import build
 
 __all__ = [
     "norm_ppf", "codebook", "quantize", "dq_sum", "dq_mean", "double_quant", "absmax_hat",
-    "dequantize", "dequantize_range", "f32_to_bf16", "bf16_to_f32", "linear_bf16", "linear_dx_bf16", "linear_lora_bf16", "unpack",
+    "dequantize", "dequantize_range", "f32_to_bf16", "bf16_to_f32", "linear_bf16", "linear_dx_bf16", "linear_lora_bf16", "lora_delta", "merge_lora", "unpack",
     "use_library",
 ]
 
@@ -50,6 +50,8 @@ def _bind(L):
     L.orc_f32_to_bf16.restype = None
     L.orc_linear_bf16.argtypes = [p, i64, p, i64, i64, p]
     L.orc_linear_bf16.restype = None
+    L.orc_lora_delta.argtypes = [p, p, i64, i64, i64, p]
+    L.orc_lora_delta.restype = None
     return L
 
 
@@ -200,6 +202,38 @@ def linear_lora_bf16(x_bf16: np.ndarray, w_bf16: np.ndarray, down_bf16: np.ndarr
     up = bf16_to_f32(up_bf16).astype(np.float64)
     t = x @ down.T                       # [m, r]: the low-rank projection of X
     return base + float(scale) * (t @ up.T)
+
+
+def lora_delta(up_bf16: np.ndarray, down_bf16: np.ndarray) -> np.ndarray:
+    """delta = up * down as an fp32 fused-multiply-add chain in rank order (see
+    orc_lora_delta).  up [n, r], down [r, k] bf16 bit patterns -> fp32 [n, k]."""
+    up = np.ascontiguousarray(up_bf16, dtype=np.uint16)
+    down = np.ascontiguousarray(down_bf16, dtype=np.uint16)
+    n, r = up.shape
+    r2, k = down.shape
+    assert r == r2
+    out = np.zeros((n, k), dtype=np.float32)
+    lib().orc_lora_delta(_ptr(up), _ptr(down), n, r, k, _ptr(out))
+    return out
+
+
+def merge_lora(wq, absmax_q, absmax_scale, mu, n: int, k: int, down_bf16, up_bf16, scale: float):
+    """Merge a trained LoRA update into the quantized base and requantize it.
+
+    Page "LLM 相關知識" (technicalnotes), section "8. LoRA 的合併（Merge）": INT4
+    weights are dequantized to BF16, W_new = W + A x B is formed in BF16, and W_new
+    is quantized again to INT4 for deployment.  Reading: What_bf16 is the bf16
+    dequantized weight; delta = up * down (fp32, rank order, lora_delta);
+    W_new = bf16_round(fp32(What_bf16 + fp32(scale * delta))); the new codes and
+    fp32 absmax are the blockwise NF4 quantization of the bf16 W_new.
+    Returns (w_new bf16 bits [n, k], wq_new uint8, absmax_new fp32)."""
+    what = f32_to_bf16(dequantize_range(wq, absmax_q, absmax_scale, mu, 0, n * k)).reshape(n, k)
+    d = lora_delta(up_bf16, down_bf16)
+    sd = (np.float32(scale) * d).astype(np.float32)                 # fp32 multiply
+    s = (bf16_to_f32(what) + sd).astype(np.float32)                  # fp32 add
+    w_new = f32_to_bf16(s)
+    wq_new, absmax_new = quantize(w_new.reshape(-1))
+    return w_new, wq_new, absmax_new
 
 
 def unpack(wq: np.ndarray) -> np.ndarray:

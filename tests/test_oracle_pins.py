@@ -446,3 +446,60 @@ def test_linear_lora_exact_small_integers():
             base = sum(int(Xi[i, c]) * int(Wi[o, c]) for c in range(k))
             low = sum(sum(int(Xi[i, c]) * int(Di[j, c]) for c in range(k)) * int(Ui[o, j]) for j in range(r))
             assert y[i, o] == base + 3 * low
+
+
+# ---------------------------------------------------------------------------
+# Merge + requantize (technicalnotes page, section "8. LoRA 的合併（Merge）").
+# Pinned by integer brute force on the delta, by the zero-scale case (W_new is the
+# bf16 dequant), and by the bound that links the merged weight to the LoRA layer.
+# ---------------------------------------------------------------------------
+
+def test_lora_delta_exact_small_integers():
+    rng = np.random.default_rng(41)
+    n, r, k = 3, 4, 5
+    Ui, Di = rng.integers(-6, 7, size=(n, r)), rng.integers(-6, 7, size=(r, k))
+    d = O.lora_delta(_bf16_bits(Ui), _bf16_bits(Di))
+    for o in range(n):
+        for c in range(k):
+            assert d[o, c] == sum(int(Ui[o, j]) * int(Di[j, c]) for j in range(r))
+
+
+def _quantized(rng, n, k):
+    W = rng.standard_normal((n, k)).astype(np.float32) * 0.02
+    wq, am = O.quantize(W)
+    q, s, mu = O.double_quant(am)
+    return wq, q, s, mu
+
+
+def test_merge_zero_scale_is_the_bf16_dequant():
+    rng = np.random.default_rng(42)
+    n, k, r = 8, 128, 4
+    wq, q, s, mu = _quantized(rng, n, k)
+    D = _bf16_bits(rng.standard_normal((r, k)))
+    U = _bf16_bits(rng.standard_normal((n, r)))
+    w_new, wq2, am2 = O.merge_lora(wq, q, s, mu, n, k, D, U, 0.0)
+    what = O.f32_to_bf16(O.dequantize(wq, q, s, mu)).reshape(n, k)
+    assert np.array_equal(w_new, what)
+    # and the requantized codes are the quantization of that bf16 weight
+    wq3, am3 = O.quantize(what.reshape(-1))
+    assert np.array_equal(wq2, wq3) and np.array_equal(am2.view(np.uint32), am3.view(np.uint32))
+
+
+def test_merged_weight_matches_the_lora_layer_within_bf16_rounding():
+    """X W_new^T differs from the fp64 LoRA layer only by W_new's rounding: each
+    element of W_new is within 2^-8 relative of What + s up down (one fp32 add,
+    one bf16 round), so |difference| <= 2^-8 * sum |x| |W_new| + fp32 slack."""
+    rng = np.random.default_rng(43)
+    n, k, r, m, sc = 16, 128, 8, 3, 2.0
+    wq, q, s, mu = _quantized(rng, n, k)
+    D = _bf16_bits(rng.standard_normal((r, k)) * 0.02)
+    U = _bf16_bits(rng.standard_normal((n, r)) * 0.02)
+    X = _bf16_bits(rng.standard_normal((m, k)))
+    w_new, _, _ = O.merge_lora(wq, q, s, mu, n, k, D, U, sc)
+    what = O.f32_to_bf16(O.dequantize(wq, q, s, mu)).reshape(n, k)
+    y_merged = O.linear_bf16(X, w_new)
+    y_layer = O.linear_lora_bf16(X, what, D, U, sc)
+    xa = np.abs(O.bf16_to_f32(X).astype(np.float64))
+    wa = np.abs(O.bf16_to_f32(w_new).astype(np.float64))
+    bound = 2.0 ** -8 * (xa @ wa.T) + 1e-6
+    assert np.all(np.abs(y_merged - y_layer) <= bound)
