@@ -65,6 +65,13 @@ def quant_bytes(n: int, k: int) -> int:
     return 2 * n * k + n * k // 2 + nb + 4 * ((nb + 255) // 256) + 4
 
 
+def merge_bytes(n: int, k: int, r: int) -> int:
+    """Merge + requantize: codes and double-quantized absmax in, codes and fp32
+    absmax out, the two bf16 LoRA matrices read once."""
+    p = n * k
+    return p // 2 + p // 64 + 4 * ((p // 64 + 255) // 256) + 4 + p // 2 + 4 * (p // 64) + 2 * r * (n + k)
+
+
 def dequant_bytes(n: int, k: int) -> int:
     nb = n * k // 64
     return n * k // 2 + nb + 4 * ((nb + 255) // 256) + 4 + 2 * n * k
@@ -499,13 +506,29 @@ def run_ours(args, rank, world, local):
         def dstep():
             for w in sub:
                 nf4.nf4_dequantize(w, torch.bfloat16, out=out[: w.n * w.k].view(w.n, w.k))
-        qstep(); dstep()
+        # merge a rank-16 LoRA update into every tensor of the layer and requantize
+        # (codes + fp32 absmax out, the merged bf16 weight not written)
+        rm = 16
+        lora_mats = [((synth.activations(rm, w.k, seed=synth.seed_for(6, i), device=dev).float() * 0.02)
+                      .to(torch.bfloat16),
+                      (synth.activations(w.n, rm, seed=synth.seed_for(6, 100 + i), device=dev).float() * 0.02)
+                      .to(torch.bfloat16)) for i, w in enumerate(sub)]
+
+        def mstep():
+            for w, (dm, um) in zip(sub, lora_mats):
+                nf4.nf4_merge_lora(w, dm, um, 2.0, wq=wq, absmax=am)
+        qstep(); dstep(); mstep()
         tq = _events_time(qstep, 5, stream)
         td = _events_time(dstep, 5, stream)
+        tm = _events_time(mstep, 5, stream)
         qb = sum(quant_bytes(w.n, w.k) for w in sub)
         db = sum(dequant_bytes(w.n, w.k) for w in sub)
+        mb = sum(merge_bytes(w.n, w.k, rm) for w in sub)
         qd = {"quantize_dq_gbs": round(qb / tq / 1e9, 1), "dequantize_bf16_gbs": round(db / td / 1e9, 1),
+              "merge_lora_gbs": round(mb / tm / 1e9, 1), "merge_lora_ms_per_layer": round(tm * 1e3, 3),
+              "merge_lora_r": rm,
               "sample": "one decoder layer (7 tensors, 202M params) per rep, bf16 in/out"}
+        del lora_mats
         del Wb, out
 
     clocks = clk.summary()

@@ -290,6 +290,34 @@ nf4_status_t nf4_linear_lora(const void* X, int64_t m, const nf4_weight_t* w, co
                              nf4_stream_t stream);
 
 /*
+ * nf4_merge_lora -- fold a trained LoRA update into the quantized weight for
+ * deployment ([P4] "8. LoRA 的合併（Merge）": the 4-bit weight is dequantized to
+ * bf16, the product of the LoRA matrices is added in bf16, and the result is
+ * quantized to 4 bits again).  Per element (o, c):
+ *   What  = bf16_rn(level * ahat)                       (as nf4_dequantize to bf16)
+ *   delta = fp32 fused-multiply-add chain over j = 0 .. r-1 of up[o][j] * down[j][c]
+ *   Wnew  = bf16_rn(What + fp32(scale * delta))
+ * Wnew is then quantized blockwise exactly as nf4_quantize quantizes a bf16
+ * weight.  The result is bit-identical to dequantize -> add -> quantize done
+ * in that arithmetic; run nf4_double_quant on absmax_out to finish the
+ * storage format.  The input weight is not modified (wq_out may not alias w->wq).
+ *   w          the [n, k] quantized weight (k % 64 == 0)
+ *   lora_down  device, bf16 [r, k] row-major, 16-byte aligned
+ *   lora_up    device, bf16 [n, r] row-major, 16-byte aligned
+ *   r          rank, 1 .. 256
+ *   scale      e.g. lora_alpha / r
+ *   w_new      device, bf16 [n, k], 16-byte aligned, or NULL to skip writing the
+ *              merged bf16 weight (output)
+ *   wq_out     device, uint8 [n * k / 2] packed codes, 16-byte aligned (output)
+ *   absmax_out device, fp32 [n * k / 64], 4-byte aligned (output)
+ * Errors: NF4_ERR_NULL, NF4_ERR_STATE, NF4_ERR_SHAPE (k % 64 != 0, r out of
+ * range), NF4_ERR_ALIGN, NF4_ERR_UNSUPPORTED, NF4_ERR_CUDA.
+ */
+nf4_status_t nf4_merge_lora(const nf4_weight_t* w, const void* lora_down, const void* lora_up, int32_t r,
+                            float scale, void* w_new, uint8_t* wq_out, float* absmax_out,
+                            nf4_stream_t stream);
+
+/*
  * nf4_linear_workspace_bytes -- bytes of the optional split-k workspace that
  * nf4_linear_ws can use for Y[m, n] = X[m, k] * What^T on the current device;
  * 0 when that product splits no k range (then no workspace is needed).  The

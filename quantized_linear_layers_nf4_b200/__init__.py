@@ -14,6 +14,9 @@ calls.  Functions carry the C names:
   the frozen base)
 * ``nf4_linear_lora(X, weight, down, up, scale, workspace=...)`` -> the QLoRA
   layer ``X @ W_hat^T + scale * (X @ down^T) @ up^T``
+* ``nf4_merge_lora(weight, down, up, scale)`` -> ``(wq, absmax, w_new)``: the
+  trained update folded into the weight and quantized again (``merge_lora``
+  adds the double quantization and returns an ``NF4Weight``)
 
 ``quantize_weight(W)`` runs the first two and returns an ``NF4Weight``.
 """
@@ -29,6 +32,7 @@ from ._lib import NF4_BF16, NF4_F32, NF4Error, nf4_weight_t
 
 __all__ = ["NF4Weight", "NF4Error", "nf4_quantize", "nf4_double_quant", "nf4_dequantize",
            "nf4_linear", "nf4_linear_ex", "nf4_linear_dx", "nf4_linear_lora", "lora_workspace",
+           "nf4_merge_lora", "merge_lora",
            "nf4_linear_workspace_bytes", "linear_workspace",
            "quantize_weight", "nf4_codebook", "library_path"]
 
@@ -248,3 +252,36 @@ def nf4_linear_lora(X: torch.Tensor, weight: NF4Weight, down: torch.Tensor, up: 
                                           workspace.numel() * workspace.element_size(), _stream(stream)),
                "nf4_linear_lora")
     return out
+
+
+def nf4_merge_lora(weight: NF4Weight, down: torch.Tensor, up: torch.Tensor, scale: float,
+                   want_bf16: bool = False, wq: torch.Tensor | None = None,
+                   absmax: torch.Tensor | None = None, stream=None):
+    """Dequantize to bf16, add scale * up @ down in bf16 and quantize again.
+    Returns (wq, absmax fp32, w_new bf16 [n, k] or None)."""
+    for t, name in ((down, "down"), (up, "up")):
+        _need_cuda(t, name)
+    if down.dtype != torch.bfloat16 or up.dtype != torch.bfloat16:
+        raise ValueError("down and up must be bfloat16")
+    r = down.shape[0]
+    if down.dim() != 2 or down.shape != (r, weight.k) or up.shape != (weight.n, r):
+        raise ValueError("shapes: down [r, k], up [n, r]")
+    numel = weight.n * weight.k
+    dev = weight.wq.device
+    if wq is None:
+        wq = torch.empty(numel // 2, dtype=torch.uint8, device=dev)
+    if absmax is None:
+        absmax = torch.empty(numel // 64, dtype=torch.float32, device=dev)
+    w_new = torch.empty((weight.n, weight.k), dtype=torch.bfloat16, device=dev) if want_bf16 else None
+    st = weight.struct()
+    _lib.check(_lib.lib().nf4_merge_lora(ctypes.byref(st), _ptr(down), _ptr(up), r, float(scale),
+                                         ctypes.c_void_p(0) if w_new is None else _ptr(w_new), _ptr(wq),
+                                         _ptr(absmax), _stream(stream)), "nf4_merge_lora")
+    return wq, absmax, w_new
+
+
+def merge_lora(weight: NF4Weight, down: torch.Tensor, up: torch.Tensor, scale: float, stream=None) -> NF4Weight:
+    """nf4_merge_lora followed by nf4_double_quant: the merged, requantized weight."""
+    wq, absmax, _ = nf4_merge_lora(weight, down, up, scale, stream=stream)
+    q, s, mu = nf4_double_quant(absmax, stream=stream)
+    return NF4Weight(weight.n, weight.k, wq, q, s, mu)

@@ -53,6 +53,8 @@ SIGNATURES = {
     "nf4_linear_lora": (ctypes.c_int, [_p, _i64, ctypes.POINTER(nf4_weight_t), _p, _p, ctypes.c_int32,
                                        ctypes.c_float, _p, ctypes.c_int, _p, ctypes.c_uint32, _p, ctypes.c_size_t,
                                        _p]),
+    "nf4_merge_lora": (ctypes.c_int, [ctypes.POINTER(nf4_weight_t), _p, _p, ctypes.c_int32, ctypes.c_float, _p,
+                                      _p, _p, _p]),
     "nf4_linear_ws": (ctypes.c_int, [_p, _i64, ctypes.POINTER(nf4_weight_t), _p, ctypes.c_int, _p,
                                      ctypes.c_uint32, _p, ctypes.c_size_t, _p]),
 }

@@ -187,6 +187,23 @@ nf4_status_t nf4_linear_lora(const void* X, int64_t m, const nf4_weight_t* w, co
                                         static_cast<char*>(workspace) + tb, lora, dev, s));
 }
 
+nf4_status_t nf4_merge_lora(const nf4_weight_t* w, const void* lora_down, const void* lora_up, int32_t r,
+                            float scale, void* w_new, uint8_t* wq_out, float* absmax_out,
+                            nf4_stream_t stream) {
+    nf4_status_t st = check_weight(w);
+    if (st != NF4_OK) return st;
+    if (!lora_down || !lora_up || !wq_out || !absmax_out) return NF4_ERR_NULL;
+    if (w->k % NF4_BLOCKSIZE != 0 || r < 1 || r > 256) return NF4_ERR_SHAPE;
+    if (!aligned(lora_down, 16) || !aligned(lora_up, 16) || !aligned(wq_out, 16) || !aligned(absmax_out, 4) ||
+        (w_new && !aligned(w_new, 16)))
+        return NF4_ERR_ALIGN;
+    nf4::DeviceInfo dev;
+    if ((st = device_ok(&dev)) != NF4_OK) return st;
+    return from_cuda(nf4::launch_merge_lora(w->wq, w->absmax_q, w->absmax_scale, w->absmax_offset, w->n, w->k,
+                                            lora_down, lora_up, r, scale, w_new, wq_out, absmax_out, dev,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t nf4_linear_lora_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t r) {
     if (m < 1 || n < 1 || k < 1 || k % NF4_BLOCKSIZE != 0 || r < 1 || r > 256) return 0;
     nf4::DeviceInfo dev;

@@ -60,6 +60,13 @@ cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int
 cudaError_t launch_lora_down(const void* X, int64_t m, int64_t k, const void* down, int r, float scale, float* t,
                              __nv_bfloat16* t_hi, __nv_bfloat16* t_lo, cudaStream_t stream);
 
+// Merge a LoRA update into the quantized weight and requantize: w_new (bf16
+// [n, k], may be null), wq_out [n*k/2] and absmax_out [n*k/64] fp32.
+cudaError_t launch_merge_lora(const uint8_t* wq, const int8_t* absmax_q, const float* absmax_scale,
+                              const float* absmax_offset, int64_t n, int64_t k, const void* down, const void* up,
+                              int r, float scale, void* w_new, uint8_t* wq_out, float* absmax_out,
+                              const DeviceInfo& dev, cudaStream_t stream);
+
 cudaError_t launch_gemm_dx(const void* dY, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                            const float* absmax_scale, const float* absmax_offset, int64_t n, int64_t k, void* dX,
                            bool dx_bf16, int32_t* dev_status, const DeviceInfo& dev, cudaStream_t stream);

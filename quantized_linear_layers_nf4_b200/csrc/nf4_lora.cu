@@ -1,4 +1,5 @@
-// nf4_lora.cu -- the down-projection of a LoRA layer, t = scale * X down^T.
+// nf4_lora.cu -- the down-projection of a LoRA layer, t = scale * X down^T, and
+// the merge of a trained update into the quantized weight (bottom of the file).
 //
 // Source: page "LLM 相關知識" (technicalnotes), section "2-2. LoRA（低秩適應）": the
 // frozen W acts as W + dW with dW = A x B of low rank r, trained in bf16; with W
@@ -62,6 +63,101 @@ __global__ void __launch_bounds__(256) k_lora_down(const __nv_bfloat16* __restri
     }
 }
 
+
+// ---------------------------------------------------------------------------
+// Merge + requantize (page "LLM 相關知識" (technicalnotes), section "8. LoRA 的
+// 合併（Merge）": the 4-bit weight is dequantized to bf16, the product of the two
+// LoRA matrices is added in bf16, and the sum is quantized back to 4 bits for
+// deployment).  Per element (o, c):
+//   What  = bf16_rn(fp32(level * ahat))                 the bf16 dequantized weight
+//   delta = fma chain over j = 0 .. r-1 of up[o][j] * down[j][c], from 0, in fp32
+//   Wnew  = bf16_rn(fp32(What + fp32(scale * delta)))
+// and Wnew is then quantized blockwise exactly as k_nf4_quantize does.  Lane
+// layout as in quantization: a lane owns 8 consecutive elements of one row
+// (k % 64 == 0 keeps each 64-block inside a row), 8 lanes one block.  down is
+// small ([r, k] bf16) and is re-read from L1/L2 by every row.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_nf4_merge_lora(const uint32_t* __restrict__ wq32,
+                                                        const int8_t* __restrict__ absmax_q,
+                                                        const float* __restrict__ absmax_scale,
+                                                        const float* __restrict__ mu_ptr, int64_t k,
+                                                        int64_t n_groups, const __nv_bfloat16* __restrict__ down,
+                                                        const __nv_bfloat16* __restrict__ up, int r, float scale,
+                                                        uint4* __restrict__ w_new, uint32_t* __restrict__ wq_out,
+                                                        float* __restrict__ absmax_out) {
+    __shared__ float lv[16];
+    if (threadIdx.x < 16) lv[threadIdx.x] = kLevels[threadIdx.x];
+    __syncthreads();
+    const float mu = __ldg(mu_ptr);
+    const uint16_t* up16 = reinterpret_cast<const uint16_t*>(up);
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    const int64_t n_chunks = (n_groups + 31) >> 5;
+    for (int64_t chunk = warp; chunk < n_chunks; chunk += n_warps) {
+        const int64_t g = (chunk << 5) + lane;   // group of 8 elements
+        const bool valid = g < n_groups;          // whole 8-lane blocks agree
+        float w[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = 0.0f;
+        if (valid) {
+            const uint32_t packed = __ldg(wq32 + g);
+            const int64_t b = g >> 3;
+            const float a = absmax_hat(__ldg(absmax_q + b), __ldg(absmax_scale + (b >> 8)), mu);
+            const int64_t e0 = g * 8;
+            const int64_t o = e0 / k;
+            const int64_t c0 = e0 - o * k;
+            float acc[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+            const uint16_t* u_row = up16 + o * r;
+            const __nv_bfloat16* d_col = down + c0;
+#pragma unroll 4
+            for (int j = 0; j < r; ++j) {
+                const float u = bf16_bits_to_float(__ldg(u_row + j));
+                const uint4 dv = __ldg(reinterpret_cast<const uint4*>(d_col + static_cast<int64_t>(j) * k));
+                const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    acc[2 * i] = __fmaf_rn(u, bf16_bits_to_float(dw[i] & 0xffffu), acc[2 * i]);
+                    acc[2 * i + 1] = __fmaf_rn(u, bf16_bits_to_float(dw[i] >> 16), acc[2 * i + 1]);
+                }
+            }
+            uint32_t out[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t byte = (packed >> (8 * i)) & 0xffu;
+                // element 2i sits in the high nibble
+                const float what0 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(lv[byte >> 4], a)));
+                const float what1 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(lv[byte & 15u], a)));
+                const float s0 = __fadd_rn(what0, __fmul_rn(scale, acc[2 * i]));
+                const float s1 = __fadd_rn(what1, __fmul_rn(scale, acc[2 * i + 1]));
+                out[i] = pack_bf16x2(s0, s1);
+                w[2 * i] = bf16_bits_to_float(out[i] & 0xffffu);
+                w[2 * i + 1] = bf16_bits_to_float(out[i] >> 16);
+            }
+            if (w_new) __stcs(w_new + g, make_uint4(out[0], out[1], out[2], out[3]));
+        }
+        float a = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(w[e]));
+        a = fmaxf(a, __shfl_xor_sync(kFull, a, 1));
+        a = fmaxf(a, __shfl_xor_sync(kFull, a, 2));
+        a = fmaxf(a, __shfl_xor_sync(kFull, a, 4));
+        uint32_t packed = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t hi = static_cast<uint32_t>(quantize_one(w[2 * i], a));
+            const uint32_t lo = static_cast<uint32_t>(quantize_one(w[2 * i + 1], a));
+            packed |= ((hi << 4) | lo) << (8 * i);
+        }
+        if (valid) {
+            wq_out[g] = packed;
+            if ((lane & 7) == 0) absmax_out[g >> 3] = a;
+        }
+    }
+}
+
 }  // namespace lora
 
 cudaError_t launch_lora_down(const void* X, int64_t m, int64_t k, const void* down, int r, float scale, float* t,
@@ -70,6 +166,23 @@ cudaError_t launch_lora_down(const void* X, int64_t m, int64_t k, const void* do
     lora::k_lora_down<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), k,
                                                                       static_cast<const __nv_bfloat16*>(down), r,
                                                                       scale, t, t_hi, t_lo);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_merge_lora(const uint8_t* wq, const int8_t* absmax_q, const float* absmax_scale,
+                              const float* absmax_offset, int64_t n, int64_t k, const void* down, const void* up,
+                              int r, float scale, void* w_new, uint8_t* wq_out, float* absmax_out,
+                              const DeviceInfo& dev, cudaStream_t stream) {
+    const int64_t n_groups = n * k / 8;
+    const int64_t n_chunks = (n_groups + 31) / 32;
+    int64_t blocks = (n_chunks + 7) / 8;
+    const int64_t cap = static_cast<int64_t>(dev.sm_count) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    lora::k_nf4_merge_lora<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        reinterpret_cast<const uint32_t*>(wq), absmax_q, absmax_scale, absmax_offset, k, n_groups,
+        static_cast<const __nv_bfloat16*>(down), static_cast<const __nv_bfloat16*>(up), r, scale,
+        static_cast<uint4*>(w_new), reinterpret_cast<uint32_t*>(wq_out), absmax_out);
     return cudaGetLastError();
 }
 

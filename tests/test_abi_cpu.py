@@ -167,6 +167,20 @@ def test_linear_lora_validation(L):
     assert L.nf4_linear_lora_workspace_bytes(4, 4096, 4096, 0) == 0
 
 
+def test_merge_lora_validation(L):
+    mg = L.nf4_merge_lora
+    w = ctypes.byref(_weight())
+    assert mg(w, None, FAKE, 16, 2.0, None, FAKE, FAKE, None) == -1            # no down
+    assert mg(w, FAKE, FAKE, 16, 2.0, None, None, FAKE, None) == -1            # no codes out
+    assert mg(w, FAKE, FAKE, 16, 2.0, None, FAKE, None, None) == -1            # no absmax out
+    assert mg(w, FAKE, FAKE, 0, 2.0, None, FAKE, FAKE, None) == -2             # rank 0
+    assert mg(w, FAKE, FAKE, 257, 2.0, None, FAKE, FAKE, None) == -2
+    assert mg(ctypes.byref(_weight(k=96)), FAKE, FAKE, 16, 2.0, None, FAKE, FAKE, None) == -2
+    assert mg(w, FAKE, ODD, 16, 2.0, None, FAKE, FAKE, None) == -3
+    assert mg(w, FAKE, FAKE, 16, 2.0, ODD, FAKE, FAKE, None) == -3             # w_new misaligned
+    assert mg(ctypes.byref(_weight(magic=7)), FAKE, FAKE, 16, 2.0, None, FAKE, FAKE, None) == -5
+
+
 def test_valid_call_without_a_gpu_reports_instead_of_crashing(L):
     """On a host without a usable B200 a fully valid call must come back with a
     status (no device / unsupported device), never crash or launch."""

@@ -346,6 +346,53 @@ def test_linear_lora(nf4, m, n, k, r, scale):
     assert torch.equal(Y0, nf4.nf4_linear(X, weight, torch.float32))
 
 
+@pytest.mark.parametrize("n,k,r,scale", [(128, 256, 16, 2.0), (100, 192, 5, 0.5), (1, 64, 1, 1.0),
+                                         (300, 640, 256, 0.125), (4096, 4096, 64, 2.0), (11008, 4096, 16, 0.25)])
+def test_merge_lora(nf4, n, k, r, scale):
+    """Merge + requantize: the merged bf16 weight, its packed codes and fp32
+    absmax bit-exact against the oracle (whole arrays), then the double
+    quantization of the merged absmax; a zero scale requantizes the bf16
+    dequantized weight."""
+    W = synth.weight_normal(n, k, seed=1900 + n + r, dtype=torch.bfloat16, device="cuda")
+    down = (synth.activations(r, k, seed=1910 + r, device="cuda").float() * 0.05).to(torch.bfloat16)
+    up = (synth.activations(n, r, seed=1920 + r, device="cuda").float() * 0.05).to(torch.bfloat16)
+    weight, orc = _check_quant(nf4, W, full_dequant=False, rows=[0, n - 1])
+    owq, oq, os_, omu = orc
+    wq, absmax, w_new = nf4.nf4_merge_lora(weight, down, up, scale, want_bf16=True)
+    wq2, absmax2, none = nf4.nf4_merge_lora(weight, down, up, scale)
+    torch.cuda.synchronize()
+    assert none is None
+    ow, owq_new, oam_new = O.merge_lora(owq, oq, os_, omu, n, k, _bits(down).reshape(r, k),
+                                        _bits(up).reshape(n, r), scale)
+    _assert_equal(w_new.view(torch.int16).view(-1), ow.view(np.int16), "merged bf16 weight")
+    _assert_equal(wq, owq_new, "merged codes")
+    _assert_equal(absmax, oam_new, "merged absmax")
+    assert torch.equal(wq, wq2) and torch.equal(absmax, absmax2)
+    merged = nf4.merge_lora(weight, down, up, scale)
+    oq2, os2, omu2 = O.double_quant(oam_new)
+    _assert_equal(merged.wq, owq_new, "merged weight codes")
+    _assert_equal(merged.absmax_q, oq2, "merged absmax_q")
+    _assert_equal(merged.absmax_scale, os2, "merged absmax_scale")
+    _assert_equal(merged.absmax_offset, np.array([omu2], np.float32), "merged mean")
+    # scale 0: the requantized bf16 dequantized weight, through the other kernels
+    wq0, absmax0, w0 = nf4.nf4_merge_lora(weight, down, up, 0.0, want_bf16=True)
+    d16 = nf4.nf4_dequantize(weight, torch.bfloat16)
+    assert torch.equal(w0, d16)
+    wq_ref, absmax_ref = nf4.nf4_quantize(d16)
+    assert torch.equal(wq0, wq_ref) and torch.equal(absmax0, absmax_ref)
+
+
+def test_merge_lora_errors(nf4):
+    W = synth.weight_normal(64, 64, seed=1950, dtype=torch.bfloat16, device="cuda")
+    weight = nf4.quantize_weight(W)
+    down = torch.zeros(4, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError):
+        nf4.nf4_merge_lora(weight, down, torch.zeros(64, 5, dtype=torch.bfloat16, device="cuda"), 1.0)
+    with pytest.raises(nf4.NF4Error):   # rank above 256
+        nf4.nf4_merge_lora(weight, torch.zeros(300, 64, dtype=torch.bfloat16, device="cuda"),
+                           torch.zeros(64, 300, dtype=torch.bfloat16, device="cuda"), 1.0)
+
+
 def test_deterministic_and_stream_aware(nf4):
     W = synth.weight_normal(512, 1024, seed=9, dtype=torch.bfloat16, device="cuda")
     X = synth.activations(16, 1024, seed=10, device="cuda")
