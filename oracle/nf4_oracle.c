@@ -93,17 +93,53 @@ static const float* codebook(void) {
 }
 
 /* ---------------------------------------------------------------------------
+ * The FP4 codebook.  [P5] §2.2 code walk: bitsandbytes' FP4 is its generic
+ * float-format builder instantiated with a sign bit, 2 exponent bits and 1
+ * mantissa bit; [P3] "4-bit 量化": FP4 is a conventional 4-bit float; [P1] "NF4 不是
+ * 一般四位元浮點格式": NF4 is not that IEEE-style FP4.  Reading: the code's bits
+ * are s | e1 e0 | m with exponent bias 1; e = 0 is subnormal with magnitude m/2,
+ * otherwise the magnitude is (1 + m/2) * 2^(e-1).  The 16 values are divided by
+ * the largest magnitude in fp64 and rounded to fp32, so that, like the NF4
+ * levels, they span [-1, 1].  The table is in code order (not sorted): codes
+ * 0..7 are the non-negative values, 8..15 their negatives, code 8 is -0.
+ * ------------------------------------------------------------------------- */
+void orc_fp4_codebook(float c[16]) {
+    double v[16];
+    double top = 0.0;
+    for (int code = 0; code < 16; ++code) {
+        const int s = code >> 3, e = (code >> 1) & 3, m = code & 1;
+        const double mag = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+        v[code] = s ? -mag : mag;
+        if (mag > top) top = mag;
+    }
+    for (int i = 0; i < 16; ++i) c[i] = (float)(v[i] / top);
+}
+
+static const float* fp4_codebook(void) {
+    static float c[16];
+    static int ready = 0;
+    if (!ready) {
+        orc_fp4_codebook(c);
+        ready = 1;
+    }
+    return c;
+}
+
+static const float* table_of(int qt) { return qt == ORC_FP4 ? fp4_codebook() : codebook(); }
+
+/* ---------------------------------------------------------------------------
  * Quantization ([P5] §2.2 example and Figure 2-2, steps 1-4):
  *   split the flattened weight into blocks of 64, absmax per block,
  *   x = w / absmax, map x to the nearest level, pack two 4-bit indices per byte.
  * ------------------------------------------------------------------------- */
 
-/* Nearest level by exhaustive search over the 16 levels, ties to the lower
- * index.  Distances are taken in fp64: x and c_i are fp32 in [-1, 1], so every
- * comparison that is close enough to tie involves operands of similar
- * magnitude whose fp64 difference is exact. */
-static int nearest_level(float x) {
-    const float* c = codebook();
+/* Nearest level by exhaustive search over the 16 levels of table c, ties to the
+ * lower index (for FP4, whose table is in code order, that sends a tie between
+ * two magnitudes toward zero and every x of either sign nearest to zero to code
+ * 0, +0).  Distances are taken in fp64: x and c_i are fp32 in [-1, 1], so every
+ * comparison that is close enough to tie involves operands of similar magnitude
+ * whose fp64 difference is exact. */
+static int nearest_level(const float* c, float x) {
     int best = 0;
     double best_d = fabs((double)x - (double)c[0]);
     for (int i = 1; i < 16; ++i) {
@@ -116,8 +152,10 @@ static int nearest_level(float x) {
     return best;
 }
 
-int orc_quantize_f32(const float* w, int64_t n_elem, uint8_t* wq, float* absmax) {
+int orc_quantize_f32_qt(const float* w, int64_t n_elem, int qt, uint8_t* wq, float* absmax) {
+    if (qt != ORC_NF4 && qt != ORC_FP4) return -4;
     if (n_elem <= 0 || n_elem % 64 != 0) return -2;
+    const float* c = table_of(qt);
     const int64_t nb = n_elem / 64;
     for (int64_t b = 0; b < nb; ++b) {
         const float* blk = w + b * 64;
@@ -131,10 +169,12 @@ int orc_quantize_f32(const float* w, int64_t n_elem, uint8_t* wq, float* absmax)
         int idx[64];
         for (int j = 0; j < 64; ++j) {
             if (am == 0.0f) {
-                idx[j] = 7; /* zero block: every element is the exact-zero level */
+                /* zero block: every element is the exact-zero level (FP4: +0) */
+                if (qt == ORC_FP4) idx[j] = 0;
+                else idx[j] = 7;
             } else {
                 float x = blk[j] / am;
-                idx[j] = nearest_level(x);
+                idx[j] = nearest_level(c, x);
             }
         }
         for (int i = 0; i < 32; ++i)
@@ -150,15 +190,23 @@ static float bf16_bits_to_f32(uint16_t h) {
     return f;
 }
 
-int orc_quantize_bf16(const uint16_t* w, int64_t n_elem, uint8_t* wq, float* absmax) {
+int orc_quantize_bf16_qt(const uint16_t* w, int64_t n_elem, int qt, uint8_t* wq, float* absmax) {
     if (n_elem <= 0 || n_elem % 64 != 0) return -2;
     float tmp[64];
     for (int64_t b = 0; b < n_elem / 64; ++b) {
         for (int j = 0; j < 64; ++j) tmp[j] = bf16_bits_to_f32(w[b * 64 + j]);
-        int rc = orc_quantize_f32(tmp, 64, wq + b * 32, absmax + b);
+        int rc = orc_quantize_f32_qt(tmp, 64, qt, wq + b * 32, absmax + b);
         if (rc) return rc;
     }
     return 0;
+}
+
+int orc_quantize_f32(const float* w, int64_t n_elem, uint8_t* wq, float* absmax) {
+    return orc_quantize_f32_qt(w, n_elem, ORC_NF4, wq, absmax);
+}
+
+int orc_quantize_bf16(const uint16_t* w, int64_t n_elem, uint8_t* wq, float* absmax) {
+    return orc_quantize_bf16_qt(w, n_elem, ORC_NF4, wq, absmax);
 }
 
 /* ---------------------------------------------------------------------------
@@ -250,10 +298,11 @@ float orc_absmax_hat(const int8_t* absmax_q, const float* absmax_scale, float mu
  * compute dtype layer by layer; [P1] "QLoRA 把 frozen 4-bit base ...": the base
  * is dequantized in forward and backward):  w = fp32(c[idx] * a).
  * ------------------------------------------------------------------------- */
-int orc_dequantize_range(const uint8_t* wq, const int8_t* absmax_q, const float* absmax_scale,
-                         float mu, int64_t begin, int64_t count, float* out_f32) {
+int orc_dequantize_range_qt(const uint8_t* wq, const int8_t* absmax_q, const float* absmax_scale,
+                            float mu, int64_t begin, int64_t count, int qt, float* out_f32) {
+    if (qt != ORC_NF4 && qt != ORC_FP4) return -4;
     if (begin < 0 || count < 0 || begin % 64 != 0 || count % 64 != 0) return -2;
-    const float* c = codebook();
+    const float* c = table_of(qt);
     for (int64_t e = 0; e < count; ++e) {
         const int64_t g = begin + e;
         const uint8_t byte = wq[g / 2];
@@ -262,6 +311,11 @@ int orc_dequantize_range(const uint8_t* wq, const int8_t* absmax_q, const float*
         out_f32[e] = c[idx] * a;
     }
     return 0;
+}
+
+int orc_dequantize_range(const uint8_t* wq, const int8_t* absmax_q, const float* absmax_scale,
+                         float mu, int64_t begin, int64_t count, float* out_f32) {
+    return orc_dequantize_range_qt(wq, absmax_q, absmax_scale, mu, begin, count, ORC_NF4, out_f32);
 }
 
 /* Round to nearest bf16, ties to even: keep the top 16 bits after adding half an

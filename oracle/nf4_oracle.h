@@ -31,7 +31,10 @@
  *     defined by orc_dq_sum; r = fp32(absmax - mu); per block of 256: s = max|r|,
  *     q = round_half_even(fp32(fp32(r / s) * 127)), q = 0 when s = 0;
  *   - absmax dequant: a = fp32(fp32(fp32(q / 127) * s) + mu), each step rounded;
- *   - weight dequant: w = fp32(c[idx] * a); the bf16 form rounds that to nearest even.
+ *   - weight dequant: w = fp32(c[idx] * a); the bf16 form rounds that to nearest even;
+ *   - FP4 (the *_qt functions): the same pipeline with the 16 values of a sign,
+ *     2-bit exponent (bias 1, subnormal at 0) and 1-bit mantissa float, in code
+ *     order, scaled to [-1, 1]; a zero block maps to code 0 (+0).
  *
  * Every floating-point step is an IEEE binary32/binary64 operation with
  * round-to-nearest-even; the library is built with -ffp-contract=off and without
@@ -53,12 +56,26 @@ double orc_norm_ppf(double p);
 /* The 16 NF4 levels, ascending, in fp32: c[0] = -1, c[7] = 0, c[15] = +1. */
 void orc_codebook(float c[16]);
 
+/* Codebook selector of the *_qt functions. */
+#define ORC_NF4 0
+#define ORC_FP4 1
+
+/* The 16 FP4 values in code order (sign | 2 exponent bits, bias 1 | 1 mantissa
+ * bit, subnormal at exponent 0), divided by the largest magnitude: codes 0..7 =
+ * 0, 1/12, 1/6, 1/4, 1/3, 1/2, 2/3, 1 (fp32-rounded); codes 8..15 their
+ * negatives (code 8 = -0). */
+void orc_fp4_codebook(float c[16]);
+
 /* Blockwise NF4 quantization of n_elem fp32 weights (n_elem % 64 == 0).
  * Writes wq[n_elem/2] packed codes and absmax[n_elem/64].  Returns 0, or -2 on a
  * bad size, -9 on a non-finite input. */
 int orc_quantize_f32(const float* w, int64_t n_elem, uint8_t* wq, float* absmax);
 /* Same, from bf16 bit patterns (widened exactly to fp32 first). */
 int orc_quantize_bf16(const uint16_t* w, int64_t n_elem, uint8_t* wq, float* absmax);
+/* The same with the codebook chosen by qt (ORC_NF4 or ORC_FP4; -4 otherwise).
+ * A zero block is code 7 for NF4 and code 0 (+0) for FP4. */
+int orc_quantize_f32_qt(const float* w, int64_t n_elem, int qt, uint8_t* wq, float* absmax);
+int orc_quantize_bf16_qt(const uint16_t* w, int64_t n_elem, int qt, uint8_t* wq, float* absmax);
 
 /* Fixed-order fp64 sum of the absmax values (the tree defined in the .c file). */
 double orc_dq_sum(const float* absmax, int64_t nb);
@@ -78,6 +95,9 @@ float orc_absmax_hat(const int8_t* absmax_q, const float* absmax_scale, float mu
  * the full arrays (global indexing). */
 int orc_dequantize_range(const uint8_t* wq, const int8_t* absmax_q, const float* absmax_scale,
                          float mu, int64_t begin, int64_t count, float* out_f32);
+/* The same with the codebook chosen by qt. */
+int orc_dequantize_range_qt(const uint8_t* wq, const int8_t* absmax_q, const float* absmax_scale,
+                            float mu, int64_t begin, int64_t count, int qt, float* out_f32);
 
 /* fp32 -> bf16 bit pattern, round to nearest, ties to even (finite inputs). */
 void orc_f32_to_bf16(const float* x, int64_t n, uint16_t* out);

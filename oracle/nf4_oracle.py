@@ -36,6 +36,14 @@ def _bind(L):
     L.orc_quantize_f32.restype = ctypes.c_int
     L.orc_quantize_bf16.argtypes = [p, i64, p, p]
     L.orc_quantize_bf16.restype = ctypes.c_int
+    L.orc_fp4_codebook.argtypes = [p]
+    L.orc_fp4_codebook.restype = None
+    L.orc_quantize_f32_qt.argtypes = [p, i64, ctypes.c_int, p, p]
+    L.orc_quantize_f32_qt.restype = ctypes.c_int
+    L.orc_quantize_bf16_qt.argtypes = [p, i64, ctypes.c_int, p, p]
+    L.orc_quantize_bf16_qt.restype = ctypes.c_int
+    L.orc_dequantize_range_qt.argtypes = [p, p, p, ctypes.c_float, i64, i64, ctypes.c_int, p]
+    L.orc_dequantize_range_qt.restype = ctypes.c_int
     L.orc_dq_sum.argtypes = [p, i64]
     L.orc_dq_sum.restype = ctypes.c_double
     L.orc_dq_mean.argtypes = [p, i64]
@@ -74,23 +82,37 @@ def norm_ppf(p: float) -> float:
     return lib().orc_norm_ppf(float(p))
 
 
-def codebook() -> np.ndarray:
+QUANT_TYPES = {"nf4": 0, "fp4": 1}
+
+
+def _qt(quant_type: str) -> int:
+    if quant_type not in QUANT_TYPES:
+        raise ValueError("quant_type must be 'nf4' or 'fp4'")
+    return QUANT_TYPES[quant_type]
+
+
+def codebook(quant_type: str = "nf4") -> np.ndarray:
+    """The 16 levels: NF4 ascending, FP4 in code order."""
     c = np.zeros(16, dtype=np.float32)
-    lib().orc_codebook(_ptr(c))
+    if _qt(quant_type) == 1:
+        lib().orc_fp4_codebook(_ptr(c))
+    else:
+        lib().orc_codebook(_ptr(c))
     return c
 
 
-def quantize(w: np.ndarray):
+def quantize(w: np.ndarray, quant_type: str = "nf4"):
     """w: float32 array, or uint16 array of bf16 bit patterns; any shape with
     size % 64 == 0.  Returns (wq uint8 [size/2], absmax float32 [size/64])."""
+    qt = _qt(quant_type)
     w = np.ascontiguousarray(w)
     n = w.size
     wq = np.zeros(n // 2, dtype=np.uint8)
     absmax = np.zeros(n // 64, dtype=np.float32)
     if w.dtype == np.float32:
-        rc = lib().orc_quantize_f32(_ptr(w), n, _ptr(wq), _ptr(absmax))
+        rc = lib().orc_quantize_f32_qt(_ptr(w), n, qt, _ptr(wq), _ptr(absmax))
     elif w.dtype == np.uint16:
-        rc = lib().orc_quantize_bf16(_ptr(w), n, _ptr(wq), _ptr(absmax))
+        rc = lib().orc_quantize_bf16_qt(_ptr(w), n, qt, _ptr(wq), _ptr(absmax))
     else:
         raise TypeError("oracle quantize takes float32 or bf16 bit patterns (uint16)")
     if rc != 0:
@@ -129,20 +151,22 @@ def absmax_hat(absmax_q: np.ndarray, absmax_scale: np.ndarray, mu) -> np.ndarray
                     dtype=np.float32)
 
 
-def dequantize_range(wq, absmax_q, absmax_scale, mu, begin: int, count: int) -> np.ndarray:
+def dequantize_range(wq, absmax_q, absmax_scale, mu, begin: int, count: int,
+                     quant_type: str = "nf4") -> np.ndarray:
+    qt = _qt(quant_type)
     wq = np.ascontiguousarray(wq, dtype=np.uint8)
     q = np.ascontiguousarray(absmax_q, dtype=np.int8)
     s = np.ascontiguousarray(absmax_scale, dtype=np.float32)
     out = np.zeros(count, dtype=np.float32)
-    rc = lib().orc_dequantize_range(_ptr(wq), _ptr(q), _ptr(s), float(mu), int(begin), int(count),
-                                    _ptr(out))
+    rc = lib().orc_dequantize_range_qt(_ptr(wq), _ptr(q), _ptr(s), float(mu), int(begin), int(count), qt,
+                                       _ptr(out))
     if rc != 0:
         raise ValueError("orc_dequantize_range failed with %d" % rc)
     return out
 
 
-def dequantize(wq, absmax_q, absmax_scale, mu) -> np.ndarray:
-    return dequantize_range(wq, absmax_q, absmax_scale, mu, 0, 2 * np.asarray(wq).size)
+def dequantize(wq, absmax_q, absmax_scale, mu, quant_type: str = "nf4") -> np.ndarray:
+    return dequantize_range(wq, absmax_q, absmax_scale, mu, 0, 2 * np.asarray(wq).size, quant_type)
 
 
 def f32_to_bf16(x: np.ndarray) -> np.ndarray:
@@ -217,7 +241,8 @@ def lora_delta(up_bf16: np.ndarray, down_bf16: np.ndarray) -> np.ndarray:
     return out
 
 
-def merge_lora(wq, absmax_q, absmax_scale, mu, n: int, k: int, down_bf16, up_bf16, scale: float):
+def merge_lora(wq, absmax_q, absmax_scale, mu, n: int, k: int, down_bf16, up_bf16, scale: float,
+               quant_type: str = "nf4"):
     """Merge a trained LoRA update into the quantized base and requantize it.
 
     Page "LLM 相關知識" (technicalnotes), section "8. LoRA 的合併（Merge）": INT4
@@ -225,14 +250,15 @@ def merge_lora(wq, absmax_q, absmax_scale, mu, n: int, k: int, down_bf16, up_bf1
     is quantized again to INT4 for deployment.  Reading: What_bf16 is the bf16
     dequantized weight; delta = up * down (fp32, rank order, lora_delta);
     W_new = bf16_round(fp32(What_bf16 + fp32(scale * delta))); the new codes and
-    fp32 absmax are the blockwise NF4 quantization of the bf16 W_new.
+    fp32 absmax are the blockwise quantization of the bf16 W_new (quant_type's
+    codebook, the same as the input's).
     Returns (w_new bf16 bits [n, k], wq_new uint8, absmax_new fp32)."""
-    what = f32_to_bf16(dequantize_range(wq, absmax_q, absmax_scale, mu, 0, n * k)).reshape(n, k)
+    what = f32_to_bf16(dequantize_range(wq, absmax_q, absmax_scale, mu, 0, n * k, quant_type)).reshape(n, k)
     d = lora_delta(up_bf16, down_bf16)
     sd = (np.float32(scale) * d).astype(np.float32)                 # fp32 multiply
     s = (bf16_to_f32(what) + sd).astype(np.float32)                  # fp32 add
     w_new = f32_to_bf16(s)
-    wq_new, absmax_new = quantize(w_new.reshape(-1))
+    wq_new, absmax_new = quantize(w_new.reshape(-1), quant_type)
     return w_new, wq_new, absmax_new
 
 

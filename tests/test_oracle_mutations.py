@@ -35,6 +35,10 @@ MUTANTS = [
     ("absmax from the signed maximum", "float a = fabsf(blk[j]);", "float a = blk[j];"),
     ("negative levels one short", "for (int i = 0; i < 7; ++i) v[k++] = -orc_norm_ppf",
      "for (int i = 1; i < 8; ++i) v[k++] = -orc_norm_ppf"),
+    ("FP4 exponent bias 0", "ldexp(1.0 + 0.5 * m, e - 1)", "ldexp(1.0 + 0.5 * m, e)"),
+    ("FP4 subnormals flushed", "(e == 0) ? 0.5 * m :", "(e == 0) ? 0.0 * m :"),
+    ("FP4 zero block mapped to -0", "if (qt == ORC_FP4) idx[j] = 0;", "if (qt == ORC_FP4) idx[j] = 8;"),
+    ("FP4 quantized with the NF4 levels", "const float* c = table_of(qt);", "const float* c = codebook();"),
 ]
 
 

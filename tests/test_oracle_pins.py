@@ -503,3 +503,134 @@ def test_merged_weight_matches_the_lora_layer_within_bf16_rounding():
     wa = np.abs(O.bf16_to_f32(w_new).astype(np.float64))
     bound = 2.0 ** -8 * (xa @ wa.T) + 1e-6
     assert np.all(np.abs(y_merged - y_layer) <= bound)
+
+
+# ---------------------------------------------------------------------------
+# FP4 codebook (xyzblog page, section 2.2 code walk: FP4 is the generic float
+# format builder with a sign bit, 2 exponent bits and 1 mantissa bit; zingnex
+# page, "4-bit 量化": FP4 is a conventional 4-bit float).  The same blockwise
+# pipeline with that table in place of the NF4 levels.
+# ---------------------------------------------------------------------------
+
+def _e2m1_decoded() -> np.ndarray:
+    """ml_dtypes' own decoding of the 16 bit patterns of its E2M1 type."""
+    import ml_dtypes
+    return np.arange(16, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+
+
+def test_fp4_codebook_is_the_scaled_e2m1_format():
+    v = _e2m1_decoded()
+    ref = (v / np.max(np.abs(v))).astype(np.float32)
+    c = O.codebook("fp4")
+    assert np.array_equal(c.view(np.uint32), ref.view(np.uint32))   # -0 at code 8 included
+    assert c[0] == 0 and not np.signbit(c[0]) and np.signbit(c[8])
+    assert c[7] == f32(1.0) and c[15] == f32(-1.0)
+    assert np.array_equal(c[8:], -c[:8])
+    assert np.all(np.diff(c[:8]) > 0)
+    # two values per binade after the subnormal pair, consecutive binades a factor 2 apart
+    assert c[3] == 3 * c[1] and c[5] == 2 * c[3] and c[7] == 2 * c[5] and c[2] == 2 * c[1]
+
+
+def test_fp4_quantize_is_exact_argmin_and_e2m1_rounding_off_ties():
+    import ml_dtypes
+    rng = np.random.default_rng(61)
+    c = O.codebook("fp4")
+    w = (rng.standard_normal(64 * 10) * 0.02).astype(np.float32)
+    w[64 * 2: 64 * 3] *= 1e-30                                     # tiny values
+    w[64 * 4: 64 * 5] = rng.integers(-6, 7, 64).astype(np.float32)   # exact grid points and ties
+    w[64 * 6 + 3] = -1e-9                                          # tiny negative next to larger values
+    # the one exact tie among the FP4 values: halfway between 0 and the smallest
+    # subnormal (the other midpoints are not fp32 values)
+    w[64 * 8: 64 * 9] = 0.0
+    w[64 * 8] = 1.0
+    w[64 * 8 + 1], w[64 * 8 + 2] = c[1] / 2, -c[1] / 2
+    wq, absmax = O.quantize(w, "fp4")
+    idx = O.unpack(wq)
+    ties = 0
+    for b in range(10):
+        blk = w[b * 64:(b + 1) * 64]
+        am = np.max(np.abs(blk))
+        assert absmax[b] == am
+        for j in range(64):
+            x = f32(blk[j]) / f32(am)
+            code = idx[b * 64 + j]
+            assert code == _exact_argmin(x, c), (b, j, blk[j], am)
+            assert code != 8, "the -0 code is never produced"
+            # off a tie, the value is E2M1 round-to-nearest of 6x scaled back
+            fx = Fraction(float(x))
+            d = sorted(abs(fx - Fraction(float(ci))) for ci in set(c.tolist()))
+            if d[0] == d[1]:
+                ties += 1
+                continue
+            e = float(np.array([6.0 * float(x)]).astype(ml_dtypes.float4_e2m1fn).astype(np.float64)[0])
+            assert c[code] == f32(e / 6.0), (x, code, e)
+    assert ties > 0
+
+
+def test_fp4_midpoints_tie_toward_zero_and_zero_blocks():
+    c = O.codebook("fp4")
+    mags = c[:8]
+    vals = []
+    for j in range(7):
+        mid = (Fraction(float(mags[j])) + Fraction(float(mags[j + 1]))) / 2
+        m32 = f32(float(mid))
+        for v in (np.nextafter(m32, f32(-2)), m32, np.nextafter(m32, f32(2))):
+            vals += [v, -v]
+    vals = np.array(vals, dtype=np.float32)
+    pad = (-(len(vals) + 1)) % 64
+    w = np.concatenate([[f32(1.0)], vals, np.zeros(pad, np.float32)]).astype(np.float32)
+    w = np.concatenate([w, np.zeros(64, np.float32)])              # a zero block
+    w[-5] = -0.0
+    wq, absmax = O.quantize(w, "fp4")
+    idx = O.unpack(wq)
+    for i, v in enumerate(w):
+        assert idx[i] == _exact_argmin(v, c), (i, v)
+    for j in range(7):
+        mid = (Fraction(float(mags[j])) + Fraction(float(mags[j + 1]))) / 2
+        if Fraction(float(f32(float(mid)))) == mid:                # an exact tie
+            pos = 1 + 6 * j + 2
+            assert idx[pos] == j and idx[pos + 1] == (8 + j if j > 0 else 0)
+    assert absmax[-1] == 0.0 and np.all(idx[-64:] == 0)
+
+
+def test_fp4_dequantize_error_bound_and_end_levels():
+    rng = np.random.default_rng(62)
+    n, k = 16, 1024
+    w = (rng.standard_normal((n, k)) * 0.02).astype(np.float32)
+    wq, absmax = O.quantize(w, "fp4")
+    q, s, mu = O.double_quant(absmax)
+    wh = O.dequantize(wq, q, s, mu, "fp4").reshape(n, k)
+    c = O.codebook("fp4").astype(np.float64)
+    half_gap = np.max(np.diff(np.sort(c))) / 2                     # (1 - 2/3) / 2
+    assert abs(half_gap - 1.0 / 6.0) < 1e-7
+    ahat = O.absmax_hat(q, s, mu).astype(np.float64)
+    wb = w.reshape(-1, 64).astype(np.float64)
+    whb = wh.reshape(-1, 64).astype(np.float64)
+    idx = O.unpack(wq).reshape(-1, 64)
+    for b in range(wb.shape[0]):
+        bound = half_gap * absmax[b] + abs(ahat[b] - absmax[b]) + 1e-6 * absmax[b]
+        assert np.all(np.abs(whb[b] - wb[b]) <= bound)
+        j = int(np.argmax(np.abs(wb[b])))
+        assert idx[b, j] == (7 if wb[b, j] > 0 else 15)
+        assert whb[b, j] == np.sign(wb[b, j]) * f32(ahat[b])
+    # the NF4 table gives a different (smaller) error on normal weights
+    wq_n, am_n = O.quantize(w)
+    qn, sn, mun = O.double_quant(am_n)
+    err_n = np.mean((O.dequantize(wq_n, qn, sn, mun).reshape(n, k) - w) ** 2)
+    err_f = np.mean((wh - w) ** 2)
+    assert err_n < err_f
+
+
+def test_fp4_merge_zero_scale_is_the_bf16_dequant():
+    rng = np.random.default_rng(63)
+    n, k, r = 8, 128, 4
+    W = rng.standard_normal((n, k)).astype(np.float32) * 0.02
+    wq, am = O.quantize(W, "fp4")
+    q, s, mu = O.double_quant(am)
+    D = _bf16_bits(rng.standard_normal((r, k)))
+    U = _bf16_bits(rng.standard_normal((n, r)))
+    w_new, wq2, am2 = O.merge_lora(wq, q, s, mu, n, k, D, U, 0.0, "fp4")
+    what = O.f32_to_bf16(O.dequantize(wq, q, s, mu, "fp4")).reshape(n, k)
+    assert np.array_equal(w_new, what)
+    wq3, am3 = O.quantize(what.reshape(-1), "fp4")
+    assert np.array_equal(wq2, wq3) and np.array_equal(am2.view(np.uint32), am3.view(np.uint32))
