@@ -448,9 +448,9 @@ def run_ours(args, rank, world, local):
             ul = (synth.activations(wl.n, rl, seed=synth.seed_for(3, 10), device=dev).float() * 0.02).to(torch.bfloat16)
             wsl = nf4.lora_workspace(ml, [(wl.n, wl.k)], rl, device=dev)
             wsp = nf4.linear_workspace([(wl.n, wl.k)], m=ml, device=dev)
-            early = ml <= 16   # the decode path runs with programmatic dependent launch
-            f_l = lambda: nf4.nf4_linear_lora(Xl, wl, dl, ul, 2.0, wsl, out=Yl, weights_early=early)
-            f_p = lambda: nf4.nf4_linear(Xl, wl, torch.bfloat16, out=Yl, workspace=wsp, weights_early=early)
+            early_l = ml <= 16   # the decode path runs with programmatic dependent launch
+            f_l = lambda: nf4.nf4_linear_lora(Xl, wl, dl, ul, 2.0, wsl, out=Yl, weights_early=early_l)
+            f_p = lambda: nf4.nf4_linear(Xl, wl, torch.bfloat16, out=Yl, workspace=wsp, weights_early=early_l)
             f_l(); f_p()
             t_l = _events_time(f_l, 20, stream)
             t_p = _events_time(f_p, 20, stream)
@@ -458,7 +458,32 @@ def run_ours(args, rank, world, local):
                          "overhead": round(t_l / t_p - 1.0, 4)}
             del Xl, Yl, dl, ul, wsl, wsp
         gemm["lora"] = lora
-        del Xg, Yg, wg
+        # the FP4 codebook on the same kernels and the same 11008 x 4096 weight:
+        # GEMM at m = 4096 and the decode GEMV at m = 16, NF4 timed alongside
+        Wf = synth.weight_normal(11008, 4096, seed=synth.seed_for(3, 0), dtype=torch.bfloat16, device=dev)
+        wf = nf4.quantize_weight(Wf, quant_type="fp4")
+        del Wf
+        fp4 = {}
+        f_f = lambda: nf4.nf4_linear(Xg, wf, torch.bfloat16, out=Yg)
+        f_f()
+        fp4["gemm_tflops_m4096"] = round(2.0 * 4096 * 4096 * 11008 / _events_time(f_f, 3, stream) / 1e12, 1)
+        X16 = synth.activations(16, 4096, seed=synth.seed_for(3, 11), device=dev)
+        Y16 = torch.empty((16, 11008), dtype=torch.bfloat16, device=dev)
+        ws16 = nf4.linear_workspace([(11008, 4096)], m=16, device=dev)
+        # eight copies of each weight per timed rep (190 MB > L2), so every launch reads HBM
+        for tag, wt in (("fp4", wf), ("nf4", wg)):
+            copies = [nf4.NF4Weight(wt.n, wt.k, wt.wq.clone(), wt.absmax_q.clone(), wt.absmax_scale.clone(),
+                                    wt.absmax_offset.clone(), wt.quant_type) for _ in range(8)]
+
+            def f_v():
+                for wc in copies:
+                    nf4.nf4_linear(X16, wc, torch.bfloat16, out=Y16, workspace=ws16)
+            f_v()
+            t_v = _events_time(f_v, 10, stream) / len(copies)
+            fp4["gemv_gbs_m16_" + tag] = round(linear_bytes(11008, 4096, 16, 2) / t_v / 1e9, 1)
+            del copies
+        gemm["fp4"] = fp4
+        del Xg, Yg, wg, wf, X16, Y16, ws16
 
     # 70B-shaped stress layer: 28672 x 8192 Student-t(4) weight with outlier input
     # columns, as GEMV (m = 1, 16) and GEMM (m = 512, 4096)

@@ -61,8 +61,19 @@ typedef enum nf4_dtype {
 #define NF4_ABI_VERSION 1
 #define NF4_BLOCKSIZE 64          /* weights per absmax ([P5] §2.2 example: "split by 64") */
 #define NF4_BLOCKSIZE2 256        /* absmax values per double-quantization block */
-#define NF4_WEIGHT_MAGIC 0x4E463442u /* "NF4B" */
+#define NF4_WEIGHT_MAGIC 0x4E463442u /* "NF4B": codes index the NF4 levels */
+#define NF4_FP4_WEIGHT_MAGIC 0x46503442u /* "FP4B": codes index the FP4 values (same layout) */
 #define NF4_WEIGHT_VERSION 1u
+
+/* The 4-bit codebook of a quantization ([P5] §2.2 code walk: quant_type "nf4"
+ * or "fp4"; FP4 is the generic float format with a sign bit, 2 exponent bits
+ * and 1 mantissa bit, [P3] "4-bit 量化"). */
+typedef enum nf4_quant_type {
+    NF4_QUANT_NF4 = 0,  /* the 16 NF4 levels, ascending, exact zero at code 7 */
+    NF4_QUANT_FP4 = 1   /* the 16 FP4 values in code order: code = s|e1 e0|m, exponent
+                           bias 1, subnormal at e = 0, magnitudes 0, 0.5, 1, 1.5, 2, 3,
+                           4, 6 divided by 6; code 8 is -0 */
+} nf4_quant_type_t;
 
 /*
  * A quantized weight W[n, k] (out_features n, in_features k) as produced by
@@ -77,7 +88,7 @@ typedef enum nf4_dtype {
  *   absmax_offset fp32   [1]          the mean subtracted before double quantization
  */
 typedef struct nf4_weight {
-    uint32_t magic;       /* NF4_WEIGHT_MAGIC */
+    uint32_t magic;       /* NF4_WEIGHT_MAGIC, or NF4_FP4_WEIGHT_MAGIC for FP4 codes */
     uint32_t version;     /* NF4_WEIGHT_VERSION */
     int64_t n;            /* rows (out_features) */
     int64_t k;            /* columns (in_features) */
@@ -101,6 +112,11 @@ const char* nf4_status_str(int status);
  * NF4_ERR_NULL.  Host-only; launches nothing. */
 nf4_status_t nf4_codebook(float* levels_out);
 
+/* The 16 values of either codebook (NF4 ascending, FP4 in code order) copied to
+ * host memory `levels_out[16]`.  Returns NF4_OK, NF4_ERR_NULL or NF4_ERR_DTYPE
+ * (unknown quant_type).  Host-only. */
+nf4_status_t nf4_codebook_typed(nf4_quant_type_t quant_type, float* levels_out);
+
 /*
  * nf4_quantize -- blockwise NF4 quantization ([P5] §2.2 worked example and
  * Figure 2-2 steps 1-4; [P1] "NF4 不是一般四位元浮點格式").
@@ -118,6 +134,19 @@ nf4_status_t nf4_codebook(float* levels_out);
  */
 nf4_status_t nf4_quantize(const void* W, nf4_dtype_t w_dtype, int64_t n, int64_t k,
                           uint8_t* wq, float* absmax, nf4_stream_t stream);
+
+/*
+ * nf4_quantize_typed -- nf4_quantize with either codebook.  NF4_QUANT_NF4 is
+ * nf4_quantize.  NF4_QUANT_FP4 runs the same pipeline with the FP4 values:
+ * code = the nearest FP4 value to x_j, ties to the lower code (toward zero),
+ * so that every x_j nearest to zero, of either sign, is code 0 (+0) and code 8
+ * is never written; a zero block is code 0.  Describe the result with
+ * magic = NF4_FP4_WEIGHT_MAGIC; every other entry point then decodes it with
+ * the FP4 values.  Errors: as nf4_quantize; NF4_ERR_DTYPE also for an unknown
+ * quant_type.
+ */
+nf4_status_t nf4_quantize_typed(const void* W, nf4_dtype_t w_dtype, int64_t n, int64_t k,
+                                nf4_quant_type_t quant_type, uint8_t* wq, float* absmax, nf4_stream_t stream);
 
 /* Bytes of workspace nf4_double_quant needs for nb absmax values (0 if nb <= 0). */
 size_t nf4_double_quant_workspace_bytes(int64_t nb);

@@ -18,7 +18,9 @@ calls.  Functions carry the C names:
   trained update folded into the weight and quantized again (``merge_lora``
   adds the double quantization and returns an ``NF4Weight``)
 
-``quantize_weight(W)`` runs the first two and returns an ``NF4Weight``.
+``quantize_weight(W)`` runs the first two and returns an ``NF4Weight``.  Every
+quantizing call takes ``quant_type="nf4"`` (the default) or ``"fp4"``; an
+``NF4Weight`` remembers which codebook its codes index.
 """
 from __future__ import annotations
 
@@ -37,6 +39,13 @@ __all__ = ["NF4Weight", "NF4Error", "nf4_quantize", "nf4_double_quant", "nf4_deq
            "quantize_weight", "nf4_codebook", "library_path"]
 
 _DTYPES = {torch.float32: NF4_F32, torch.bfloat16: NF4_BF16}
+_QUANT_TYPES = {"nf4": _lib.NF4_QUANT_NF4, "fp4": _lib.NF4_QUANT_FP4}
+
+
+def _quant_type(quant_type: str) -> int:
+    if quant_type not in _QUANT_TYPES:
+        raise ValueError("quant_type must be 'nf4' or 'fp4'")
+    return _QUANT_TYPES[quant_type]
 
 
 def library_path() -> str:
@@ -59,16 +68,17 @@ def _need_cuda(t: torch.Tensor, name: str) -> None:
         raise ValueError("%s must be contiguous" % name)
 
 
-def nf4_codebook() -> torch.Tensor:
-    """The 16 levels the library uses (host copy)."""
+def nf4_codebook(quant_type: str = "nf4") -> torch.Tensor:
+    """The 16 levels the library uses (host copy): NF4 ascending, FP4 in code order."""
     out = torch.zeros(16, dtype=torch.float32)
-    _lib.check(_lib.lib().nf4_codebook(_ptr(out)), "nf4_codebook")
+    _lib.check(_lib.lib().nf4_codebook_typed(_quant_type(quant_type), _ptr(out)), "nf4_codebook")
     return out
 
 
 def nf4_quantize(W: torch.Tensor, wq: torch.Tensor | None = None, absmax: torch.Tensor | None = None,
-                 stream=None):
-    """Blockwise NF4 quantization of a 2-D fp32/bf16 CUDA tensor [n, k]."""
+                 stream=None, quant_type: str = "nf4"):
+    """Blockwise NF4 (or FP4) quantization of a 2-D fp32/bf16 CUDA tensor [n, k]."""
+    qt = _quant_type(quant_type)
     _need_cuda(W, "W")
     if W.dim() != 2 or W.dtype not in _DTYPES:
         raise ValueError("W must be a 2-D float32 or bfloat16 tensor")
@@ -78,8 +88,8 @@ def nf4_quantize(W: torch.Tensor, wq: torch.Tensor | None = None, absmax: torch.
         wq = torch.empty(numel // 2, dtype=torch.uint8, device=W.device)
     if absmax is None:
         absmax = torch.empty(numel // 64, dtype=torch.float32, device=W.device)
-    _lib.check(_lib.lib().nf4_quantize(_ptr(W), _DTYPES[W.dtype], n, k, _ptr(wq), _ptr(absmax),
-                                       _stream(stream)), "nf4_quantize")
+    _lib.check(_lib.lib().nf4_quantize_typed(_ptr(W), _DTYPES[W.dtype], n, k, qt, _ptr(wq), _ptr(absmax),
+                                             _stream(stream)), "nf4_quantize")
     return wq, absmax
 
 
@@ -116,9 +126,11 @@ class NF4Weight:
     absmax_q: torch.Tensor
     absmax_scale: torch.Tensor
     absmax_offset: torch.Tensor
+    quant_type: str = "nf4"
 
     def struct(self) -> nf4_weight_t:
-        return nf4_weight_t(_lib.NF4_WEIGHT_MAGIC, _lib.NF4_WEIGHT_VERSION, self.n, self.k,
+        magic = _lib.NF4_FP4_WEIGHT_MAGIC if self.quant_type == "fp4" else _lib.NF4_WEIGHT_MAGIC
+        return nf4_weight_t(magic, _lib.NF4_WEIGHT_VERSION, self.n, self.k,
                             _lib.NF4_BLOCKSIZE, _lib.NF4_BLOCKSIZE2, self.wq.data_ptr(),
                             self.absmax_q.data_ptr(), self.absmax_scale.data_ptr(),
                             self.absmax_offset.data_ptr())
@@ -127,11 +139,11 @@ class NF4Weight:
         return (self.wq.numel() + self.absmax_q.numel() + 4 * self.absmax_scale.numel())
 
 
-def quantize_weight(W: torch.Tensor, stream=None) -> NF4Weight:
+def quantize_weight(W: torch.Tensor, stream=None, quant_type: str = "nf4") -> NF4Weight:
     """nf4_quantize followed by nf4_double_quant; the fp32 absmax is dropped."""
-    wq, absmax = nf4_quantize(W, stream=stream)
+    wq, absmax = nf4_quantize(W, stream=stream, quant_type=quant_type)
     q, s, mu = nf4_double_quant(absmax, stream=stream)
-    return NF4Weight(W.shape[0], W.shape[1], wq, q, s, mu)
+    return NF4Weight(W.shape[0], W.shape[1], wq, q, s, mu, quant_type)
 
 
 def nf4_dequantize(weight: NF4Weight, dtype=torch.bfloat16, out: torch.Tensor | None = None,
@@ -284,4 +296,4 @@ def merge_lora(weight: NF4Weight, down: torch.Tensor, up: torch.Tensor, scale: f
     """nf4_merge_lora followed by nf4_double_quant: the merged, requantized weight."""
     wq, absmax, _ = nf4_merge_lora(weight, down, up, scale, stream=stream)
     q, s, mu = nf4_double_quant(absmax, stream=stream)
-    return NF4Weight(weight.n, weight.k, wq, q, s, mu)
+    return NF4Weight(weight.n, weight.k, wq, q, s, mu, weight.quant_type)

@@ -17,6 +17,9 @@ NF4_BF16 = 1
 NF4_BLOCKSIZE = 64
 NF4_BLOCKSIZE2 = 256
 NF4_WEIGHT_MAGIC = 0x4E463442
+NF4_FP4_WEIGHT_MAGIC = 0x46503442
+NF4_QUANT_NF4 = 0
+NF4_QUANT_FP4 = 1
 NF4_WEIGHT_VERSION = 1
 NF4_ABI_VERSION = 1
 NF4_DQ_NOALLOC_MAX_NB = 16777216
@@ -39,6 +42,8 @@ SIGNATURES = {
     "nf4_abi_version": (ctypes.c_int, []),
     "nf4_status_str": (ctypes.c_char_p, [ctypes.c_int]),
     "nf4_codebook": (ctypes.c_int, [_p]),
+    "nf4_codebook_typed": (ctypes.c_int, [ctypes.c_int, _p]),
+    "nf4_quantize_typed": (ctypes.c_int, [_p, ctypes.c_int, _i64, _i64, ctypes.c_int, _p, _p, _p]),
     "nf4_quantize": (ctypes.c_int, [_p, ctypes.c_int, _i64, _i64, _p, _p, _p]),
     "nf4_double_quant_workspace_bytes": (ctypes.c_size_t, [_i64]),
     "nf4_double_quant": (ctypes.c_int, [_p, _i64, _p, ctypes.c_size_t, _p, _p, _p, _p]),

@@ -56,7 +56,7 @@ nf4_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? NF4_OK : NF4_E
 
 nf4_status_t check_weight(const nf4_weight_t* w) {
     if (!w) return NF4_ERR_NULL;
-    if (w->magic != NF4_WEIGHT_MAGIC || w->version != NF4_WEIGHT_VERSION ||
+    if ((w->magic != NF4_WEIGHT_MAGIC && w->magic != NF4_FP4_WEIGHT_MAGIC) || w->version != NF4_WEIGHT_VERSION ||
         w->blocksize != NF4_BLOCKSIZE || w->blocksize2 != NF4_BLOCKSIZE2)
         return NF4_ERR_STATE;
     if (!w->wq || !w->absmax_q || !w->absmax_scale || !w->absmax_offset) return NF4_ERR_NULL;
@@ -67,6 +67,9 @@ nf4_status_t check_weight(const nf4_weight_t* w) {
         return NF4_ERR_ALIGN;
     return NF4_OK;
 }
+
+// The codebook a (checked) weight's codes index: its magic says NF4 or FP4.
+int codebook_of(const nf4_weight_t* w) { return w->magic == NF4_FP4_WEIGHT_MAGIC ? 1 : 0; }
 
 }  // namespace
 
@@ -90,23 +93,38 @@ const char* nf4_status_str(int status) {
     }
 }
 
-nf4_status_t nf4_codebook(float* levels_out) {
+nf4_status_t nf4_codebook(float* levels_out) { return nf4_codebook_typed(NF4_QUANT_NF4, levels_out); }
+
+nf4_status_t nf4_codebook_typed(nf4_quant_type_t quant_type, float* levels_out) {
     if (!levels_out) return NF4_ERR_NULL;
-    static const float levels[16] = NF4_LEVELS_INIT;
-    std::memcpy(levels_out, levels, sizeof levels);
+    static const float nf4_levels[16] = NF4_LEVELS_INIT;
+    static const float fp4_levels[16] = FP4_LEVELS_INIT;
+    if (quant_type == NF4_QUANT_NF4)
+        std::memcpy(levels_out, nf4_levels, sizeof nf4_levels);
+    else if (quant_type == NF4_QUANT_FP4)
+        std::memcpy(levels_out, fp4_levels, sizeof fp4_levels);
+    else
+        return NF4_ERR_DTYPE;
     return NF4_OK;
 }
 
 nf4_status_t nf4_quantize(const void* W, nf4_dtype_t w_dtype, int64_t n, int64_t k, uint8_t* wq,
                           float* absmax, nf4_stream_t stream) {
+    return nf4_quantize_typed(W, w_dtype, n, k, NF4_QUANT_NF4, wq, absmax, stream);
+}
+
+nf4_status_t nf4_quantize_typed(const void* W, nf4_dtype_t w_dtype, int64_t n, int64_t k,
+                                nf4_quant_type_t quant_type, uint8_t* wq, float* absmax, nf4_stream_t stream) {
     if (!W || !wq || !absmax) return NF4_ERR_NULL;
+    if (quant_type != NF4_QUANT_NF4 && quant_type != NF4_QUANT_FP4) return NF4_ERR_DTYPE;
     if (w_dtype != NF4_F32 && w_dtype != NF4_BF16) return NF4_ERR_DTYPE;
     if (n <= 0 || k <= 0 || n > INT64_MAX / k || (n * k) % NF4_BLOCKSIZE != 0) return NF4_ERR_SHAPE;
     if (!aligned(W, 16) || !aligned(wq, 16) || !aligned(absmax, 4)) return NF4_ERR_ALIGN;
     nf4::DeviceInfo dev;
     nf4_status_t st = device_ok(&dev);
     if (st != NF4_OK) return st;
-    return from_cuda(nf4::launch_quantize(W, w_dtype == NF4_BF16, n * k, wq, absmax, dev,
+    return from_cuda(nf4::launch_quantize(W, w_dtype == NF4_BF16, n * k, wq, absmax,
+                                          quant_type == NF4_QUANT_FP4 ? 1 : 0, dev,
                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -139,7 +157,7 @@ nf4_status_t nf4_dequantize(const nf4_weight_t* w, void* out, nf4_dtype_t out_dt
     nf4::DeviceInfo dev;
     if ((st = device_ok(&dev)) != NF4_OK) return st;
     return from_cuda(nf4::launch_dequantize(w->wq, w->absmax_q, w->absmax_scale, w->absmax_offset,
-                                            w->n * w->k, out, out_dtype == NF4_BF16, dev,
+                                            w->n * w->k, out, out_dtype == NF4_BF16, codebook_of(w), dev,
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -184,7 +202,7 @@ nf4_status_t nf4_linear_lora(const void* X, int64_t m, const nf4_weight_t* w, co
     lora.t_lo = t_lo;
     return from_cuda(nf4::launch_linear(X, m, w->wq, w->absmax_q, w->absmax_scale, w->absmax_offset, w->n, w->k,
                                         Y, y_dtype == NF4_BF16, dev_status, (flags & NF4_LINEAR_WEIGHTS_EARLY) != 0,
-                                        static_cast<char*>(workspace) + tb, lora, dev, s));
+                                        static_cast<char*>(workspace) + tb, lora, codebook_of(w), dev, s));
 }
 
 nf4_status_t nf4_merge_lora(const nf4_weight_t* w, const void* lora_down, const void* lora_up, int32_t r,
@@ -200,7 +218,8 @@ nf4_status_t nf4_merge_lora(const nf4_weight_t* w, const void* lora_down, const 
     nf4::DeviceInfo dev;
     if ((st = device_ok(&dev)) != NF4_OK) return st;
     return from_cuda(nf4::launch_merge_lora(w->wq, w->absmax_q, w->absmax_scale, w->absmax_offset, w->n, w->k,
-                                            lora_down, lora_up, r, scale, w_new, wq_out, absmax_out, dev,
+                                            lora_down, lora_up, r, scale, w_new, wq_out, absmax_out,
+                                            codebook_of(w), dev,
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -229,7 +248,8 @@ nf4_status_t nf4_linear_ws(const void* X, int64_t m, const nf4_weight_t* w, void
     if (workspace && ws_bytes < nf4::linear_workspace_bytes(m, w->n, w->k, dev)) return NF4_ERR_WORKSPACE;
     return from_cuda(nf4::launch_linear(X, m, w->wq, w->absmax_q, w->absmax_scale, w->absmax_offset,
                                         w->n, w->k, Y, y_dtype == NF4_BF16, dev_status,
-                                        (flags & NF4_LINEAR_WEIGHTS_EARLY) != 0, workspace, nf4::LoraArgs(), dev,
+                                        (flags & NF4_LINEAR_WEIGHTS_EARLY) != 0, workspace, nf4::LoraArgs(),
+                                        codebook_of(w), dev,
                                         reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -250,7 +270,7 @@ nf4_status_t nf4_linear_dx(const void* dY, int64_t m, const nf4_weight_t* w, voi
     nf4::DeviceInfo dev;
     if ((st = device_ok(&dev)) != NF4_OK) return st;
     return from_cuda(nf4::launch_gemm_dx(dY, m, w->wq, w->absmax_q, w->absmax_scale, w->absmax_offset, w->n,
-                                         w->k, dX, dx_dtype == NF4_BF16, dev_status, dev,
+                                         w->k, dX, dx_dtype == NF4_BF16, dev_status, codebook_of(w), dev,
                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 

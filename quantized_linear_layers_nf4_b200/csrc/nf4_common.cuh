@@ -26,6 +26,14 @@ constexpr unsigned kFull = 0xffffffffu;
 static __constant__ float kLevels[16] = NF4_LEVELS_INIT;
 static __constant__ float kThresh[15] = NF4_THRESHOLDS_INIT;
 
+// Codebook ids: the weight's 4-bit codes index the NF4 levels or the FP4 values
+// ([P5] §2.2 code walk: quant_type "nf4" or "fp4", the latter the generic float
+// format with a sign, 2 exponent bits and 1 mantissa bit).  Same storage, same
+// pipeline; only the table and the encoder differ.
+constexpr int kCbNf4 = 0;
+constexpr int kCbFp4 = 1;
+static __constant__ float kCodebook[2][16] = {NF4_LEVELS_INIT, FP4_LEVELS_INIT};
+
 // Thresholds as compile-time values, so that the encoder's comparisons use
 // immediates and never index memory per element.
 struct Thr {
@@ -56,6 +64,38 @@ __device__ __forceinline__ int encode_nf4(float x) {
 __device__ __forceinline__ int quantize_one(float w, float a) {
     if (a == 0.0f) return 7;
     return encode_nf4(__fdiv_rn(w, a));
+}
+
+struct Fp4Thr {
+    static constexpr float t[7] = FP4_THRESHOLDS_INIT;
+};
+
+// FP4 code of x in [-1, 1]: the magnitude index #{j : |x| > u_j} over the 7
+// round-down midpoints of the magnitudes (three-step binary search), with the
+// sign bit set for negative x, except that a zero magnitude is always code 0
+// (+0).  This is the nearest FP4 value with ties going to the lower code (toward
+// zero); code 8 (-0) is never produced.
+__device__ __forceinline__ int encode_fp4(float x) {
+    constexpr float U0 = Fp4Thr::t[0], U1 = Fp4Thr::t[1], U2 = Fp4Thr::t[2], U3 = Fp4Thr::t[3];
+    constexpr float U4 = Fp4Thr::t[4], U5 = Fp4Thr::t[5], U6 = Fp4Thr::t[6];
+    const float a = fabsf(x);
+    const bool b2 = a > U3;
+    const bool b1 = a > (b2 ? U5 : U1);
+    const float u0 = b2 ? (b1 ? U6 : U4) : (b1 ? U2 : U0);
+    const bool b0 = a > u0;
+    const int mag = (b2 ? 4 : 0) | (b1 ? 2 : 0) | (b0 ? 1 : 0);
+    return (mag != 0 && x < 0.0f) ? (8 | mag) : mag;
+}
+
+// Code of weight w in a block with absmax a under codebook CB; a zero block is
+// the exact-zero code (NF4 7, FP4 0).
+template <int CB>
+__device__ __forceinline__ int quantize_code(float w, float a) {
+    if (CB == kCbFp4) {
+        if (a == 0.0f) return 0;
+        return encode_fp4(__fdiv_rn(w, a));
+    }
+    return quantize_one(w, a);
 }
 
 // fp32(q / 127), the correctly rounded quotient, for an int8 code q, without a

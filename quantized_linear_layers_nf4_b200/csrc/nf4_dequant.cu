@@ -19,9 +19,10 @@ __global__ void __launch_bounds__(256) k_nf4_dequantize(const uint32_t* __restri
                                                         const int8_t* __restrict__ absmax_q,
                                                         const float* __restrict__ absmax_scale,
                                                         const float* __restrict__ mu_ptr,
-                                                        int64_t n_groups, void* __restrict__ out) {
+                                                        int64_t n_groups, void* __restrict__ out,
+                                                        int codebook) {
     __shared__ float lv[16];
-    if (threadIdx.x < 16) lv[threadIdx.x] = kLevels[threadIdx.x];
+    if (threadIdx.x < 16) lv[threadIdx.x] = kCodebook[codebook][threadIdx.x];
     __syncthreads();
     const float mu = __ldg(mu_ptr);
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -53,7 +54,7 @@ __global__ void __launch_bounds__(256) k_nf4_dequantize(const uint32_t* __restri
 }
 
 cudaError_t launch_dequantize(const uint8_t* wq, const int8_t* absmax_q, const float* absmax_scale,
-                              const float* absmax_offset, int64_t n_elem, void* out, bool out_bf16,
+                              const float* absmax_offset, int64_t n_elem, void* out, bool out_bf16, int codebook,
                               const DeviceInfo& dev, cudaStream_t stream) {
     const int64_t n_groups = n_elem / 8;
     int64_t blocks = (n_groups + 255) / 256;
@@ -63,10 +64,10 @@ cudaError_t launch_dequantize(const uint8_t* wq, const int8_t* absmax_q, const f
     const uint32_t* wq32 = reinterpret_cast<const uint32_t*>(wq);
     if (out_bf16)
         k_nf4_dequantize<true><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-            wq32, absmax_q, absmax_scale, absmax_offset, n_groups, out);
+            wq32, absmax_q, absmax_scale, absmax_offset, n_groups, out, codebook);
     else
         k_nf4_dequantize<false><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-            wq32, absmax_q, absmax_scale, absmax_offset, n_groups, out);
+            wq32, absmax_q, absmax_scale, absmax_offset, n_groups, out, codebook);
     return cudaGetLastError();
 }
 

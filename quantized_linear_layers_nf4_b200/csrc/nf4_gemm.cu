@@ -144,7 +144,7 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
            int32_t* __restrict__ dev_status, const float* __restrict__ lora_t,
            const __nv_bfloat16* __restrict__ lora_up, int lora_r, int lora_tc,
            const __grid_constant__ CUtensorMap tm_thi, const __grid_constant__ CUtensorMap tm_tlo,
-           const __grid_constant__ CUtensorMap tm_up) {
+           const __grid_constant__ CUtensorMap tm_up, int codebook) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -296,7 +296,7 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         const float mu = __ldg(mu_ptr);
         uint64_t cpair[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) cpair[j] = pack_f32x2(kLevels[2 * j], kLevels[2 * j + 1]);
+        for (int j = 0; j < 8; ++j) cpair[j] = pack_f32x2(kCodebook[codebook][2 * j], kCodebook[codebook][2 * j + 1]);
         const uint32_t prow = sbase + kOffP + t * 32;
         const uint32_t brow = sbase + kOffB + t * 128;
         const uint32_t swz = static_cast<uint32_t>(t & 7);
@@ -478,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_nf4_gemm_dx(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_w,
               const int8_t* __restrict__ absmax_q, const float* __restrict__ absmax_scale,
               const float* __restrict__ mu_ptr, int64_t m, int64_t n, int64_t k, void* __restrict__ dX,
-              int32_t* __restrict__ dev_status) {
+              int32_t* __restrict__ dev_status, int codebook) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -597,7 +597,7 @@ k_nf4_gemm_dx(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
         const float mu = __ldg(mu_ptr);
         uint64_t cpair[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) cpair[j] = pack_f32x2(kLevels[2 * j], kLevels[2 * j + 1]);
+        for (int j = 0; j < 8; ++j) cpair[j] = pack_f32x2(kCodebook[codebook][2 * j], kCodebook[codebook][2 * j + 1]);
         const uint32_t swz = static_cast<uint32_t>(r & 7);
         const uint32_t prow = sbase + kOffP + r * 128;
         const uint32_t brow = sbase + kOffB + cb * (kBKX * 128) + r * 128;
@@ -697,8 +697,8 @@ k_nf4_gemm_dx(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
 
 cudaError_t launch_gemm(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                         const float* absmax_scale, const float* absmax_offset, int64_t n, int64_t k, void* Y,
-                        bool y_bf16, int32_t* dev_status, const LoraArgs& lora, const DeviceInfo& dev,
-                        cudaStream_t stream) {
+                        bool y_bf16, int32_t* dev_status, const LoraArgs& lora, int codebook,
+                        const DeviceInfo& dev, cudaStream_t stream) {
     static bool attr_set[64][4] = {};
     if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
     const bool lo = lora.t != nullptr;
@@ -741,7 +741,7 @@ cudaError_t launch_gemm(const void* X, int64_t m, const uint8_t* wq, const int8_
 #define NF4_GEMM_LAUNCH(B, L)                                                                               \
     gemm::k_nf4_gemm<B, L><<<grid, gemm::kThreads, gemm::kSmemBytes, stream>>>(                              \
         tm_x, tm_w, absmax_q, absmax_scale, absmax_offset, m, n, k, Y, dev_status, lora.t, lora.up, lora.r,  \
-        lora_tc, tm_thi, tm_tlo, tm_up)
+        lora_tc, tm_thi, tm_tlo, tm_up, codebook)
     if (y_bf16) {
         if (lo) NF4_GEMM_LAUNCH(true, true); else NF4_GEMM_LAUNCH(true, false);
     } else {
@@ -753,7 +753,8 @@ cudaError_t launch_gemm(const void* X, int64_t m, const uint8_t* wq, const int8_
 
 cudaError_t launch_gemm_dx(const void* dY, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                            const float* absmax_scale, const float* absmax_offset, int64_t n, int64_t k, void* dX,
-                           bool dx_bf16, int32_t* dev_status, const DeviceInfo& dev, cudaStream_t stream) {
+                           bool dx_bf16, int32_t* dev_status, int codebook, const DeviceInfo& dev,
+                           cudaStream_t stream) {
     static bool attr_set[64][2] = {};
     if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
     const void* fn = dx_bf16 ? reinterpret_cast<const void*>(&gemm::k_nf4_gemm_dx<true>)
@@ -777,10 +778,10 @@ cudaError_t launch_gemm_dx(const void* dY, int64_t m, const uint8_t* wq, const i
                     static_cast<unsigned>((m + gemm::kBM - 1) / gemm::kBM));
     if (dx_bf16)
         gemm::k_nf4_gemm_dx<true><<<grid, gemm::kThreads, gemm::kSmemBytes, stream>>>(
-            tm_dy, tm_w, absmax_q, absmax_scale, absmax_offset, m, n, k, dX, dev_status);
+            tm_dy, tm_w, absmax_q, absmax_scale, absmax_offset, m, n, k, dX, dev_status, codebook);
     else
         gemm::k_nf4_gemm_dx<false><<<grid, gemm::kThreads, gemm::kSmemBytes, stream>>>(
-            tm_dy, tm_w, absmax_q, absmax_scale, absmax_offset, m, n, k, dX, dev_status);
+            tm_dy, tm_w, absmax_q, absmax_scale, absmax_offset, m, n, k, dX, dev_status, codebook);
     return cudaGetLastError();
 }
 

@@ -220,7 +220,7 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
            const float* __restrict__ mu_ptr, int m, int64_t n, int64_t k, int cluster, int weights_early,
            void* __restrict__ Y, int32_t* __restrict__ dev_status, uint32_t* __restrict__ ws_cnt,
            float4* __restrict__ ws_part, const float* __restrict__ lora_t, const __nv_bfloat16* __restrict__ lora_up,
-           int lora_r) {
+           int lora_r, int codebook) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* ring = smem;
@@ -343,20 +343,33 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
         // thread t writes 16-byte chunks c = t + 256 it (two copies of byte
         // c / 8): its low nibble (t / 8) mod 16 is fixed and its high nibble is
         // 2 it + t / 128, so every level is an immediate and the build touches
-        // no memory but the table.
+        // no memory but the table.  The FP4 codebook reads its values from
+        // constant memory instead.
         static_assert(kLutBytes / 16 == 8 * 32 * kConsumers, "eight chunks per consumer thread");
         {
-            constexpr float kLv[16] = NF4_LEVELS_INIT;
             const int lo_idx = (threadIdx.x >> 3) & 15;
-            float lo = kLv[0];
-#pragma unroll
-            for (int v = 1; v < 16; ++v) lo = (lo_idx == v) ? kLv[v] : lo;
             const bool odd = (threadIdx.x >> 7) != 0;
+            if (codebook == kCbNf4) {
+                constexpr float kLv[16] = NF4_LEVELS_INIT;
+                float lo = kLv[0];
 #pragma unroll
-            for (int it = 0; it < 8; ++it) {
-                const float hi = odd ? kLv[2 * it + 1] : kLv[2 * it];
-                sts128(smem_u32(lut) + 16u * (threadIdx.x + 32 * kConsumers * it),
-                       make_uint4(__float_as_uint(hi), __float_as_uint(lo), __float_as_uint(hi), __float_as_uint(lo)));
+                for (int v = 1; v < 16; ++v) lo = (lo_idx == v) ? kLv[v] : lo;
+#pragma unroll
+                for (int it = 0; it < 8; ++it) {
+                    const float hi = odd ? kLv[2 * it + 1] : kLv[2 * it];
+                    sts128(smem_u32(lut) + 16u * (threadIdx.x + 32 * kConsumers * it),
+                           make_uint4(__float_as_uint(hi), __float_as_uint(lo), __float_as_uint(hi),
+                                      __float_as_uint(lo)));
+                }
+            } else {
+                const float lo = kCodebook[kCbFp4][lo_idx];
+#pragma unroll
+                for (int it = 0; it < 8; ++it) {
+                    const float hi = kCodebook[kCbFp4][2 * it + (odd ? 1 : 0)];
+                    sts128(smem_u32(lut) + 16u * (threadIdx.x + 32 * kConsumers * it),
+                           make_uint4(__float_as_uint(hi), __float_as_uint(lo), __float_as_uint(hi),
+                                      __float_as_uint(lo)));
+                }
             }
         }
         named_bar_sync(1, 32 * kConsumers);
@@ -596,7 +609,7 @@ template <bool kBf16Out, bool kM16, bool kLora>
 static cudaError_t launch_gemv(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const int8_t* absmax_q,
                                const float* absmax_scale, const float* absmax_offset, int mt, int64_t n,
                                int64_t k, int cluster, bool weights_early, void* Yt, int32_t* dev_status,
-                               void* ws, const LoraArgs& lora, int device, cudaStream_t stream) {
+                               void* ws, const LoraArgs& lora, int codebook, int device, cudaStream_t stream) {
     static bool attr_set[64] = {};
     if (!attr_set[device]) {
         const cudaError_t e = cudaFuncSetAttribute(gemv::k_nf4_gemv<kBf16Out, kM16, kLora>,
@@ -631,18 +644,18 @@ static cudaError_t launch_gemv(const CUtensorMap& tm_w, const CUtensorMap& tm_x,
     cfg.numAttrs = na;
     return cudaLaunchKernelEx(&cfg, gemv::k_nf4_gemv<kBf16Out, kM16, kLora>, tm_w, tm_x, absmax_q, absmax_scale,
                               absmax_offset, mt, n, k, cluster, weights_early ? 1 : 0, Yt, dev_status, ws_cnt,
-                              ws_part, lora.t, lora.up, lora.r);
+                              ws_part, lora.t, lora.up, lora.r, codebook);
 }
 
 // One of the eight instantiations: output type, more than 8 tokens, LoRA term.
 static cudaError_t dispatch_gemv(bool bf16, bool m16, bool lora_on, const CUtensorMap& tm_w, const CUtensorMap& tm_x,
                                  const int8_t* absmax_q, const float* absmax_scale, const float* absmax_offset,
                                  int mt, int64_t n, int64_t k, int cluster, bool early, void* Yt, int32_t* ds,
-                                 void* ws, const LoraArgs& lora, int device, cudaStream_t stream) {
+                                 void* ws, const LoraArgs& lora, int codebook, int device, cudaStream_t stream) {
 #define NF4_GEMV_CASE(B, M, L)                                                                                   \
     if (bf16 == B && m16 == M && lora_on == L)                                                                  \
         return launch_gemv<B, M, L>(tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt, n, k, cluster, early, \
-                                    Yt, ds, ws, lora, device, stream);
+                                    Yt, ds, ws, lora, codebook, device, stream);
     NF4_GEMV_CASE(true, true, false)
     NF4_GEMV_CASE(true, false, false)
     NF4_GEMV_CASE(false, true, false)
@@ -658,11 +671,12 @@ static cudaError_t dispatch_gemv(bool bf16, bool m16, bool lora_on, const CUtens
 cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                           const float* absmax_scale, const float* absmax_offset, int64_t n,
                           int64_t k, void* Y, bool y_bf16, int32_t* dev_status, bool weights_early,
-                          void* ws, const LoraArgs& lora, const DeviceInfo& dev, cudaStream_t stream) {
+                          void* ws, const LoraArgs& lora, int codebook, const DeviceInfo& dev,
+                          cudaStream_t stream) {
     if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
     if (m > kGemvMaxTokens)
-        return launch_gemm(X, m, wq, absmax_q, absmax_scale, absmax_offset, n, k, Y, y_bf16, dev_status, lora, dev,
-                           stream);
+        return launch_gemm(X, m, wq, absmax_q, absmax_scale, absmax_offset, n, k, Y, y_bf16, dev_status, lora,
+                           codebook, dev, stream);
     CUtensorMap tm_w;
     cudaError_t e = tmap_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, static_cast<uint64_t>(k / 2),
                             static_cast<uint64_t>(n), static_cast<uint64_t>(k / 2), 128, gemv::kRows,
@@ -681,7 +695,7 @@ cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int
         if (e != cudaSuccess) return e;
         void* Yt = static_cast<char*>(Y) + static_cast<size_t>(t0) * n * ybytes;
         e = dispatch_gemv(y_bf16, mt > 8, lora.t != nullptr, tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt,
-                          n, k, cluster, weights_early, Yt, dev_status, ws, lora, dev.device, stream);
+                          n, k, cluster, weights_early, Yt, dev_status, ws, lora, codebook, dev.device, stream);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

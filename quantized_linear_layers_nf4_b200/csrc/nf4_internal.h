@@ -32,7 +32,8 @@ struct LoraArgs {
 // Properties of the current device (cached per device).
 cudaError_t current_device(DeviceInfo* out);
 
-cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n_elem, uint8_t* wq, float* absmax,
+// `codebook` in the launchers below: 0 = NF4 levels, 1 = FP4 values.
+cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n_elem, uint8_t* wq, float* absmax, int codebook,
                             const DeviceInfo& dev, cudaStream_t stream);
 
 // Maximum number of absmax values double quantization accepts in one call.
@@ -43,7 +44,7 @@ cudaError_t launch_double_quant(const float* absmax, int64_t nb, double* workspa
                                 cudaStream_t stream);
 
 cudaError_t launch_dequantize(const uint8_t* wq, const int8_t* absmax_q, const float* absmax_scale,
-                              const float* absmax_offset, int64_t n_elem, void* out, bool out_bf16,
+                              const float* absmax_offset, int64_t n_elem, void* out, bool out_bf16, int codebook,
                               const DeviceInfo& dev, cudaStream_t stream);
 
 // Bytes of the split-k workspace the decode path needs for (m, n, k); 0 if none.
@@ -53,7 +54,8 @@ size_t linear_workspace_bytes(int64_t m, int64_t n, int64_t k, const DeviceInfo&
 cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                           const float* absmax_scale, const float* absmax_offset, int64_t n,
                           int64_t k, void* Y, bool y_bf16, int32_t* dev_status, bool weights_early,
-                          void* ws, const LoraArgs& lora, const DeviceInfo& dev, cudaStream_t stream);
+                          void* ws, const LoraArgs& lora, int codebook, const DeviceInfo& dev,
+                          cudaStream_t stream);
 
 // t[m, r] = scale * X[m, k] down[r, k]^T in fp32 (fixed order); also its two bf16
 // halves when t_hi / t_lo are given.
@@ -64,17 +66,18 @@ cudaError_t launch_lora_down(const void* X, int64_t m, int64_t k, const void* do
 // [n, k], may be null), wq_out [n*k/2] and absmax_out [n*k/64] fp32.
 cudaError_t launch_merge_lora(const uint8_t* wq, const int8_t* absmax_q, const float* absmax_scale,
                               const float* absmax_offset, int64_t n, int64_t k, const void* down, const void* up,
-                              int r, float scale, void* w_new, uint8_t* wq_out, float* absmax_out,
+                              int r, float scale, void* w_new, uint8_t* wq_out, float* absmax_out, int codebook,
                               const DeviceInfo& dev, cudaStream_t stream);
 
 cudaError_t launch_gemm_dx(const void* dY, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                            const float* absmax_scale, const float* absmax_offset, int64_t n, int64_t k, void* dX,
-                           bool dx_bf16, int32_t* dev_status, const DeviceInfo& dev, cudaStream_t stream);
+                           bool dx_bf16, int32_t* dev_status, int codebook, const DeviceInfo& dev,
+                           cudaStream_t stream);
 
 cudaError_t launch_gemm(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                         const float* absmax_scale, const float* absmax_offset, int64_t n, int64_t k, void* Y,
-                        bool y_bf16, int32_t* dev_status, const LoraArgs& lora, const DeviceInfo& dev,
-                        cudaStream_t stream);
+                        bool y_bf16, int32_t* dev_status, const LoraArgs& lora, int codebook,
+                        const DeviceInfo& dev, cudaStream_t stream);
 
 // Token counts up to this run the decode GEMV; larger ones the tcgen05 GEMM.
 constexpr int64_t kGemvMaxTokens = 16;

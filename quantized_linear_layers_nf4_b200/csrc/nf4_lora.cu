@@ -72,10 +72,11 @@ __global__ void __launch_bounds__(256) k_lora_down(const __nv_bfloat16* __restri
 //   What  = bf16_rn(fp32(level * ahat))                 the bf16 dequantized weight
 //   delta = fma chain over j = 0 .. r-1 of up[o][j] * down[j][c], from 0, in fp32
 //   Wnew  = bf16_rn(fp32(What + fp32(scale * delta)))
-// and Wnew is then quantized blockwise exactly as k_nf4_quantize does.  Lane
-// layout as in quantization: a lane owns 8 consecutive elements of one row
-// (k % 64 == 0 keeps each 64-block inside a row), 8 lanes one block.  down is
-// small ([r, k] bf16) and is re-read from L1/L2 by every row.
+// and Wnew is then quantized blockwise exactly as k_nf4_quantize does, with the
+// weight's own codebook (NF4 or FP4).  Lane layout as in quantization: a lane
+// owns 8 consecutive elements of one row (k % 64 == 0 keeps each 64-block
+// inside a row), 8 lanes one block.  down is small ([r, k] bf16) and is re-read
+// from L1/L2 by every row.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_nf4_merge_lora(const uint32_t* __restrict__ wq32,
                                                         const int8_t* __restrict__ absmax_q,
@@ -84,9 +85,9 @@ __global__ void __launch_bounds__(256) k_nf4_merge_lora(const uint32_t* __restri
                                                         int64_t n_groups, const __nv_bfloat16* __restrict__ down,
                                                         const __nv_bfloat16* __restrict__ up, int r, float scale,
                                                         uint4* __restrict__ w_new, uint32_t* __restrict__ wq_out,
-                                                        float* __restrict__ absmax_out) {
+                                                        float* __restrict__ absmax_out, int codebook) {
     __shared__ float lv[16];
-    if (threadIdx.x < 16) lv[threadIdx.x] = kLevels[threadIdx.x];
+    if (threadIdx.x < 16) lv[threadIdx.x] = kCodebook[codebook][threadIdx.x];
     __syncthreads();
     const float mu = __ldg(mu_ptr);
     const uint16_t* up16 = reinterpret_cast<const uint16_t*>(up);
@@ -147,8 +148,11 @@ __global__ void __launch_bounds__(256) k_nf4_merge_lora(const uint32_t* __restri
         uint32_t packed = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const uint32_t hi = static_cast<uint32_t>(quantize_one(w[2 * i], a));
-            const uint32_t lo = static_cast<uint32_t>(quantize_one(w[2 * i + 1], a));
+            const float wh = w[2 * i], wl = w[2 * i + 1];
+            const uint32_t hi = static_cast<uint32_t>(codebook == kCbFp4 ? quantize_code<kCbFp4>(wh, a)
+                                                                          : quantize_code<kCbNf4>(wh, a));
+            const uint32_t lo = static_cast<uint32_t>(codebook == kCbFp4 ? quantize_code<kCbFp4>(wl, a)
+                                                                          : quantize_code<kCbNf4>(wl, a));
             packed |= ((hi << 4) | lo) << (8 * i);
         }
         if (valid) {
@@ -171,7 +175,7 @@ cudaError_t launch_lora_down(const void* X, int64_t m, int64_t k, const void* do
 
 cudaError_t launch_merge_lora(const uint8_t* wq, const int8_t* absmax_q, const float* absmax_scale,
                               const float* absmax_offset, int64_t n, int64_t k, const void* down, const void* up,
-                              int r, float scale, void* w_new, uint8_t* wq_out, float* absmax_out,
+                              int r, float scale, void* w_new, uint8_t* wq_out, float* absmax_out, int codebook,
                               const DeviceInfo& dev, cudaStream_t stream) {
     const int64_t n_groups = n * k / 8;
     const int64_t n_chunks = (n_groups + 31) / 32;
@@ -182,7 +186,7 @@ cudaError_t launch_merge_lora(const uint8_t* wq, const int8_t* absmax_q, const f
     lora::k_nf4_merge_lora<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
         reinterpret_cast<const uint32_t*>(wq), absmax_q, absmax_scale, absmax_offset, k, n_groups,
         static_cast<const __nv_bfloat16*>(down), static_cast<const __nv_bfloat16*>(up), r, scale,
-        static_cast<uint4*>(w_new), reinterpret_cast<uint32_t*>(wq_out), absmax_out);
+        static_cast<uint4*>(w_new), reinterpret_cast<uint32_t*>(wq_out), absmax_out, codebook);
     return cudaGetLastError();
 }
 

@@ -41,7 +41,7 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* __restrict__ W, int64
     }
 }
 
-template <typename T>
+template <typename T, int CB>
 __global__ void __launch_bounds__(256) k_nf4_quantize(const T* __restrict__ W, int64_t n_groups,
                                                       uint32_t* __restrict__ wq32,
                                                       float* __restrict__ absmax) {
@@ -68,8 +68,8 @@ __global__ void __launch_bounds__(256) k_nf4_quantize(const T* __restrict__ W, i
         uint32_t packed = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const uint32_t hi = static_cast<uint32_t>(quantize_one(w[2 * i], a));
-            const uint32_t lo = static_cast<uint32_t>(quantize_one(w[2 * i + 1], a));
+            const uint32_t hi = static_cast<uint32_t>(quantize_code<CB>(w[2 * i], a));
+            const uint32_t lo = static_cast<uint32_t>(quantize_code<CB>(w[2 * i + 1], a));
             packed |= ((hi << 4) | lo) << (8 * i);      // element 2i in the high nibble
         }
         if (valid) {
@@ -79,21 +79,29 @@ __global__ void __launch_bounds__(256) k_nf4_quantize(const T* __restrict__ W, i
     }
 }
 
-cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n_elem, uint8_t* wq, float* absmax,
+template <int CB>
+static void launch_quantize_cb(const void* W, bool w_bf16, int64_t n_groups, uint8_t* wq, float* absmax,
+                               int64_t blocks, cudaStream_t stream) {
+    if (w_bf16)
+        k_nf4_quantize<__nv_bfloat16, CB><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(W), n_groups, reinterpret_cast<uint32_t*>(wq), absmax);
+    else
+        k_nf4_quantize<float, CB><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+            static_cast<const float*>(W), n_groups, reinterpret_cast<uint32_t*>(wq), absmax);
+}
+
+cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n_elem, uint8_t* wq, float* absmax, int codebook,
                             const DeviceInfo& dev, cudaStream_t stream) {
     const int64_t n_groups = n_elem / 8;
     const int64_t n_chunks = (n_groups + 31) / 32;
-    const int threads = 256;
     int64_t blocks = (n_chunks + 7) / 8;
     const int64_t cap = static_cast<int64_t>(dev.sm_count) * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    if (w_bf16)
-        k_nf4_quantize<__nv_bfloat16><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(W), n_groups, reinterpret_cast<uint32_t*>(wq), absmax);
+    if (codebook == kCbFp4)
+        launch_quantize_cb<kCbFp4>(W, w_bf16, n_groups, wq, absmax, blocks, stream);
     else
-        k_nf4_quantize<float><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
-            static_cast<const float*>(W), n_groups, reinterpret_cast<uint32_t*>(wq), absmax);
+        launch_quantize_cb<kCbNf4>(W, w_bf16, n_groups, wq, absmax, blocks, stream);
     return cudaGetLastError();
 }
 

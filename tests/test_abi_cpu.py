@@ -68,6 +68,16 @@ def test_library_levels_equal_the_oracle_levels(L):
     assert L.nf4_codebook(None) == -1
 
 
+def test_library_fp4_values_equal_the_oracle_fp4_values(L):
+    out = np.zeros(16, dtype=np.float32)
+    assert L.nf4_codebook_typed(1, out.ctypes.data_as(ctypes.c_void_p)) == 0
+    assert np.array_equal(out.view(np.uint32), O.codebook("fp4").view(np.uint32))
+    assert L.nf4_codebook_typed(0, out.ctypes.data_as(ctypes.c_void_p)) == 0
+    assert np.array_equal(out.view(np.uint32), O.codebook().view(np.uint32))
+    assert L.nf4_codebook_typed(2, out.ctypes.data_as(ctypes.c_void_p)) == -4
+    assert L.nf4_codebook_typed(1, None) == -1
+
+
 def test_workspace_size(L):
     assert L.nf4_double_quant_workspace_bytes(0) == 0
     assert L.nf4_double_quant_workspace_bytes(1) == 8
@@ -179,6 +189,20 @@ def test_merge_lora_validation(L):
     assert mg(w, FAKE, ODD, 16, 2.0, None, FAKE, FAKE, None) == -3
     assert mg(w, FAKE, FAKE, 16, 2.0, ODD, FAKE, FAKE, None) == -3             # w_new misaligned
     assert mg(ctypes.byref(_weight(magic=7)), FAKE, FAKE, 16, 2.0, None, FAKE, FAKE, None) == -5
+
+
+def test_fp4_quantize_and_weight_validation(L):
+    qt = L.nf4_quantize_typed
+    assert qt(FAKE, 0, 4, 64, 2, FAKE, FAKE, None) == -4                      # unknown codebook
+    assert qt(FAKE, 0, 4, 64, -1, FAKE, FAKE, None) == -4
+    assert qt(None, 0, 4, 64, 1, FAKE, FAKE, None) == -1
+    assert qt(FAKE, 0, 4, 65, 1, FAKE, FAKE, None) == -2
+    assert L.nf4_dequantize(ctypes.byref(_weight(magic=_lib.NF4_FP4_WEIGHT_MAGIC + 1)), FAKE, 1, None) == -5
+    # an FP4 weight passes the struct check and then needs a device (only asked
+    # where there is none: these pointers are never valid device memory)
+    import torch
+    if not torch.cuda.is_available():
+        assert L.nf4_dequantize(ctypes.byref(_weight(magic=_lib.NF4_FP4_WEIGHT_MAGIC)), FAKE, 1, None) in (-7, -9)
 
 
 def test_valid_call_without_a_gpu_reports_instead_of_crashing(L):

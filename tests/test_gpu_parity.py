@@ -37,15 +37,15 @@ def _bits(t: torch.Tensor) -> np.ndarray:
     return t.numpy().reshape(-1)
 
 
-def _gpu_chain(nf4, W):
-    wq, absmax = nf4.nf4_quantize(W)
+def _gpu_chain(nf4, W, quant_type="nf4"):
+    wq, absmax = nf4.nf4_quantize(W, quant_type=quant_type)
     q, s, mu = nf4.nf4_double_quant(absmax)
-    weight = nf4.NF4Weight(W.shape[0], W.shape[1], wq, q, s, mu)
+    weight = nf4.NF4Weight(W.shape[0], W.shape[1], wq, q, s, mu, quant_type)
     return weight, absmax
 
 
-def _oracle_chain(Wh):
-    wq, absmax = O.quantize(Wh)
+def _oracle_chain(Wh, quant_type="nf4"):
+    wq, absmax = O.quantize(Wh, quant_type)
     q, s, mu = O.double_quant(absmax)
     return wq, absmax, q, s, mu
 
@@ -61,13 +61,13 @@ def _assert_equal(gpu: torch.Tensor, ref: np.ndarray, what: str):
         what, bad.size, bad[:5], g[bad[:5]], ref[bad[:5]])
 
 
-def _check_quant(nf4, W, full_dequant=True, rows=None):
+def _check_quant(nf4, W, full_dequant=True, rows=None, quant_type="nf4"):
     """Quantize + double-quant + dequant on the GPU and compare with the oracle.
     Returns (weight, oracle arrays) for further checks."""
-    weight, absmax = _gpu_chain(nf4, W)
+    weight, absmax = _gpu_chain(nf4, W, quant_type)
     n, k = W.shape
     Wh = _bits(W)
-    owq, oam, oq, os_, omu = _oracle_chain(Wh)
+    owq, oam, oq, os_, omu = _oracle_chain(Wh, quant_type)
     _assert_equal(absmax, oam, "absmax")
     _assert_equal(weight.wq, owq, "packed codes")
     _assert_equal(weight.absmax_q, oq, "absmax_q")
@@ -76,14 +76,14 @@ def _check_quant(nf4, W, full_dequant=True, rows=None):
     if full_dequant:
         d32 = nf4.nf4_dequantize(weight, torch.float32)
         d16 = nf4.nf4_dequantize(weight, torch.bfloat16)
-        ref = O.dequantize(owq, oq, os_, omu)
+        ref = O.dequantize(owq, oq, os_, omu, quant_type)
         _assert_equal(d32, ref, "dequant fp32")
         _assert_equal(d16.view(torch.int16).view(-1), O.f32_to_bf16(ref).view(np.int16), "dequant bf16")
     else:
         d32 = nf4.nf4_dequantize(weight, torch.float32)
         d16 = nf4.nf4_dequantize(weight, torch.bfloat16)
         for r in rows:
-            ref = O.dequantize_range(owq, oq, os_, omu, r * k, k)
+            ref = O.dequantize_range(owq, oq, os_, omu, r * k, k, quant_type)
             _assert_equal(d32[r], ref, "dequant fp32 row %d" % r)
             _assert_equal(d16[r].view(torch.int16), O.f32_to_bf16(ref).view(np.int16),
                           "dequant bf16 row %d" % r)
@@ -106,7 +106,8 @@ def _check_linear(nf4, X, weight, orc, token_rows=None, weight_rows=None, tol=LI
     Y32 = nf4.nf4_linear(X, weight, torch.float32)
     Y16 = nf4.nf4_linear(X, weight, torch.bfloat16)
     torch.cuda.synchronize()
-    wrows = np.stack([O.f32_to_bf16(O.dequantize_range(owq, oq, os_, omu, int(r) * k, k)) for r in R])
+    wrows = np.stack([O.f32_to_bf16(O.dequantize_range(owq, oq, os_, omu, int(r) * k, k, weight.quant_type))
+                      for r in R])
     xb = _bits(X).reshape(m, k)[T]
     ref = O.linear_bf16(np.ascontiguousarray(xb), np.ascontiguousarray(wrows))
     y32 = Y32.cpu().numpy()[np.ix_(T, R)]
@@ -273,7 +274,7 @@ def _check_dx(nf4, dY, weight, orc, token_rows=None, tol=LINEAR_TOL):
     D32 = nf4.nf4_linear_dx(dY, weight, torch.float32)
     D16 = nf4.nf4_linear_dx(dY, weight, torch.bfloat16)
     torch.cuda.synchronize()
-    what = O.f32_to_bf16(O.dequantize_range(owq, oq, os_, omu, 0, n * k)).reshape(n, k)
+    what = O.f32_to_bf16(O.dequantize_range(owq, oq, os_, omu, 0, n * k, weight.quant_type)).reshape(n, k)
     ref = O.linear_dx_bf16(np.ascontiguousarray(_bits(dY).reshape(m, n)[T]), what)
     d32 = D32.cpu().numpy()[T]
     e32 = _rel_fro(d32, ref)
@@ -333,7 +334,8 @@ def test_linear_lora(nf4, m, n, k, r, scale):
     Y32 = nf4.nf4_linear_lora(X, weight, down, up, scale, ws, dtype=torch.float32)
     Y16 = nf4.nf4_linear_lora(X, weight, down, up, scale, ws, dtype=torch.bfloat16)
     torch.cuda.synchronize()
-    wrows = np.stack([O.f32_to_bf16(O.dequantize_range(owq, oq, os_, omu, int(rr) * k, k)) for rr in R])
+    wrows = np.stack([O.f32_to_bf16(O.dequantize_range(owq, oq, os_, omu, int(rr) * k, k, weight.quant_type))
+                      for rr in R])
     ref = O.linear_lora_bf16(np.ascontiguousarray(_bits(X).reshape(m, k)[T]), wrows, _bits(down).reshape(r, k),
                              np.ascontiguousarray(_bits(up).reshape(n, r)[R]), scale)
     y32 = Y32.cpu().numpy()[np.ix_(T, R)]
@@ -391,6 +393,84 @@ def test_merge_lora_errors(nf4):
     with pytest.raises(nf4.NF4Error):   # rank above 256
         nf4.nf4_merge_lora(weight, torch.zeros(300, 64, dtype=torch.bfloat16, device="cuda"),
                            torch.zeros(64, 300, dtype=torch.bfloat16, device="cuda"), 1.0)
+
+
+# ---------------------------------------------------------------------------
+# FP4 codebook: the same kernels with the FP4 values in place of the NF4 levels.
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("n,k", [(1, 64), (5, 192), (257, 320), (100, 6400)])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_fp4_quantize_chain(nf4, n, k, dtype):
+    W = synth.weight_normal(n, k, seed=2000 + n * 7 + k, std=0.02, dtype=dtype, device="cuda")
+    weight, _ = _check_quant(nf4, W, quant_type="fp4")
+    assert weight.quant_type == "fp4"
+    assert torch.equal(nf4.nf4_codebook("fp4"), torch.from_numpy(O.codebook("fp4")))
+
+
+def test_fp4_edge_values(nf4):
+    n, k = 4, 256
+    W = synth.weight_normal(n, k, seed=2050, std=0.02, dtype=torch.float32, device="cuda")
+    W[0, 0:64] = 0.0                                   # zero block -> code 0
+    W[0, 64:128] = -0.0
+    W[1, 0] = 1.0                                      # absmax 1
+    c = torch.from_numpy(O.codebook("fp4")).cuda()
+    W[1, 1:8] = c[1:8]                                 # exact values
+    W[1, 9:16] = c[9:16]
+    W[1, 16] = c[1] / 2                                # the exact tie between 0 and 1/12
+    W[1, 17] = -c[1] / 2
+    W[1, 18] = -1e-12                                  # tiny negative -> +0
+    W[2, 0:64] = torch.arange(64, dtype=torch.float32, device="cuda") - 31.5
+    weight, _ = _check_quant(nf4, W, quant_type="fp4")
+    codes = O.unpack(weight.wq.cpu().numpy())
+    assert np.all(codes[:128] == 0) and codes[k + 16] == 0 and codes[k + 17] == 0 and codes[k + 18] == 0
+    assert not np.any(codes == 8)
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 200, 576), (16, 1000, 1024), (7, 11008, 512), (300, 520, 640),
+                                   (1024, 1024, 1024)])
+def test_fp4_linear(nf4, m, n, k):
+    """Decode GEMV and tcgen05 GEMM on FP4 codes against the fp64 oracle."""
+    W = synth.weight_normal(n, k, seed=2100 + n + m, dtype=torch.bfloat16, device="cuda")
+    X = synth.activations(m, k, seed=2110 + m, device="cuda")
+    weight, orc = _check_quant(nf4, W, full_dequant=False, rows=[0, n - 1], quant_type="fp4")
+    R = np.arange(n) if n <= 2048 else _sample_rows(n, 256, n)
+    _check_linear(nf4, X, weight, orc, weight_rows=R)
+    ws = nf4.linear_workspace([(n, k)], m=m)
+    a = nf4.nf4_linear(X, weight, torch.float32)
+    b = nf4.nf4_linear(X, weight, torch.float32, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_fp4_dx_lora_and_merge(nf4):
+    """Backward dX, the QLoRA layer (decode and prefill) and merge + requantize on
+    an FP4 weight."""
+    n, k, r = 520, 640, 16
+    W = synth.weight_normal(n, k, seed=2200, dtype=torch.bfloat16, device="cuda")
+    weight, orc = _check_quant(nf4, W, full_dequant=False, rows=[0, n - 1], quant_type="fp4")
+    owq, oq, os_, omu = orc
+    dY = synth.activations(300, n, seed=2201, device="cuda")
+    _check_dx(nf4, dY, weight, orc)
+    down = (synth.activations(r, k, seed=2202, device="cuda").float() * 0.02).to(torch.bfloat16)
+    up = (synth.activations(n, r, seed=2203, device="cuda").float() * 0.02).to(torch.bfloat16)
+    for m in (16, 300):
+        X = synth.activations(m, k, seed=2204 + m, device="cuda")
+        ws = nf4.lora_workspace(m, [(n, k)], r)
+        Y = nf4.nf4_linear_lora(X, weight, down, up, 2.0, ws, dtype=torch.float32)
+        torch.cuda.synchronize()
+        wrows = O.f32_to_bf16(O.dequantize(owq, oq, os_, omu, "fp4")).reshape(n, k)
+        ref = O.linear_lora_bf16(_bits(X).reshape(m, k), wrows, _bits(down).reshape(r, k), _bits(up).reshape(n, r),
+                                 2.0)
+        assert _rel_fro(Y.cpu().numpy(), ref) <= LINEAR_TOL
+    wq, absmax, w_new = nf4.nf4_merge_lora(weight, down, up, 2.0, want_bf16=True)
+    torch.cuda.synchronize()
+    ow, owq_new, oam_new = O.merge_lora(owq, oq, os_, omu, n, k, _bits(down).reshape(r, k),
+                                        _bits(up).reshape(n, r), 2.0, "fp4")
+    _assert_equal(w_new.view(torch.int16).view(-1), ow.view(np.int16), "merged bf16 weight (fp4)")
+    _assert_equal(wq, owq_new, "merged fp4 codes")
+    _assert_equal(absmax, oam_new, "merged absmax (fp4)")
+    assert nf4.merge_lora(weight, down, up, 2.0).quant_type == "fp4"
 
 
 def test_deterministic_and_stream_aware(nf4):

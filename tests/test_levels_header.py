@@ -48,3 +48,19 @@ def test_thresholds_are_round_down_midpoints():
         assert tj <= mid
         nxt = Fraction(float(np.nextafter(np.float32(t[j]), np.float32(2))))
         assert nxt > mid, "t_%d is not the largest fp32 <= midpoint" % j
+
+
+def test_header_fp4_levels_equal_oracle_fp4_codebook():
+    lv = np.array(_parse("FP4_LEVELS_INIT"), dtype=np.float32)
+    assert lv.size == 16
+    assert np.array_equal(lv.view(np.uint32), O.codebook("fp4").view(np.uint32))
+
+
+def test_fp4_thresholds_are_round_down_midpoints_of_the_magnitudes():
+    c = [Fraction(float(v)) for v in O.codebook("fp4")[:8]]
+    t = _parse("FP4_THRESHOLDS_INIT")
+    assert len(t) == 7
+    for j in range(7):
+        mid = (c[j] + c[j + 1]) / 2
+        assert Fraction(t[j]) <= mid
+        assert Fraction(float(np.nextafter(np.float32(t[j]), np.float32(2)))) > mid
