@@ -39,6 +39,19 @@ MUTANTS = [
     ("FP4 subnormals flushed", "(e == 0) ? 0.5 * m :", "(e == 0) ? 0.0 * m :"),
     ("FP4 zero block mapped to -0", "if (qt == ORC_FP4) idx[j] = 0;", "if (qt == ORC_FP4) idx[j] = 8;"),
     ("FP4 quantized with the NF4 levels", "const float* c = table_of(qt);", "const float* c = codebook();"),
+    # rounding-order readings (each result is still close; only the bits differ)
+    ("absmax dequant as q * (s / 127)",
+     "float t = (float)absmax_q[b] / 127.0f;\n    float u = t * absmax_scale[b / 256];",
+     "float t = absmax_scale[b / 256] / 127.0f;\n    float u = (float)absmax_q[b] * t;"),
+    ("absmax dequant with the rounded reciprocal of 127", "float t = (float)absmax_q[b] / 127.0f;",
+     "float t = (float)absmax_q[b] * (1.0f / 127.0f);"),
+    ("DQ code as r * (127 / s)", "float t = r / s;\n                float u = t * 127.0f;",
+     "float t = 127.0f / s;\n                float u = r * t;"),
+    ("DQ code rounds half away from zero", "q = (int)nearbyintf(u);", "q = (int)roundf(u);"),
+    ("DQ mean divided in fp32", "return (float)(orc_dq_sum(absmax, nb) / (double)nb);",
+     "return (float)orc_dq_sum(absmax, nb) / (float)nb;"),
+    ("weight dequant product in fp64 with a tiny bias", "out_f32[e] = c[idx] * a;",
+     "out_f32[e] = (float)((double)c[idx] * (double)a * (1.0 + 1e-9));"),
 ]
 
 

@@ -634,3 +634,190 @@ def test_fp4_merge_zero_scale_is_the_bf16_dequant():
     assert np.array_equal(w_new, what)
     wq3, am3 = O.quantize(what.reshape(-1), "fp4")
     assert np.array_equal(wq2, wq3) and np.array_equal(am2.view(np.uint32), am3.view(np.uint32))
+
+
+# ---------------------------------------------------------------------------
+# The rounding sequences, bit for bit.  Each expected value is recomputed in
+# exact rational arithmetic with an explicit round-to-nearest-even after every
+# step the readings name (xyzblog page, section 2.2 ② and Figure 2-2 step 5 for
+# the double quantization; technicalnotes page, section 5, for the dequantized
+# weight): absmax dequant a = RN(RN(RN(q / 127) * s) + mu); code
+# q = RNE(RN(RN(r / s) * 127)); mean mu = RN32(RN64(S / nb)); weight RN(c * a).
+# ---------------------------------------------------------------------------
+
+def _rn(x: Fraction, p: int, emin: int) -> Fraction:
+    """x rounded to the nearest binary floating-point value with p significant
+    bits and smallest normal exponent emin (gradual underflow), ties to even."""
+    if x == 0:
+        return Fraction(0)
+    a = abs(x)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    e = max(e, emin)
+    ulp = Fraction(2) ** (e - p + 1)
+    n, rem = divmod(a, ulp)
+    if 2 * rem > ulp or (2 * rem == ulp and n % 2 == 1):
+        n += 1
+    return n * ulp if x > 0 else -n * ulp
+
+
+def _rn32(x: Fraction) -> Fraction:
+    return _rn(x, 24, -126)
+
+
+def _rn64(x: Fraction) -> Fraction:
+    return _rn(x, 53, -1022)
+
+
+def _rne_int(x: Fraction) -> int:
+    n, rem = divmod(x, 1)
+    if 2 * rem > 1 or (2 * rem == 1 and n % 2 == 1):
+        n += 1
+    return int(n)
+
+
+def _F(v) -> Fraction:
+    return Fraction(float(v))
+
+
+def test_rounding_helper_against_ieee_hardware():
+    """The exact-rational rounding used below agrees with numpy's IEEE fp32 and
+    Python's fp64 arithmetic on random quotients, ties and subnormals."""
+    rng = np.random.default_rng(40)
+    for _ in range(2000):
+        a, b = f32(rng.standard_normal()), f32(rng.uniform(0.01, 10))
+        assert _rn32(_F(a) / _F(b)) == _F(a / b)
+        assert _rn32(_F(a) * _F(b)) == _F(a * b)
+        x, y = rng.standard_normal(), rng.uniform(0.1, 10)
+        assert _rn64(Fraction(x) / Fraction(y)) == Fraction(x / y)
+    assert _rn32(Fraction(1) + Fraction(1, 2 ** 24)) == 1                 # tie to even (down)
+    assert _rn32(Fraction(1) + Fraction(3, 2 ** 24)) == 1 + Fraction(2, 2 ** 23)
+    tiny = Fraction(3, 2 ** 150)                                           # half-way between subnormals
+    assert _rn32(tiny) == _F(np.float32(float(tiny)))
+    assert [_rne_int(Fraction(k, 2)) for k in (1, 3, 5, -1, -3)] == [0, 2, 2, 0, -2]
+
+
+def test_absmax_dequant_is_three_roundings_in_order():
+    """a = RN(RN(RN(q / 127) * s) + mu) for every int8 code: q / 127 a true
+    quotient (not q * RN(1/127)), multiplied by s (not q * RN(s / 127)), then mu
+    added.  s = 1, mu = 0 isolates the quotient."""
+    rng = np.random.default_rng(41)
+    q = np.arange(-127, 128, dtype=np.int8)
+    cases = [(f32(1.0), f32(0.0))] + [(f32(rng.uniform(1e-3, 0.3)), f32(rng.uniform(0.0, 0.1)))
+                                     for _ in range(6)] + [(f32(2.0 ** -20 * 3), f32(1e-6))]
+    for s, mu in cases:
+        got = O.absmax_hat(q, np.array([s], dtype=np.float32), mu)
+        for qi, g in zip(q, got):
+            want = _rn32(_rn32(_rn32(Fraction(int(qi), 127)) * _F(s)) + _F(mu))
+            assert _F(g) == want, (int(qi), float(s), float(mu))
+
+
+def _spec_mean(absmax: np.ndarray) -> np.float32:
+    """mu = RN32(RN64(S / nb)) with S the oracle's fixed-tree fp64 sum (pinned
+    on its own above)."""
+    return np.float32(O.dq_sum(absmax) / float(absmax.size))
+
+
+def test_dq_mean_divides_in_fp64_then_rounds_once_to_fp32():
+    rng = np.random.default_rng(42)
+    differ = 0
+    for trial in range(60):
+        nb = int(rng.integers(257, 3000)) | 1         # odd: the division is inexact
+        absmax = (np.abs(rng.standard_normal(nb)) * 0.05 + 1e-3).astype(np.float32)
+        S = O.dq_sum(absmax)
+        want = _rn32(_rn64(Fraction(S) / nb))          # fp64 quotient, then fp32
+        assert _F(O.dq_mean(absmax)) == want, (trial, nb)
+        if _rn32(_rn32(Fraction(S)) / nb) != want:     # an fp32 division would differ here
+            differ += 1
+    assert differ > 0, "no sample separates fp64 from fp32 division"
+
+
+def _spec_codes(absmax: np.ndarray):
+    """The double-quantization codes and scales from the stated sequence."""
+    mu = _F(_spec_mean(absmax))
+    r = [_rn32(_F(a) - mu) for a in absmax]
+    qs, ss = [], []
+    for j in range(0, len(r), 256):
+        blk = r[j:j + 256]
+        s = max(abs(v) for v in blk)
+        ss.append(s)
+        for v in blk:
+            qs.append(0 if s == 0 else _rne_int(_rn32(_rn32(v / s) * 127)))
+    return qs, ss
+
+
+def test_double_quant_code_is_the_stated_rounding_sequence():
+    rng = np.random.default_rng(43)
+    for nb in (1000, 256, 77):
+        absmax = (np.abs(rng.standard_normal(nb)) * 0.04 + 2e-3).astype(np.float32)
+        q, s, mu = O.double_quant(absmax)
+        wq, ws = _spec_codes(absmax)
+        assert [int(v) for v in q] == wq
+        assert [_F(v) for v in s] == ws
+        assert _F(mu) == _F(_spec_mean(absmax))
+
+
+def _tie_block(n_target: int, seed: int):
+    """An absmax vector in which one entry's RN(RN(r / s) * 127) is exactly
+    n_target + 1/2, found by a short fixed-point search in fp32 arithmetic."""
+    rng = np.random.default_rng(seed)
+    nb = 2048
+    absmax = (np.abs(rng.standard_normal(nb)) * 0.01 + 0.02).astype(np.float32)
+    blk0 = 3 * 256                       # the tie entry sits in DQ block 3 ...
+    absmax[blk0] = f32(0.2)              # ... whose largest |r| is set here
+    j = blk0 + 17
+    for _ in range(20):
+        mu = _spec_mean(absmax)
+        r = (absmax[blk0:blk0 + 256] - mu).astype(np.float32)
+        s = f32(np.max(np.abs(r)))
+        t = f32((n_target + 0.5) / 127.0)
+        for _k in range(64):             # walk t until t * 127 rounds onto the half
+            u = f32(t * f32(127.0))
+            if u == f32(n_target + 0.5):
+                break
+            t = np.nextafter(t, f32(np.inf) if u < n_target + 0.5 else f32(-np.inf))
+        rj = f32(t * s)
+        x = f32(mu + rj)
+        if absmax[j] == x:
+            break
+        absmax[j] = x
+    return absmax, j
+
+
+def test_double_quant_ties_round_half_to_even():
+    """Entries whose scaled code RN(RN(r / s) * 127) is exactly k + 1/2 go to the
+    even neighbour (both parities of k, both signs of r checked when found)."""
+    found = 0
+    for n_target, seed in ((40, 1), (41, 2), (70, 3), (9, 4), (100, 5)):
+        absmax, j = _tie_block(n_target, seed)
+        q, s, mu = O.double_quant(absmax)
+        mu_e = _F(_spec_mean(absmax))
+        r = _rn32(_F(absmax[j]) - mu_e)
+        blk = 3 * 256
+        smax = max(abs(_rn32(_F(a) - mu_e)) for a in absmax[blk:blk + 256])
+        u = _rn32(_rn32(r / smax) * 127)
+        if u.denominator != 2:
+            continue                      # the search missed this target; others must hit
+        found += 1
+        assert int(q[j]) == _rne_int(u), (n_target, float(u))
+        assert int(q[j]) % 2 == 0
+    assert found >= 2, "too few exact ties constructed"
+
+
+def test_weight_dequant_is_one_fp32_product():
+    """w = RN(c[idx] * a): one fp32 rounding of the exact product, on random
+    codes, scales and means (fp64-then-fp32 or any biased product differs on a
+    few percent of these)."""
+    rng = np.random.default_rng(44)
+    c = O.codebook()
+    nb = 300
+    absmax = (np.abs(rng.standard_normal(nb)) * 0.03 + 1e-3).astype(np.float32)
+    q, s, mu = O.double_quant(absmax)
+    wq = rng.integers(0, 256, size=nb * 32, dtype=np.uint8)
+    got = O.dequantize_range(wq, q, s, mu, 0, nb * 64)
+    ahat = O.absmax_hat(q, s, mu)
+    idx = O.unpack(wq)
+    for e in range(0, nb * 64, 7):
+        want = _rn32(_F(c[idx[e]]) * _F(ahat[e // 64]))
+        assert _F(got[e]) == want, e
