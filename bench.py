@@ -324,17 +324,28 @@ def run_ours(args, rank, world, local):
     shapes = sorted(set((w.n, w.k) for w in weights))
 
     early = not args.no_weights_early
+    # launch groups of the step: per layer q/k/v (one X), o, gate/up (one X), down
+    groups = []
+    for li in range(args.layers):
+        lw = weights[7 * li: 7 * li + 7]
+        groups += ([[w] for w in lw] if args.no_group else [lw[0:3], [lw[3]], lw[4:6], [lw[6]]])
 
     def decode_setup(m):
         xs = {k: synth.activations(m, k, seed=synth.seed_for(2, 100 + m) + k, device=dev)
               for k in set(k for _, k in shapes)}
-        ys = {n: torch.empty((m, n), dtype=torch.bfloat16, device=dev) for n in set(n for n, _ in shapes)}
+        # outputs: one buffer per (n, position in the launch group)
+        ys = {}
+        for grp in groups:
+            for i, w in enumerate(grp):
+                ys.setdefault((w.n, i), torch.empty((m, w.n), dtype=torch.bfloat16, device=dev))
         # one split-k workspace serves every linear of the step (they run one after another)
         ws = None if args.no_workspace else nf4.linear_workspace(shapes, m=m, device=dev)
 
         def step():
-            for w in weights:
-                nf4.nf4_linear(xs[w.k], w, torch.bfloat16, out=ys[w.n], weights_early=early, workspace=ws)
+            for grp in groups:
+                nf4.nf4_linear_group(xs[grp[0].k], grp, torch.bfloat16,
+                                     outs=[ys[(w.n, i)] for i, w in enumerate(grp)],
+                                     weights_early=early, workspace=ws)
         step()
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
@@ -367,13 +378,14 @@ def run_ours(args, rank, world, local):
     t_step_max = max_over_ranks(t_step, world)
     total_bytes = sum_over_ranks(float(step_bytes), world)
     value = total_bytes / t_step_max / 1e9
-    launches_per_step = len(weights)
+    # nf4_linear_group launches one dequant-GEMV per weight (m <= 16)
+    launches_per_step = sum(len(grp) for grp in groups)
     avg_launch_s = t_step / launches_per_step
     bytes_per_launch = step_bytes / launches_per_step
 
     # ---- e2e: host buffers through the C ABI, copies inside the timed region ----
     xh = {k: x.cpu().pin_memory() for k, x in xs.items()}
-    yh = {n: torch.empty(y.shape, dtype=y.dtype).pin_memory() for n, y in ys.items()}
+    yh = {key: torch.empty(y.shape, dtype=y.dtype).pin_memory() for key, y in ys.items()}
     h2d = sum(x.numel() * x.element_size() for x in xh.values())
     d2h = sum(y.numel() * y.element_size() for y in yh.values())
 
@@ -381,8 +393,8 @@ def run_ours(args, rank, world, local):
         for k, x in xh.items():
             xs[k].copy_(x, non_blocking=True)
         g.replay()
-        for n, y in ys.items():
-            yh[n].copy_(y, non_blocking=True)
+        for key, y in ys.items():
+            yh[key].copy_(y, non_blocking=True)
     for _ in range(args.warmup):
         e2e_step()
     barrier(world)
@@ -401,6 +413,32 @@ def run_ours(args, rank, world, local):
         by_m[m] = round(bm / _events_time(gm.replay, max(2, args.steps // 2), stream) / 1e9, 1)
         del gm
 
+    # one weight shape alone: back-to-back launches on rotating copies of the
+    # weight (about 300 MB, beyond L2), graph-captured, m = 16
+    single = {}
+    for tag, w0 in (("4096x4096", weights[0]), ("11008x4096", weights[4]), ("4096x11008", weights[6])):
+        ncopy = max(2, int(300e6 // linear_bytes(w0.n, w0.k, 16, 2)) + 1)
+        copies = [w0] + [nf4.NF4Weight(w0.n, w0.k, w0.wq.clone(), w0.absmax_q.clone(), w0.absmax_scale.clone(),
+                                       w0.absmax_offset.clone(), w0.quant_type) for _ in range(ncopy - 1)]
+        Xs1 = synth.activations(16, w0.k, seed=synth.seed_for(2, 300), device=dev)
+        Ys1 = torch.empty((16, w0.n), dtype=torch.bfloat16, device=dev)
+        ws1 = nf4.linear_workspace([(w0.n, w0.k)], m=16)
+
+        def f_single():
+            for wc in copies:
+                nf4.nf4_linear(Xs1, wc, torch.bfloat16, out=Ys1, workspace=ws1, weights_early=early)
+        f_single()
+        g1 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g1):
+            f_single()
+        for _ in range(3):
+            g1.replay()
+        t1 = _events_time(g1.replay, 20, stream) / len(copies)
+        single[tag] = {"gbs": round(linear_bytes(w0.n, w0.k, 16, 2) / t1 / 1e9, 1),
+                       "us_per_launch": round(t1 * 1e6, 2), "copies": len(copies)}
+        del g1, copies
+    single_note = "back-to-back nf4_linear_ws launches (m = 16) over rotating copies beyond L2, graph-captured"
+
     # dequant-GEMM at M = 4096, K = 4096, N = 11008
     gemm = None
     if not args.skip_gemm:
@@ -410,8 +448,9 @@ def run_ours(args, rank, world, local):
         Xg = synth.activations(4096, 4096, seed=synth.seed_for(3, 1), device=dev)
         Yg = torch.empty((4096, 11008), dtype=torch.bfloat16, device=dev)
         fn = lambda: nf4.nf4_linear(Xg, wg, torch.bfloat16, out=Yg)
-        fn()
-        t_g = _events_time(fn, 3, stream)
+        for _ in range(3):
+            fn()
+        t_g = _events_time(fn, 20, stream)
         tflops = 2.0 * 4096 * 4096 * 11008 / t_g / 1e12
         gemm = {"m": 4096, "k": 4096, "n": 11008, "tflops": round(tflops, 2),
                 "ms": round(t_g * 1e3, 3), "peak_tflops": pk["bf16_tflops"],
@@ -422,8 +461,9 @@ def run_ours(args, rank, world, local):
             Xs = synth.activations(mm, 4096, seed=synth.seed_for(3, 2) + mm, device=dev)
             Ys = torch.empty((mm, 11008), dtype=torch.bfloat16, device=dev)
             fs = lambda: nf4.nf4_linear(Xs, wg, torch.bfloat16, out=Ys)
-            fs()
-            ts = _events_time(fs, 5 if mm < 8192 else 3, stream)
+            for _ in range(3):
+                fs()
+            ts = _events_time(fs, 20, stream)
             sweep[mm] = round(2.0 * mm * 4096 * 11008 / ts / 1e12, 1)
             del Xs, Ys
         sweep[4096] = gemm["tflops"]
@@ -432,8 +472,9 @@ def run_ours(args, rank, world, local):
         dYg = synth.activations(4096, 11008, seed=synth.seed_for(3, 7), device=dev)
         dXg = torch.empty((4096, 4096), dtype=torch.bfloat16, device=dev)
         fdx = lambda: nf4.nf4_linear_dx(dYg, wg, torch.bfloat16, out=dXg)
-        fdx()
-        t_dx = _events_time(fdx, 3, stream)
+        for _ in range(3):
+            fdx()
+        t_dx = _events_time(fdx, 20, stream)
         gemm["dx"] = {"m": 4096, "n": 11008, "k": 4096, "tflops": round(2.0 * 4096 * 11008 * 4096 / t_dx / 1e12, 2),
                       "ms": round(t_dx * 1e3, 3), "frac": round(2.0 * 4096 * 11008 * 4096 / t_dx / 1e12 / pk["bf16_tflops"], 4)}
         del dYg, dXg
@@ -465,8 +506,9 @@ def run_ours(args, rank, world, local):
         del Wf
         fp4 = {}
         f_f = lambda: nf4.nf4_linear(Xg, wf, torch.bfloat16, out=Yg)
-        f_f()
-        fp4["gemm_tflops_m4096"] = round(2.0 * 4096 * 4096 * 11008 / _events_time(f_f, 3, stream) / 1e12, 1)
+        for _ in range(3):
+            f_f()
+        fp4["gemm_tflops_m4096"] = round(2.0 * 4096 * 4096 * 11008 / _events_time(f_f, 20, stream) / 1e12, 1)
         X16 = synth.activations(16, 4096, seed=synth.seed_for(3, 11), device=dev)
         Y16 = torch.empty((16, 11008), dtype=torch.bfloat16, device=dev)
         ws16 = nf4.linear_workspace([(11008, 4096)], m=16, device=dev)
@@ -497,9 +539,11 @@ def run_ours(args, rank, world, local):
         for mm in (1, 16, 512, 4096):
             X5 = synth.activations(mm, k5, seed=synth.seed_for(5, 1) + mm, device=dev)
             Y5 = torch.empty((mm, n5), dtype=torch.bfloat16, device=dev)
-            f5 = lambda: nf4.nf4_linear(X5, w5, torch.bfloat16, out=Y5)
-            f5()
-            t5 = _events_time(f5, 5, stream)
+            ws5 = nf4.linear_workspace([(n5, k5)], m=mm)
+            f5 = lambda: nf4.nf4_linear(X5, w5, torch.bfloat16, out=Y5, workspace=ws5)
+            for _ in range(3):
+                f5()
+            t5 = _events_time(f5, 20, stream)
             if mm <= 16:
                 stress["gemv_gbs"][mm] = round(linear_bytes(n5, k5, mm, 2) / t5 / 1e9, 1)
             else:
@@ -571,13 +615,18 @@ def run_ours(args, rank, world, local):
                        "l2": "inputs larger than L2 (%.2f GB of NF4 weights per step vs 126 MB)"
                              % (sum(w.nbytes() for w in weights) / 1e9),
                        "y_dtype": "bf16", "parallelism": "replicas (weak scaling)",
-                       "launch": ("CUDA graph of nf4_linear_ws(NF4_LINEAR_WEIGHTS_EARLY): programmatic "
-                                  "dependent launches, weight loads overlap the previous layer") if early
-                                 else "CUDA graph of nf4_linear_ws: each layer starts after the previous ends",
-                       "split_k": "cluster (distributed shared memory)" if args.no_workspace
-                                  else "global workspace, last CTA of a tile reduces"},
+                       "launch": ("CUDA graph of %d launches per step (%s)%s"
+                                  % (launches_per_step, "nf4_linear_ws per weight" if args.no_group else
+                                     "per layer: nf4_linear_group q/k/v, o, nf4_linear_group gate/up, down; "
+                                     "one launch per weight",
+                                     ", NF4_LINEAR_WEIGHTS_EARLY: programmatic dependent launches, weight loads "
+                                     "overlap the previous launch" if early else "")),
+                       "split_k": "thread-block clusters, partial sums through distributed shared memory"
+                                  if args.no_workspace
+                                  else "global workspace, last CTA of a tile adds the partial sums"},
             "frac_of_peak": round(value / world / pk["hbm_gbs"], 4),
             "decode_gbs_by_m": by_m,
+            "decode_single_shape": {"note": single_note, **single},
             "gemm": gemm,
             "stress_70b_layer": stress,
             "quant": qd,
@@ -602,7 +651,9 @@ def main():
     ap.add_argument("--m", type=int, default=16, help="tokens per decode step (1..16)")
     ap.add_argument("--layers", type=int, default=32)
     ap.add_argument("--no-workspace", action="store_true",
-                    help="split-k through thread-block clusters instead of a global workspace")
+                    help="split k through thread-block clusters instead of a global workspace")
+    ap.add_argument("--no-group", action="store_true",
+                    help="one launch per weight instead of grouping q/k/v and gate/up")
     ap.add_argument("--no-weights-early", action="store_true",
                     help="launch each linear without programmatic dependent launch")
     ap.add_argument("--skip-gemm", action="store_true")

@@ -250,7 +250,8 @@ nf4_status_t nf4_linear(const void* X, int64_t m, const nf4_weight_t* w, void* Y
 #define NF4_LINEAR_WEIGHTS_EARLY 1u
 
 /*
- * nf4_linear_ex -- nf4_linear with launch flags (0 or NF4_LINEAR_WEIGHTS_EARLY);
+ * nf4_linear_ex -- nf4_linear with launch flags (0, NF4_LINEAR_WEIGHTS_EARLY,
+ * NF4_LINEAR_TEST_TIMEOUT);
  * same arithmetic and results.  Arguments and errors as for nf4_linear, plus
  * NF4_ERR_DTYPE for an unknown flag bit.  Same source passages as nf4_linear;
  * the overlap of consecutive layers follows the per-layer dequantize-then-
@@ -259,6 +260,14 @@ nf4_status_t nf4_linear(const void* X, int64_t m, const nf4_weight_t* w, void* Y
 nf4_status_t nf4_linear_ex(const void* X, int64_t m, const nf4_weight_t* w, void* Y,
                            nf4_dtype_t y_dtype, int32_t* dev_status, uint32_t flags,
                            nf4_stream_t stream);
+
+/* Flag for nf4_linear_ex / nf4_linear_ws / nf4_linear_group, for tests of the
+ * bounded device waits only: the kernel's copy producers issue nothing and every
+ * device wait gives up after a few polls, so the call writes
+ * NF4_ERR_DEVICE_TIMEOUT to dev_status (when given) with no copy or tensor-core
+ * operation left in flight (the GEMM frees its tensor memory).  Y is not
+ * written.  The split-k workspace is left as it was. */
+#define NF4_LINEAR_TEST_TIMEOUT 0x80000000u
 
 /*
  * nf4_linear_dx -- backward through the frozen quantized base:
@@ -348,11 +357,12 @@ nf4_status_t nf4_merge_lora(const nf4_weight_t* w, const void* lora_down, const 
 
 /*
  * nf4_linear_workspace_bytes -- bytes of the optional split-k workspace that
- * nf4_linear_ws can use for Y[m, n] = X[m, k] * What^T on the current device;
- * 0 when that product splits no k range (then no workspace is needed).  The
- * workspace holds one counter per 128-row tile and the fp32 partial sums of
- * every CTA; one buffer serves every call whose requirement it meets.
- * Returns 0 for invalid sizes.  Same source passages as nf4_linear.
+ * nf4_linear_ws / nf4_linear_group can use for Y[m, n] = X[m, k] * What^T on the
+ * current device; 0 when that product splits no k range (then no workspace is
+ * needed), and always for m > 16 (the dequant-GEMM path).  The workspace holds
+ * one counter per 128-row tile and the fp32 partial sums of every CTA; one
+ * buffer serves every call whose requirement it meets.  Returns 0 for invalid
+ * sizes.  Same source passages as nf4_linear.
  */
 size_t nf4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k);
 
@@ -367,9 +377,11 @@ size_t nf4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k);
  * once.  (Same source passages as nf4_linear.)
  *   workspace  device, 16-byte aligned, at least nf4_linear_workspace_bytes(m,
  *              n, k) bytes, or NULL (the cluster path).  Its counters must be
- *              zero before first use: zero-fill the buffer once; every call
- *              leaves them zero again.  A workspace must not serve two calls
- *              that can run at the same time (for example on two streams).
+ *              zero before first use:
+ *              zero-fill the buffer once; every call leaves them zero again (a
+ *              call that ends in NF4_ERR_DEVICE_TIMEOUT may not: zero it again).
+ *              A workspace must not serve two calls that can run at the same
+ *              time (for example on two streams).
  *   ws_bytes   size of workspace in bytes
  * Errors: as nf4_linear_ex, plus NF4_ERR_WORKSPACE (workspace smaller than
  * required) and NF4_ERR_ALIGN (workspace not 16-byte aligned).
@@ -377,6 +389,34 @@ size_t nf4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k);
 nf4_status_t nf4_linear_ws(const void* X, int64_t m, const nf4_weight_t* w, void* Y,
                            nf4_dtype_t y_dtype, int32_t* dev_status, uint32_t flags,
                            void* workspace, size_t ws_bytes, nf4_stream_t stream);
+
+/* Most weights one nf4_linear_group call takes. */
+#define NF4_LINEAR_GROUP_MAX 4
+
+/*
+ * nf4_linear_group -- Y_i = X * What_i^T for up to NF4_LINEAR_GROUP_MAX quantized
+ * weights that share the input X (the query, key and value projections of an
+ * attention block, the gate and up projections of an MLP), in one call.  Same
+ * source passages as nf4_linear: per layer, each 4-bit weight is dequantized on
+ * chip and multiplied in bf16 ([P4] §5; [P5] §2.2 code walk).  The weights are
+ * launched one after another on the stream (the dequant-GEMV for m <= 16, the
+ * dequant-GEMM above), each spreading its own tiles over every SM; every output
+ * has the bits nf4_linear_ws gives for that weight alone, with or without a
+ * workspace.
+ *   X          device, bf16 [m, k], 16-byte aligned
+ *   w          host array of `count` pointers to weight structs, all with the same
+ *              k and the same codebook (magic)
+ *   count      1 .. NF4_LINEAR_GROUP_MAX
+ *   Y          host array of `count` device pointers, Y[i] [m, w[i]->n] of y_dtype,
+ *              16-byte aligned (outputs)
+ *   dev_status, flags, workspace, ws_bytes  as for nf4_linear_ws (the workspace
+ *              must meet nf4_linear_workspace_bytes for every weight)
+ * Errors: as nf4_linear_ws; NF4_ERR_SHAPE also for a count out of range or
+ * weights of different k, NF4_ERR_STATE for mixed codebooks.
+ */
+nf4_status_t nf4_linear_group(const void* X, int64_t m, const nf4_weight_t* const* w, int32_t count,
+                              void* const* Y, nf4_dtype_t y_dtype, int32_t* dev_status, uint32_t flags,
+                              void* workspace, size_t ws_bytes, nf4_stream_t stream);
 
 #ifdef __cplusplus
 }

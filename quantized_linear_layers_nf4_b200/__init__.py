@@ -10,6 +10,8 @@ calls.  Functions carry the C names:
 * ``nf4_dequantize(weight, dtype)`` -> dense tensor
 * ``nf4_linear(X, weight, dtype)`` -> ``Y = X @ W_hat^T`` (optionally with a
   split-k ``workspace`` from ``linear_workspace``)
+* ``nf4_linear_group(X, weights, dtype)`` -> ``[X @ W_i^T]`` for weights that
+  share X (q/k/v, gate/up), in one launch
 * ``nf4_linear_dx(dY, weight, dtype)`` -> ``dX = dY @ W_hat`` (backward through
   the frozen base)
 * ``nf4_linear_lora(X, weight, down, up, scale, workspace=...)`` -> the QLoRA
@@ -33,7 +35,7 @@ from . import _lib
 from ._lib import NF4_BF16, NF4_F32, NF4Error, nf4_weight_t
 
 __all__ = ["NF4Weight", "NF4Error", "nf4_quantize", "nf4_double_quant", "nf4_dequantize",
-           "nf4_linear", "nf4_linear_ex", "nf4_linear_dx", "nf4_linear_lora", "lora_workspace",
+           "nf4_linear", "nf4_linear_ex", "nf4_linear_group", "nf4_linear_dx", "nf4_linear_lora", "lora_workspace",
            "nf4_merge_lora", "merge_lora",
            "nf4_linear_workspace_bytes", "linear_workspace",
            "quantize_weight", "nf4_codebook", "library_path"]
@@ -159,10 +161,10 @@ def nf4_dequantize(weight: NF4Weight, dtype=torch.bfloat16, out: torch.Tensor | 
 
 
 def nf4_linear_ex(X, weight, dtype=torch.bfloat16, out=None, dev_status=None, stream=None,
-                  flags: int = 0):
-    """Same as nf4_linear with the C flags word (0 or NF4_LINEAR_WEIGHTS_EARLY)."""
-    return nf4_linear(X, weight, dtype, out, dev_status, stream,
-                      weights_early=bool(flags & _lib.NF4_LINEAR_WEIGHTS_EARLY))
+                  flags: int = 0, workspace=None):
+    """Same as nf4_linear with the C flags word (NF4_LINEAR_WEIGHTS_EARLY,
+    NF4_LINEAR_TEST_TIMEOUT)."""
+    return nf4_linear(X, weight, dtype, out, dev_status, stream, workspace=workspace, flags=flags)
 
 
 def nf4_linear_workspace_bytes(m: int, n: int, k: int) -> int:
@@ -181,15 +183,16 @@ def linear_workspace(shapes, m: int = 16, device=None) -> torch.Tensor:
 def nf4_linear(X: torch.Tensor, weight: NF4Weight, dtype=torch.bfloat16,
                out: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
                stream=None, weights_early: bool = False,
-               workspace: torch.Tensor | None = None) -> torch.Tensor:
+               workspace: torch.Tensor | None = None, flags: int = 0) -> torch.Tensor:
     """Y = X @ W_hat^T for bf16 X [m, k]; Y [m, n] in ``dtype`` (bf16 or fp32).
 
     ``weights_early=True`` sets NF4_LINEAR_WEIGHTS_EARLY: the weight was not
     written by the work just before this call on the stream, so its loads may
     overlap that work (programmatic dependent launch).  ``workspace`` (from
-    ``linear_workspace``) lets the decode path's split-k CTAs meet in global
-    memory instead of waiting for each other in a cluster; the results are the
-    same bits.  The call goes to ``nf4_linear_ws``."""
+    ``linear_workspace``) lets the decode path split the tiles of a weight over
+    all SMs, with partial sums meeting in global memory; the results are the
+    same bits as without it.  ``flags`` is OR'ed into the C flags word.  The
+    call goes to ``nf4_linear_ws``."""
     _need_cuda(X, "X")
     if X.dtype != torch.bfloat16 or X.dim() != 2:
         raise ValueError("X must be a 2-D bfloat16 tensor")
@@ -200,15 +203,46 @@ def nf4_linear(X: torch.Tensor, weight: NF4Weight, dtype=torch.bfloat16,
         out = torch.empty((m, weight.n), dtype=dtype, device=X.device)
     st = weight.struct()
     ds = ctypes.c_void_p(0) if dev_status is None else _ptr(dev_status)
-    flags = _lib.NF4_LINEAR_WEIGHTS_EARLY if weights_early else 0
-    if workspace is None:
-        ws, ws_bytes = ctypes.c_void_p(0), 0
-    else:
-        _need_cuda(workspace, "workspace")
-        ws, ws_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+    flags |= _lib.NF4_LINEAR_WEIGHTS_EARLY if weights_early else 0
+    ws, ws_bytes = _ws(workspace)
     _lib.check(_lib.lib().nf4_linear_ws(_ptr(X), m, ctypes.byref(st), _ptr(out), _DTYPES[dtype], ds,
                                         flags, ws, ws_bytes, _stream(stream)), "nf4_linear_ws")
     return out
+
+
+def _ws(workspace):
+    if workspace is None:
+        return ctypes.c_void_p(0), 0
+    _need_cuda(workspace, "workspace")
+    return _ptr(workspace), workspace.numel() * workspace.element_size()
+
+
+def nf4_linear_group(X: torch.Tensor, weights, dtype=torch.bfloat16, outs=None,
+                     dev_status: torch.Tensor | None = None, stream=None, weights_early: bool = False,
+                     workspace: torch.Tensor | None = None, flags: int = 0):
+    """[X @ W_i^T for W_i in weights] in one call for weights that share X and k
+    (at most NF4_LINEAR_GROUP_MAX), launched one after another on the stream;
+    each output has the bits of nf4_linear on that weight alone.  Returns the
+    list of outputs."""
+    _need_cuda(X, "X")
+    if X.dtype != torch.bfloat16 or X.dim() != 2:
+        raise ValueError("X must be a 2-D bfloat16 tensor")
+    if dtype not in _DTYPES:
+        raise ValueError("dtype must be float32 or bfloat16")
+    weights = list(weights)
+    count = len(weights)
+    m = X.shape[0]
+    if outs is None:
+        outs = [torch.empty((m, w.n), dtype=dtype, device=X.device) for w in weights]
+    structs = [w.struct() for w in weights]
+    wptrs = (ctypes.POINTER(nf4_weight_t) * max(count, 1))(*[ctypes.pointer(s) for s in structs])
+    yptrs = (ctypes.c_void_p * max(count, 1))(*[o.data_ptr() for o in outs])
+    ds = ctypes.c_void_p(0) if dev_status is None else _ptr(dev_status)
+    flags |= _lib.NF4_LINEAR_WEIGHTS_EARLY if weights_early else 0
+    ws, ws_bytes = _ws(workspace)
+    _lib.check(_lib.lib().nf4_linear_group(_ptr(X), m, wptrs, count, yptrs, _DTYPES[dtype], ds, flags, ws,
+                                           ws_bytes, _stream(stream)), "nf4_linear_group")
+    return outs
 
 
 def nf4_linear_dx(dY: torch.Tensor, weight: NF4Weight, dtype=torch.bfloat16,

@@ -12,6 +12,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "lib", "libnf4.so")
 
 NF4_OK = 0
+NF4_ERR_DEVICE_TIMEOUT = -8
 NF4_F32 = 0
 NF4_BF16 = 1
 NF4_BLOCKSIZE = 64
@@ -24,6 +25,8 @@ NF4_WEIGHT_VERSION = 1
 NF4_ABI_VERSION = 1
 NF4_DQ_NOALLOC_MAX_NB = 16777216
 NF4_LINEAR_WEIGHTS_EARLY = 1
+NF4_LINEAR_TEST_TIMEOUT = 0x80000000
+NF4_LINEAR_GROUP_MAX = 4
 
 # Every function include/nf4.h declares, with (restype, argtypes).
 _p = ctypes.c_void_p
@@ -62,6 +65,9 @@ SIGNATURES = {
                                       _p, _p, _p]),
     "nf4_linear_ws": (ctypes.c_int, [_p, _i64, ctypes.POINTER(nf4_weight_t), _p, ctypes.c_int, _p,
                                      ctypes.c_uint32, _p, ctypes.c_size_t, _p]),
+    "nf4_linear_group": (ctypes.c_int, [_p, _i64, ctypes.POINTER(ctypes.POINTER(nf4_weight_t)), ctypes.c_int32,
+                                        ctypes.POINTER(_p), ctypes.c_int, _p, ctypes.c_uint32, _p, ctypes.c_size_t,
+                                        _p]),
 }
 
 

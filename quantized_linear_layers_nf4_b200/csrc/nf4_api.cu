@@ -230,27 +230,50 @@ size_t nf4_linear_lora_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t 
     return lora_t_bytes(m, r) + nf4::linear_workspace_bytes(m, n, k, dev);
 }
 
-nf4_status_t nf4_linear_ws(const void* X, int64_t m, const nf4_weight_t* w, void* Y,
-                           nf4_dtype_t y_dtype, int32_t* dev_status, uint32_t flags, void* workspace,
-                           size_t ws_bytes, nf4_stream_t stream) {
-    nf4_status_t st = check_weight(w);
-    if (st != NF4_OK) return st;
-    if (!X || !Y) return NF4_ERR_NULL;
+nf4_status_t nf4_linear_group(const void* X, int64_t m, const nf4_weight_t* const* w, int32_t count,
+                              void* const* Y, nf4_dtype_t y_dtype, int32_t* dev_status, uint32_t flags,
+                              void* workspace, size_t ws_bytes, nf4_stream_t stream) {
+    if (!X || !w || !Y) return NF4_ERR_NULL;
+    if (count < 1 || count > nf4::kMaxGroup) return NF4_ERR_SHAPE;
+    nf4_status_t st;
+    for (int32_t i = 0; i < count; ++i) {
+        if ((st = check_weight(w[i])) != NF4_OK) return st;
+        if (!Y[i]) return NF4_ERR_NULL;
+        if (w[i]->k != w[0]->k) return NF4_ERR_SHAPE;
+        if (w[i]->magic != w[0]->magic) return NF4_ERR_STATE;
+        if (m >= 1 && m > INT64_MAX / w[i]->n) return NF4_ERR_SHAPE;
+        if (!aligned(Y[i], 16)) return NF4_ERR_ALIGN;
+    }
+    const int64_t k = w[0]->k;
     if (y_dtype != NF4_F32 && y_dtype != NF4_BF16) return NF4_ERR_DTYPE;
-    if ((flags & ~static_cast<uint32_t>(NF4_LINEAR_WEIGHTS_EARLY)) != 0) return NF4_ERR_DTYPE;
-    if (m < 1 || w->k % NF4_BLOCKSIZE != 0) return NF4_ERR_SHAPE;
-    if (m > INT64_MAX / w->k || m > INT64_MAX / w->n) return NF4_ERR_SHAPE;
-    if (!aligned(X, 16) || !aligned(Y, 16) || (dev_status && !aligned(dev_status, 4)))
-        return NF4_ERR_ALIGN;
+    if ((flags & ~static_cast<uint32_t>(NF4_LINEAR_WEIGHTS_EARLY | NF4_LINEAR_TEST_TIMEOUT)) != 0)
+        return NF4_ERR_DTYPE;
+    if (m < 1 || k % NF4_BLOCKSIZE != 0 || m > INT64_MAX / k) return NF4_ERR_SHAPE;
+    if (!aligned(X, 16) || (dev_status && !aligned(dev_status, 4))) return NF4_ERR_ALIGN;
     if (workspace && !aligned(workspace, 16)) return NF4_ERR_ALIGN;
     nf4::DeviceInfo dev;
     if ((st = device_ok(&dev)) != NF4_OK) return st;
-    if (workspace && ws_bytes < nf4::linear_workspace_bytes(m, w->n, w->k, dev)) return NF4_ERR_WORKSPACE;
-    return from_cuda(nf4::launch_linear(X, m, w->wq, w->absmax_q, w->absmax_scale, w->absmax_offset,
-                                        w->n, w->k, Y, y_dtype == NF4_BF16, dev_status,
-                                        (flags & NF4_LINEAR_WEIGHTS_EARLY) != 0, workspace, nf4::LoraArgs(),
-                                        codebook_of(w), dev,
-                                        reinterpret_cast<cudaStream_t>(stream)));
+    nf4::LinearWeight lw[nf4::kMaxGroup];
+    for (int32_t i = 0; i < count; ++i) {
+        if (workspace && ws_bytes < nf4::linear_workspace_bytes(m, w[i]->n, k, dev)) return NF4_ERR_WORKSPACE;
+        lw[i].wq = w[i]->wq;
+        lw[i].absmax_q = w[i]->absmax_q;
+        lw[i].absmax_scale = w[i]->absmax_scale;
+        lw[i].absmax_offset = w[i]->absmax_offset;
+        lw[i].n = w[i]->n;
+        lw[i].y = Y[i];
+    }
+    const uint32_t test = (flags & NF4_LINEAR_TEST_TIMEOUT) ? nf4::kTestStall : 0u;
+    return from_cuda(nf4::launch_linear_group(X, m, k, lw, count, y_dtype == NF4_BF16, dev_status,
+                                              (flags & NF4_LINEAR_WEIGHTS_EARLY) != 0, workspace, nf4::LoraArgs(),
+                                              codebook_of(w[0]), test, dev, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nf4_status_t nf4_linear_ws(const void* X, int64_t m, const nf4_weight_t* w, void* Y,
+                           nf4_dtype_t y_dtype, int32_t* dev_status, uint32_t flags, void* workspace,
+                           size_t ws_bytes, nf4_stream_t stream) {
+    if (!w) return NF4_ERR_NULL;
+    return nf4_linear_group(X, m, &w, 1, &Y, y_dtype, dev_status, flags, workspace, ws_bytes, stream);
 }
 
 nf4_status_t nf4_linear_ex(const void* X, int64_t m, const nf4_weight_t* w, void* Y,

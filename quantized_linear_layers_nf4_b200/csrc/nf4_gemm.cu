@@ -32,6 +32,7 @@
 // NF4_ERR_DEVICE_TIMEOUT, the CTA drains what it issued and frees its tensor
 // memory before returning.
 #include "nf4_common.cuh"
+#include "nf4_decode.cuh"
 #include "nf4_internal.h"
 #include "nf4_ptx.cuh"
 #include "nf4_tmap.h"
@@ -71,71 +72,6 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     return v;
 }
 
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-    uint32_t d;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-    return d;
-}
-
-// (a & ~c) | (b & c)
-__device__ __forceinline__ uint32_t select_bytes(uint32_t a, uint32_t b, uint32_t c) {
-    uint32_t d;
-    asm("lop3.b32 %0, %1, %2, %3, 0xD8;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
-
-__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-
-// bf16 table of one (row, block), as byte planes: plane h[q] holds the high
-// bytes of entries 4q..4q+3, plane l[q] their low bytes.
-struct Planes {
-    uint32_t h[4], l[4];
-};
-
-// T[i] = bf16(fp32(c_i * a)) for the 16 levels (pairs of levels multiplied by
-// one packed f32x2 multiply), split into byte planes.
-__device__ __forceinline__ void build_planes(const uint64_t (&cpair)[8], float a, Planes& P) {
-    uint64_t aa;
-    asm("mov.b64 %0, {%1, %1};" : "=l"(aa) : "f"(a));
-    uint32_t t[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        asm("{\n\t.reg .b64 r;\n\t.reg .f32 lo, hi;\n\t"
-            "mul.rn.f32x2 r, %1, %2;\n\t"
-            "mov.b64 {lo, hi}, r;\n\t"
-            "cvt.rn.bf16x2.f32 %0, hi, lo;\n\t}"
-            : "=r"(t[j])
-            : "l"(cpair[j]), "l"(aa));
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        P.h[q] = prmt(t[2 * q], t[2 * q + 1], 0x7531);
-        P.l[q] = prmt(t[2 * q], t[2 * q + 1], 0x6420);
-    }
-}
-
-// Four nibbles (the low 16 bits of s; s ^ 0x8888 in sx) -> two bf16x2 words in
-// k order.  For a nibble n < 8 the first permute picks T[n]'s byte and the
-// second yields a sign fill; for n >= 8 the other way round; a byte mask built
-// from each nibble's top bit selects the right one.  Nibble order in a packed
-// byte is (element 2i high, element 2i+1 low), so the final permutes swap
-// each pair back into k order.
-__device__ __forceinline__ void decode4(uint32_t s, uint32_t sx, const Planes& P, uint32_t& o0, uint32_t& o1) {
-    const uint32_t hA = prmt(P.h[0], P.h[1], s);
-    const uint32_t hB = prmt(P.h[2], P.h[3], sx);
-    const uint32_t lA = prmt(P.l[0], P.l[1], s);
-    const uint32_t lB = prmt(P.l[2], P.l[3], sx);
-    const uint32_t m = prmt(s << 4, s, 0xD9C8);  // byte k = 0xff iff nibble k >= 8
-    const uint32_t h = select_bytes(hA, hB, m);
-    const uint32_t l = select_bytes(lA, lB, m);
-    o0 = prmt(l, h, 0x4051);
-    o1 = prmt(l, h, 0x6273);
-}
-
 template <bool kBf16Out, bool kLora>
 __global__ void __launch_bounds__(kThreads, 1)
 k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
@@ -144,7 +80,7 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
            int32_t* __restrict__ dev_status, const float* __restrict__ lora_t,
            const __nv_bfloat16* __restrict__ lora_up, int lora_r, int lora_tc,
            const __grid_constant__ CUtensorMap tm_thi, const __grid_constant__ CUtensorMap tm_tlo,
-           const __grid_constant__ CUtensorMap tm_up, int codebook) {
+           const __grid_constant__ CUtensorMap tm_up, int codebook, uint32_t lim, int stall) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -198,9 +134,9 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         if (lane == 0) {
             prefetch_tensormap(&tm_x);
             int issued = 0;
-            for (int kt = 0; kt < nk; ++kt) {
+            for (int kt = 0; kt < (stall ? 0 : nk); ++kt) {
                 const int s = kt % kStagesA;
-                if (kt >= kStagesA && !mbar_wait(&empty_a[s], ((kt / kStagesA) - 1) & 1)) {
+                if (kt >= kStagesA && !mbar_wait_n(&empty_a[s], ((kt / kStagesA) - 1) & 1, lim)) {
                     timed_out = true;
                     break;
                 }
@@ -210,16 +146,16 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             }
             if (timed_out)  // leave no copy in flight
                 for (int kt = (issued > kStagesA ? issued - kStagesA : 0); kt < issued; ++kt)
-                    mbar_wait(&full_a[kt % kStagesA], (kt / kStagesA) & 1);
+                    mbar_wait_n(&full_a[kt % kStagesA], (kt / kStagesA) & 1, kWaitLimit);
         }
     } else if (warp == 2) {
         // ------------------------ packed-weight producer ----------------------
         if (lane == 0) {
             prefetch_tensormap(&tm_w);
             int issued = 0;
-            for (int kt = 0; kt < nk; ++kt) {
+            for (int kt = 0; kt < (stall ? 0 : nk); ++kt) {
                 const int s = kt % kStagesP;
-                if (kt >= kStagesP && !mbar_wait(&empty_p[s], ((kt / kStagesP) - 1) & 1)) {
+                if (kt >= kStagesP && !mbar_wait_n(&empty_p[s], ((kt / kStagesP) - 1) & 1, lim)) {
                     timed_out = true;
                     break;
                 }
@@ -230,7 +166,7 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             }
             if (timed_out)
                 for (int kt = (issued > kStagesP ? issued - kStagesP : 0); kt < issued; ++kt)
-                    mbar_wait(&full_p[kt % kStagesP], (kt / kStagesP) & 1);
+                    mbar_wait_n(&full_p[kt % kStagesP], (kt / kStagesP) & 1, kWaitLimit);
         }
     } else if (warp == 1) {
         // ------------------------------ MMA issuer ----------------------------
@@ -238,7 +174,7 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             for (int kt = 0; kt < nk; ++kt) {
                 const int sa = kt % kStagesA;
                 const int sb = kt % kStagesB;
-                if (!mbar_wait(&full_a[sa], (kt / kStagesA) & 1) || !mbar_wait(&full_b[sb], (kt / kStagesB) & 1)) {
+                if (!mbar_wait_n(&full_a[sa], (kt / kStagesA) & 1, lim) || !mbar_wait_n(&full_b[sb], (kt / kStagesB) & 1, lim)) {
                     timed_out = true;
                     break;
                 }
@@ -262,7 +198,7 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 const int nlt = (lora_r + 63) / 64;
                 for (int lt = 0; lt < nlt && !timed_out; ++lt) {
                     tc_commit(mma_done);
-                    if (!mbar_wait(mma_done, lt & 1)) {
+                    if (!mbar_wait_n(mma_done, lt & 1, lim)) {
                         timed_out = true;
                         break;
                     }
@@ -270,7 +206,7 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                     tma_load_2d(smem, &tm_thi, lt * 64, static_cast<int32_t>(m0), lora_full);
                     tma_load_2d(smem + kABytes, &tm_tlo, lt * 64, static_cast<int32_t>(m0), lora_full);
                     tma_load_2d(smem + 2 * kABytes, &tm_up, lt * 64, static_cast<int32_t>(n0), lora_full);
-                    if (!mbar_wait(lora_full, lt & 1)) {
+                    if (!mbar_wait_n(lora_full, lt & 1, lim)) {
                         timed_out = true;
                         break;
                     }
@@ -286,7 +222,7 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 }
             }
             tc_commit(timed_out ? drained : acc_ready);
-            if (timed_out) mbar_wait(drained, 0);  // issued MMAs finish before TMEM is freed
+            if (timed_out) mbar_wait_n(drained, 0, kWaitLimit);  // issued MMAs finish before TMEM is freed
         }
     } else if (warp >= 4) {
         // ------------------------ dequantize, then epilogue --------------------
@@ -332,7 +268,7 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 q = __ldg(absmax_q + bidx);
                 sc = __ldg(absmax_scale + (bidx >> 8));
             }
-            if (!__all_sync(kFull, mbar_wait(&full_p[sp], (kt / kStagesP) & 1))) {
+            if (!__all_sync(kFull, mbar_wait_n(&full_p[sp], (kt / kStagesP) & 1, lim))) {
                 timed_out = true;
                 break;
             }
@@ -342,7 +278,7 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             if (lane == 0) mbar_arrive(&empty_p[sp]);
             Planes P;
             build_planes(cpair, absmax_hat(q, sc, mu), P);
-            if (kt >= kStagesB && !__all_sync(kFull, mbar_wait(&empty_b[sb], ((kt / kStagesB) - 1) & 1))) {
+            if (kt >= kStagesB && !__all_sync(kFull, mbar_wait_n(&empty_b[sb], ((kt / kStagesB) - 1) & 1, lim))) {
                 timed_out = true;
                 break;
             }
@@ -361,7 +297,7 @@ k_nf4_gemm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             if (lane == 0) mbar_arrive(&full_b[sb]);
         }
         // epilogue: accumulators -> Y
-        const bool ok = !timed_out && __all_sync(kFull, mbar_wait(acc_ready, 0));
+        const bool ok = !timed_out && __all_sync(kFull, mbar_wait_n(acc_ready, 0, lim));
         if (!ok) timed_out = true;
         tc_fence_after();
         const int wd = warp - 4;
@@ -698,7 +634,7 @@ k_nf4_gemm_dx(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
 cudaError_t launch_gemm(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                         const float* absmax_scale, const float* absmax_offset, int64_t n, int64_t k, void* Y,
                         bool y_bf16, int32_t* dev_status, const LoraArgs& lora, int codebook,
-                        const DeviceInfo& dev, cudaStream_t stream) {
+                        uint32_t test_flags, const DeviceInfo& dev, cudaStream_t stream) {
     static bool attr_set[64][4] = {};
     if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
     const bool lo = lora.t != nullptr;
@@ -741,7 +677,8 @@ cudaError_t launch_gemm(const void* X, int64_t m, const uint8_t* wq, const int8_
 #define NF4_GEMM_LAUNCH(B, L)                                                                               \
     gemm::k_nf4_gemm<B, L><<<grid, gemm::kThreads, gemm::kSmemBytes, stream>>>(                              \
         tm_x, tm_w, absmax_q, absmax_scale, absmax_offset, m, n, k, Y, dev_status, lora.t, lora.up, lora.r,  \
-        lora_tc, tm_thi, tm_tlo, tm_up, codebook)
+        lora_tc, tm_thi, tm_tlo, tm_up, codebook, (test_flags & kTestStall) ? 64u : kWaitLimit,            \
+        (test_flags & kTestStall) ? 1 : 0)
     if (y_bf16) {
         if (lo) NF4_GEMM_LAUNCH(true, true); else NF4_GEMM_LAUNCH(true, false);
     } else {

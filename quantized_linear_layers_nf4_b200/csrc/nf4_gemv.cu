@@ -31,6 +31,8 @@
 // * Split-k: the CTAs of a thread-block cluster share a row tile and split k;
 //   their fp32 partials are added through distributed shared memory in a fixed
 //   rank order, so results are deterministic and no global scratch is needed.
+#include <mutex>
+
 #include "nf4_common.cuh"
 #include "nf4_internal.h"
 #include "nf4_ptx.cuh"
@@ -220,7 +222,7 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
            const float* __restrict__ mu_ptr, int m, int64_t n, int64_t k, int cluster, int weights_early,
            void* __restrict__ Y, int32_t* __restrict__ dev_status, uint32_t* __restrict__ ws_cnt,
            float4* __restrict__ ws_part, const float* __restrict__ lora_t, const __nv_bfloat16* __restrict__ lora_up,
-           int lora_r, int codebook) {
+           int lora_r, int codebook, uint32_t lim, int stall) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* ring = smem;
@@ -237,7 +239,9 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
     const int s0 = static_cast<int>((static_cast<int64_t>(n_stages) * rank) / cluster);
     const int s1 = static_cast<int>((static_cast<int64_t>(n_stages) * (rank + 1)) / cluster);
 
+    __shared__ int s_bad;  // some warp of this CTA gave up a wait
     if (threadIdx.x == 0) {
+        s_bad = 0;
         for (int s = 0; s < kRing; ++s) {
             mbar_init(&full[s], 2);   // the TMA bytes' arrive + the absmax-ready arrive
             mbar_init(&empty[s], kConsumers);
@@ -265,7 +269,7 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
 #pragma unroll
         for (int d = 0; d < kPrefetch; ++d)
             load_absmax_in(pre[d], absmax_q, absmax_scale, row0, lane, min(s0 + d, n_stages - 1), n, kblocks, aligned4);
-        for (int st0 = s0; st0 < s1 && !timed_out; st0 += kPrefetch) {
+        for (int st0 = s0; st0 < s1 && !timed_out && !stall; st0 += kPrefetch) {
 #pragma unroll
             for (int d = 0; d < kPrefetch; ++d) {
                 const int st = st0 + d;
@@ -273,7 +277,7 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
                 const int j = st - s0;
                 const int slot = j % kRing;
                 const int use = j / kRing;
-                if (j >= kRing && !__all_sync(kFull, mbar_wait(&empty[slot], (use - 1) & 1))) {
+                if (j >= kRing && !__all_sync(kFull, mbar_wait_n(&empty[slot], (use - 1) & 1, lim))) {
                     timed_out = true;
                     break;
                 }
@@ -390,7 +394,7 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
             const int j = st - s0;
             const int slot = j % kRing;
             // every lane polls; the warp proceeds only if all of them saw the stage
-            if (!__all_sync(kFull, mbar_wait(&full[slot], (j / kRing) & 1))) {
+            if (!__all_sync(kFull, mbar_wait_n(&full[slot], (j / kRing) & 1, lim))) {
                 timed_out = true;
                 break;
             }
@@ -439,8 +443,13 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
         }
         grid_dependency_wait();  // Y may still be in use by the preceding kernel
     }
-    if (timed_out) record_timeout(dev_status);
+    if (timed_out) {
+        record_timeout(dev_status);
+        s_bad = 1;
+    }
     __syncthreads();
+    // after a timeout the CTA writes neither Y nor the workspace (its sums are incomplete)
+    const bool bad = s_bad != 0;
     const float* redf = reinterpret_cast<const float*>(ring);
     float4* part4 = reinterpret_cast<float4*>(ring) + 4 * 16 * kRedPitch / 4;
     constexpr int kQ = 16 * kRows / 4;  // float4s of partial sums per CTA
@@ -459,6 +468,7 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
         // Split-k through the caller's workspace: each CTA stores its partial
         // sums and counts itself in; the last of the tile's C CTAs adds the
         // partials in rank order (the order the cluster path uses) and writes Y.
+        if (bad) return;
         const int tile = static_cast<int>(blockIdx.x);
         float4* part_g = ws_part + static_cast<int64_t>(tile) * cluster * kQ;
         for (int e = threadIdx.x; e < m * (kRows / 4); e += kThreads) part_g[rank * kQ + e] = part4[e];
@@ -504,7 +514,7 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
     const int rows_per_rank = ((rank + 1) * kRows) / cluster - r_lo;
     const int quads = rows_per_rank / 4;
     const uint32_t part_addr = smem_u32(part4);
-    if (kRows % (4 * cluster) != 0) {
+    if (!bad && kRows % (4 * cluster) != 0) {
         // C = 3, 5, 6, 7: row ranges of uneven length, one float per load
         for (int e = threadIdx.x; e < m * rows_per_rank; e += kThreads) {
             const int tok = e / rows_per_rank;
@@ -528,7 +538,7 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
             }
         }
     }
-    for (int e = threadIdx.x; e < (kRows % (4 * cluster) == 0 ? m * quads : 0); e += kThreads) {
+    for (int e = threadIdx.x; e < (!bad && kRows % (4 * cluster) == 0 ? m * quads : 0); e += kThreads) {
         const int tok = e / quads;
         const int r = r_lo + 4 * (e % quads);
         const uint32_t off = static_cast<uint32_t>((tok * kRows + r) * 4);
@@ -609,13 +619,18 @@ template <bool kBf16Out, bool kM16, bool kLora>
 static cudaError_t launch_gemv(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const int8_t* absmax_q,
                                const float* absmax_scale, const float* absmax_offset, int mt, int64_t n,
                                int64_t k, int cluster, bool weights_early, void* Yt, int32_t* dev_status,
-                               void* ws, const LoraArgs& lora, int codebook, int device, cudaStream_t stream) {
+                               void* ws, const LoraArgs& lora, int codebook, uint32_t test_flags, int device,
+                               cudaStream_t stream) {
+    static std::mutex mu;
     static bool attr_set[64] = {};
-    if (!attr_set[device]) {
-        const cudaError_t e = cudaFuncSetAttribute(gemv::k_nf4_gemv<kBf16Out, kM16, kLora>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, gemv::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set[device] = true;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!attr_set[device]) {
+            const cudaError_t e = cudaFuncSetAttribute(gemv::k_nf4_gemv<kBf16Out, kM16, kLora>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemv::kSmemBytes);
+            if (e != cudaSuccess) return e;
+            attr_set[device] = true;
+        }
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>((n + gemv::kRows - 1) / gemv::kRows), cluster, 1);
@@ -644,18 +659,20 @@ static cudaError_t launch_gemv(const CUtensorMap& tm_w, const CUtensorMap& tm_x,
     cfg.numAttrs = na;
     return cudaLaunchKernelEx(&cfg, gemv::k_nf4_gemv<kBf16Out, kM16, kLora>, tm_w, tm_x, absmax_q, absmax_scale,
                               absmax_offset, mt, n, k, cluster, weights_early ? 1 : 0, Yt, dev_status, ws_cnt,
-                              ws_part, lora.t, lora.up, lora.r, codebook);
+                              ws_part, lora.t, lora.up, lora.r, codebook,
+                              (test_flags & kTestStall) ? 64u : kWaitLimit, (test_flags & kTestStall) ? 1 : 0);
 }
 
 // One of the eight instantiations: output type, more than 8 tokens, LoRA term.
 static cudaError_t dispatch_gemv(bool bf16, bool m16, bool lora_on, const CUtensorMap& tm_w, const CUtensorMap& tm_x,
                                  const int8_t* absmax_q, const float* absmax_scale, const float* absmax_offset,
                                  int mt, int64_t n, int64_t k, int cluster, bool early, void* Yt, int32_t* ds,
-                                 void* ws, const LoraArgs& lora, int codebook, int device, cudaStream_t stream) {
+                                 void* ws, const LoraArgs& lora, int codebook, uint32_t test_flags, int device,
+                                 cudaStream_t stream) {
 #define NF4_GEMV_CASE(B, M, L)                                                                                   \
     if (bf16 == B && m16 == M && lora_on == L)                                                                  \
         return launch_gemv<B, M, L>(tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt, n, k, cluster, early, \
-                                    Yt, ds, ws, lora, codebook, device, stream);
+                                    Yt, ds, ws, lora, codebook, test_flags, device, stream);
     NF4_GEMV_CASE(true, true, false)
     NF4_GEMV_CASE(true, false, false)
     NF4_GEMV_CASE(false, true, false)
@@ -668,15 +685,14 @@ static cudaError_t dispatch_gemv(bool bf16, bool m16, bool lora_on, const CUtens
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
-                          const float* absmax_scale, const float* absmax_offset, int64_t n,
-                          int64_t k, void* Y, bool y_bf16, int32_t* dev_status, bool weights_early,
-                          void* ws, const LoraArgs& lora, int codebook, const DeviceInfo& dev,
-                          cudaStream_t stream) {
+static cudaError_t linear_one(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
+                              const float* absmax_scale, const float* absmax_offset, int64_t n, int64_t k, void* Y,
+                              bool y_bf16, int32_t* dev_status, bool weights_early, void* ws, const LoraArgs& lora,
+                              int codebook, uint32_t test_flags, const DeviceInfo& dev, cudaStream_t stream) {
     if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
     if (m > kGemvMaxTokens)
         return launch_gemm(X, m, wq, absmax_q, absmax_scale, absmax_offset, n, k, Y, y_bf16, dev_status, lora,
-                           codebook, dev, stream);
+                           codebook, test_flags, dev, stream);
     CUtensorMap tm_w;
     cudaError_t e = tmap_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, static_cast<uint64_t>(k / 2),
                             static_cast<uint64_t>(n), static_cast<uint64_t>(k / 2), 128, gemv::kRows,
@@ -695,7 +711,33 @@ cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int
         if (e != cudaSuccess) return e;
         void* Yt = static_cast<char*>(Y) + static_cast<size_t>(t0) * n * ybytes;
         e = dispatch_gemv(y_bf16, mt > 8, lora.t != nullptr, tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt,
-                          n, k, cluster, weights_early, Yt, dev_status, ws, lora, codebook, dev.device, stream);
+                          n, k, cluster, weights_early, Yt, dev_status, ws, lora, codebook, test_flags, dev.device,
+                          stream);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
+                          const float* absmax_scale, const float* absmax_offset, int64_t n,
+                          int64_t k, void* Y, bool y_bf16, int32_t* dev_status, bool weights_early,
+                          void* ws, const LoraArgs& lora, int codebook, const DeviceInfo& dev,
+                          cudaStream_t stream) {
+    return linear_one(X, m, wq, absmax_q, absmax_scale, absmax_offset, n, k, Y, y_bf16, dev_status, weights_early,
+                      ws, lora, codebook, 0u, dev, stream);
+}
+
+// The weights of a group are launched one after the other on the stream (each
+// launch spreads its own tiles over every SM); one workspace serves them all,
+// since each launch leaves its counters at zero.
+cudaError_t launch_linear_group(const void* X, int64_t m, int64_t k, const LinearWeight* w, int count,
+                                bool y_bf16, int32_t* dev_status, bool weights_early, void* ws, const LoraArgs& lora,
+                                int codebook, uint32_t test_flags, const DeviceInfo& dev, cudaStream_t stream) {
+    if (count < 1 || count > kMaxGroup) return cudaErrorInvalidValue;
+    for (int i = 0; i < count; ++i) {
+        const cudaError_t e = linear_one(X, m, w[i].wq, w[i].absmax_q, w[i].absmax_scale, w[i].absmax_offset, w[i].n,
+                                         k, w[i].y, y_bf16, dev_status, weights_early, ws, lora, codebook, test_flags,
+                                         dev, stream);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -50,6 +50,30 @@ cudaError_t launch_dequantize(const uint8_t* wq, const int8_t* absmax_q, const f
 // Bytes of the split-k workspace the decode path needs for (m, n, k); 0 if none.
 size_t linear_workspace_bytes(int64_t m, int64_t n, int64_t k, const DeviceInfo& dev);
 
+// Weights one decode launch may serve together (they share X and k).
+constexpr int kMaxGroup = 4;
+
+// Test hook for the bounded waits: the kernel's copy producers issue nothing
+// and every wait gives up after a few polls, so the call ends with
+// NF4_ERR_DEVICE_TIMEOUT in dev_status and nothing left in flight.
+constexpr uint32_t kTestStall = 1u;
+
+// One weight of a (grouped) linear and the output it writes, Y [m, n].
+struct LinearWeight {
+    const uint8_t* wq = nullptr;
+    const int8_t* absmax_q = nullptr;
+    const float* absmax_scale = nullptr;
+    const float* absmax_offset = nullptr;
+    int64_t n = 0;
+    void* y = nullptr;
+};
+
+// Y_i = X * What_i^T for `count` (1 .. kMaxGroup) weights of the same k in one
+// launch (m <= kGemvMaxTokens); larger m runs the GEMM once per weight.
+cudaError_t launch_linear_group(const void* X, int64_t m, int64_t k, const LinearWeight* w, int count,
+                                bool y_bf16, int32_t* dev_status, bool weights_early, void* ws, const LoraArgs& lora,
+                                int codebook, uint32_t test_flags, const DeviceInfo& dev, cudaStream_t stream);
+
 // `ws` (nullable) must hold linear_workspace_bytes(m, n, k, dev) bytes, 16-byte aligned.
 cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                           const float* absmax_scale, const float* absmax_offset, int64_t n,
@@ -77,7 +101,7 @@ cudaError_t launch_gemm_dx(const void* dY, int64_t m, const uint8_t* wq, const i
 cudaError_t launch_gemm(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                         const float* absmax_scale, const float* absmax_offset, int64_t n, int64_t k, void* Y,
                         bool y_bf16, int32_t* dev_status, const LoraArgs& lora, int codebook,
-                        const DeviceInfo& dev, cudaStream_t stream);
+                        uint32_t test_flags, const DeviceInfo& dev, cudaStream_t stream);
 
 // Token counts up to this run the decode GEMV; larger ones the tcgen05 GEMM.
 constexpr int64_t kGemvMaxTokens = 16;

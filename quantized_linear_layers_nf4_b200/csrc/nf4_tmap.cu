@@ -33,14 +33,10 @@ struct Entry {
 
 }  // namespace
 
-cudaError_t tmap_2d(CUtensorMap* out, CUtensorMapDataType dtype, const void* base, uint64_t dim0,
-                    uint64_t dim1, uint64_t stride1, uint32_t box0, uint32_t box1,
-                    CUtensorMapSwizzle swizzle) {
+static cudaError_t tmap_nd(CUtensorMap* out, const TmapKey& key) {
     static std::mutex mu;
     static Entry cache[kCache];
     static int next = 0;
-    const TmapKey key{base, dim0, dim1, stride1, box0, box1, static_cast<int>(dtype),
-                      static_cast<int>(swizzle)};
     {
         std::lock_guard<std::mutex> lock(mu);
         for (int i = 0; i < kCache; ++i)
@@ -51,13 +47,14 @@ cudaError_t tmap_2d(CUtensorMap* out, CUtensorMapDataType dtype, const void* bas
     }
     auto fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
-    const cuuint64_t dims[2] = {dim0, dim1};
-    const cuuint64_t strides[1] = {stride1};
-    const cuuint32_t box[2] = {box0, box1};
-    const cuuint32_t estr[2] = {1, 1};
+    const cuuint64_t dims[3] = {key.dim0, key.dim1, key.dim2};
+    const cuuint64_t strides[2] = {key.stride1, key.stride2};
+    const cuuint32_t box[3] = {key.box0, key.box1, key.box2};
+    const cuuint32_t estr[3] = {1, 1, 1};
     CUtensorMap map;
-    const CUresult r = fn(&map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    const CUresult r = fn(&map, static_cast<CUtensorMapDataType>(key.dtype), static_cast<cuuint32_t>(key.rank),
+                          const_cast<void*>(key.base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          static_cast<CUtensorMapSwizzle>(key.swizzle), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     std::lock_guard<std::mutex> lock(mu);
@@ -67,6 +64,14 @@ cudaError_t tmap_2d(CUtensorMap* out, CUtensorMapDataType dtype, const void* bas
     next = (next + 1) % kCache;
     *out = map;
     return cudaSuccess;
+}
+
+cudaError_t tmap_2d(CUtensorMap* out, CUtensorMapDataType dtype, const void* base, uint64_t dim0,
+                    uint64_t dim1, uint64_t stride1, uint32_t box0, uint32_t box1,
+                    CUtensorMapSwizzle swizzle) {
+    const TmapKey key{base, dim0, dim1, 1, stride1, 0, box0, box1, 1, 2, static_cast<int>(dtype),
+                      static_cast<int>(swizzle)};
+    return tmap_nd(out, key);
 }
 
 }  // namespace nf4

@@ -13,12 +13,13 @@ namespace nf4 {
 
 struct TmapKey {
     const void* base;
-    uint64_t dim0, dim1, stride1;
-    uint32_t box0, box1;
-    int dtype, swizzle;
+    uint64_t dim0, dim1, dim2, stride1, stride2;
+    uint32_t box0, box1, box2;
+    int rank, dtype, swizzle;
     bool operator==(const TmapKey& o) const {
-        return base == o.base && dim0 == o.dim0 && dim1 == o.dim1 && stride1 == o.stride1 &&
-               box0 == o.box0 && box1 == o.box1 && dtype == o.dtype && swizzle == o.swizzle;
+        return base == o.base && dim0 == o.dim0 && dim1 == o.dim1 && dim2 == o.dim2 && stride1 == o.stride1 &&
+               stride2 == o.stride2 && box0 == o.box0 && box1 == o.box1 && box2 == o.box2 && rank == o.rank &&
+               dtype == o.dtype && swizzle == o.swizzle;
     }
 };
 

@@ -201,15 +201,21 @@ def test_gemv_three_way_split_k(nf4, m):
     _check_linear(nf4, X, weight, orc)
 
 
+def _same_bits(a: torch.Tensor, b: torch.Tensor) -> bool:
+    return torch.equal(a.view(torch.int16) if a.dtype == torch.bfloat16 else a.view(torch.int32),
+                       b.view(torch.int16) if b.dtype == torch.bfloat16 else b.view(torch.int32))
+
+
 @pytest.mark.parametrize("n,k,m", [(4096, 4096, 16), (11008, 4096, 16), (11000, 2304, 3), (1000, 1024, 7),
-                                   (4096, 11008, 1), (300, 576, 16), (64, 128, 5)])
+                                   (4096, 11008, 1), (300, 576, 16), (64, 128, 5), (128, 64, 1),
+                                   (2048, 640, 9), (19000, 4096, 16)])
 def test_workspace_split_k_is_bit_identical(nf4, n, k, m):
     """nf4_linear_ws with a workspace (CTAs meet in global memory, the last one
-    reduces) gives the same bits as the cluster path, for split-k factors
-    1, 2, 3, 4 and 8, and leaves every counter at zero."""
+    reduces) gives the same bits as the cluster path, for split-k factors 1 to
+    8, leaves every counter at zero and matches the oracle on sampled rows."""
     W = synth.weight_normal(n, k, seed=1200 + n + k, dtype=torch.bfloat16, device="cuda")
     X = synth.activations(m, k, seed=1300 + m, device="cuda")
-    weight = nf4.quantize_weight(W)
+    weight, orc = _check_quant(nf4, W, full_dequant=False, rows=[0, n - 1])
     nb = nf4.nf4_linear_workspace_bytes(m, n, k)
     ws = nf4.linear_workspace([(n, k)], m=m)
     ds = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -218,12 +224,12 @@ def test_workspace_split_k_is_bit_identical(nf4, n, k, m):
         for _ in range(2):   # twice: the counters must have been reset by the first call
             got = nf4.nf4_linear(X, weight, dtype, workspace=ws, dev_status=ds)
             torch.cuda.synchronize()
-            assert torch.equal(got.view(torch.int16) if dtype == torch.bfloat16 else got.view(torch.int32),
-                               ref.view(torch.int16) if dtype == torch.bfloat16 else ref.view(torch.int32))
+            assert _same_bits(got, ref)
     tiles = (n + 127) // 128
     if nb:
         assert int(ws[: 4 * tiles].view(torch.int32).abs().sum()) == 0, "split-k counters not reset"
     assert ds.item() == 0
+    _check_linear(nf4, X, weight, orc, weight_rows=_sample_rows(n, 64, n + k))
 
 
 def test_workspace_errors_and_graph_reuse(nf4):
@@ -511,6 +517,68 @@ def test_weights_early_launch_gives_identical_results(nf4):
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(a, b) and torch.equal(a, c)
+
+
+@pytest.mark.parametrize("m", [1, 16])
+def test_linear_group_matches_single_launches(nf4, m):
+    """Weights that share X (q/k/v-like and gate/up-like) in one nf4_linear_group
+    call: with and without a workspace, each output has the bits of nf4_linear
+    on that weight alone, and the oracle is matched on sampled rows."""
+    k = 2048
+    shapes = [(2048, k), (512, k), (512, k)]
+    Ws = [synth.weight_normal(n, k, seed=2100 + i, dtype=torch.bfloat16, device="cuda") for i, (n, _) in enumerate(shapes)]
+    X = synth.activations(m, k, seed=2110 + m, device="cuda")
+    checked = [_check_quant(nf4, W, full_dequant=False, rows=[0, W.shape[0] - 1]) for W in Ws]
+    weights = [wo[0] for wo in checked]
+    ws = nf4.linear_workspace(shapes, m=m)
+    for dtype in (torch.float32, torch.bfloat16):
+        singles = [nf4.nf4_linear(X, w, dtype) for w in weights]
+        with_ws = nf4.nf4_linear_group(X, weights, dtype, workspace=ws)
+        without = nf4.nf4_linear_group(X, weights, dtype)
+        torch.cuda.synchronize()
+        for a, b, s1 in zip(with_ws, without, singles):
+            assert _same_bits(a, s1) and _same_bits(b, s1), "grouped vs single launch"
+    for (weight, orc), (n, _) in zip(checked, shapes):
+        _check_linear(nf4, X, weight, orc, weight_rows=_sample_rows(n, 96, n))
+    # two weights (gate/up-like), the bench's layout
+    gu = [nf4.quantize_weight(synth.weight_normal(1408, k, seed=2120 + i, dtype=torch.bfloat16, device="cuda"))
+          for i in range(2)]
+    outs = nf4.nf4_linear_group(X, gu, torch.float32, workspace=ws, weights_early=True)
+    for a, w in zip(outs, gu):
+        assert _same_bits(a, nf4.nf4_linear(X, w, torch.float32))
+    with pytest.raises(nf4.NF4Error):  # different k
+        nf4.nf4_linear_group(X, [weights[0], nf4.quantize_weight(Ws[0][:, :1024].contiguous())])
+    with pytest.raises(nf4.NF4Error):  # too many weights
+        nf4.nf4_linear_group(X, weights + weights)
+
+
+@pytest.mark.parametrize("m,n,k", [(16, 4096, 4096), (3, 300, 576), (64, 512, 1024)])
+def test_bounded_wait_timeout_path(nf4, m, n, k):
+    """NF4_LINEAR_TEST_TIMEOUT: the copy producers issue nothing and every device
+    wait gives up after a few polls.  The call must end with NF4_ERR_DEVICE_TIMEOUT
+    in dev_status, leave Y and the workspace untouched (the GEMM frees its tensor memory) and
+    leave the stream usable: the next ordinary call is correct.  m = 64 runs the
+    tcgen05 GEMM's timeout branches, m <= 16 the GEMV's."""
+    W = synth.weight_normal(n, k, seed=2200 + n, dtype=torch.bfloat16, device="cuda")
+    X = synth.activations(m, k, seed=2201 + m, device="cuda")
+    weight = nf4.quantize_weight(W)
+    ws = nf4.linear_workspace([(n, k)], m=m)
+    for wsp in (ws, None):
+        ref = nf4.nf4_linear(X, weight, torch.float32, workspace=wsp)
+        ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+        y = torch.full((m, n), 7.0, dtype=torch.float32, device="cuda")
+        before = ws.clone()
+        nf4.nf4_linear(X, weight, torch.float32, out=y, dev_status=ds, workspace=wsp,
+                       flags=nf4._lib.NF4_LINEAR_TEST_TIMEOUT)
+        torch.cuda.synchronize()
+        assert int(ds.item()) == nf4._lib.NF4_ERR_DEVICE_TIMEOUT
+        assert bool((y == 7.0).all()), "a timed-out call wrote Y"
+        assert torch.equal(ws, before), "a timed-out call touched the workspace"
+        ds.zero_()
+        again = nf4.nf4_linear(X, weight, torch.float32, dev_status=ds, workspace=wsp)
+        torch.cuda.synchronize()
+        assert int(ds.item()) == 0
+        assert torch.equal(again, ref)
 
 
 def test_dev_status_stays_clear(nf4):
