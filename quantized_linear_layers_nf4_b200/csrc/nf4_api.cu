@@ -192,7 +192,8 @@ nf4_status_t nf4_linear_lora(const void* X, int64_t m, const nf4_weight_t* w, co
     float* t = static_cast<float*>(workspace);
     __nv_bfloat16* t_hi = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(workspace) + lora_t_region(m, r, 4));
     __nv_bfloat16* t_lo = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<char*>(t_hi) + lora_t_region(m, r, 2));
-    st = from_cuda(nf4::launch_lora_down(X, m, w->k, lora_down, r, scale, t, t_hi, t_lo, s));
+    st = from_cuda(nf4::launch_lora_down(X, m, w->k, lora_down, r, scale, t, t_hi, t_lo,
+                                         (flags & NF4_LINEAR_WEIGHTS_EARLY) != 0, s));
     if (st != NF4_OK) return st;
     nf4::LoraArgs lora;
     lora.t = t;

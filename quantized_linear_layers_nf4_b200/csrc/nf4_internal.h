@@ -83,8 +83,10 @@ cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int
 
 // t[m, r] = scale * X[m, k] down[r, k]^T in fp32 (fixed order); also its two bf16
 // halves when t_hi / t_lo are given.
+// With `early`, launched as a programmatic dependent of the preceding kernel
+// (it waits for it before reading X) and letting the next kernel start at once.
 cudaError_t launch_lora_down(const void* X, int64_t m, int64_t k, const void* down, int r, float scale, float* t,
-                             __nv_bfloat16* t_hi, __nv_bfloat16* t_lo, cudaStream_t stream);
+                             __nv_bfloat16* t_hi, __nv_bfloat16* t_lo, bool early, cudaStream_t stream);
 
 // Merge a LoRA update into the quantized weight and requantize: w_new (bf16
 // [n, k], may be null), wq_out [n*k/2] and absmax_out [n*k/64] fp32.

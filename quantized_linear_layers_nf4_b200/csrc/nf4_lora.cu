@@ -14,55 +14,74 @@
 
 #include "nf4_common.cuh"
 #include "nf4_internal.h"
+#include "nf4_ptx.cuh"
 
 namespace nf4 {
 namespace lora {
 
+// t[tok, j] = scale * sum_c X[tok, c] * down[j, c] in fp32.  CTA (token, pair of
+// ranks): warp w computes rank 2 * blockIdx.y + w / 4 over the k quarter w % 4;
+// within a quarter lane l sums the 8-element chunks l, l + 32, ... into two
+// accumulators (even and odd chunk rounds), and the quarters are added in
+// order (q0 + q1) + (q2 + q3).  Under a programmatic dependent launch the next
+// kernel (the dequant-GEMV, which prefetches its weights) may start at once;
+// X may be the preceding kernel's output, so it is read after the wait.
 __global__ void __launch_bounds__(256) k_lora_down(const __nv_bfloat16* __restrict__ X, int64_t k,
                                                    const __nv_bfloat16* __restrict__ down, int r, float scale,
                                                    float* __restrict__ t, __nv_bfloat16* __restrict__ t_hi,
                                                    __nv_bfloat16* __restrict__ t_lo) {
-    // block (token, group of 8 ranks); warp w computes rank 8 * blockIdx.y + w
+    __shared__ float part[2][4];
+    grid_launch_dependents();
+    grid_dependency_wait();
     const int64_t tok = blockIdx.x;
-    const int j = static_cast<int>(blockIdx.y) * 8 + (threadIdx.x >> 5);
+    const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    if (j >= r) return;
-    const __nv_bfloat16* x = X + tok * k;
-    const __nv_bfloat16* d = down + static_cast<int64_t>(j) * k;
-    // lane l sums the 8-element chunks l, l + 32, l + 64, ...; chunk i goes to
-    // accumulator i mod 4 (four loads in flight), combined in a fixed order
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const int j = static_cast<int>(blockIdx.y) * 2 + (warp >> 2);
+    const int quarter = warp & 3;
     const int64_t nch = k / 8;
-    for (int64_t base = lane; base < nch; base += 128) {
+    const int64_t c0 = nch * quarter / 4, c1 = nch * (quarter + 1) / 4;
+    float v = 0.0f;
+    if (j < r) {
+        const __nv_bfloat16* x = X + tok * k;
+        const __nv_bfloat16* d = down + static_cast<int64_t>(j) * k;
+        float acc[2] = {0.0f, 0.0f};
+        for (int64_t base = c0 + lane; base < c1; base += 64) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int64_t ch = base + 32 * q;
-            if (ch < nch) {
-                const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + ch * 8));
-                const uint4 dv = __ldg(reinterpret_cast<const uint4*>(d + ch * 8));
-                const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, dw[4] = {dv.x, dv.y, dv.z, dv.w};
+            for (int q = 0; q < 2; ++q) {
+                const int64_t ch = base + 32 * q;
+                if (ch < c1) {
+                    const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + ch * 8));
+                    const uint4 dv = __ldg(reinterpret_cast<const uint4*>(d + ch * 8));
+                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, dw[4] = {dv.x, dv.y, dv.z, dv.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    acc[q] = __fmaf_rn(bf16_bits_to_float(xw[e] & 0xffffu), bf16_bits_to_float(dw[e] & 0xffffu), acc[q]);
-                    acc[q] = __fmaf_rn(bf16_bits_to_float(xw[e] >> 16), bf16_bits_to_float(dw[e] >> 16), acc[q]);
+                    for (int e = 0; e < 4; ++e) {
+                        acc[q] = __fmaf_rn(bf16_bits_to_float(xw[e] & 0xffffu), bf16_bits_to_float(dw[e] & 0xffffu),
+                                           acc[q]);
+                        acc[q] = __fmaf_rn(bf16_bits_to_float(xw[e] >> 16), bf16_bits_to_float(dw[e] >> 16), acc[q]);
+                    }
                 }
             }
         }
-    }
-    float v = __fadd_rn(__fadd_rn(acc[0], acc[1]), __fadd_rn(acc[2], acc[3]));
+        v = __fadd_rn(acc[0], acc[1]);
 #pragma unroll
-    for (int h = 16; h >= 1; h >>= 1) v = __fadd_rn(v, __shfl_xor_sync(kFull, v, h));
-    if (lane == 0) {
-        const float tv = __fmul_rn(v, scale);
-        t[tok * r + j] = tv;
-        if (t_hi) {
-            const __nv_bfloat16 h = __float2bfloat16_rn(tv);
-            t_hi[tok * r + j] = h;
-            t_lo[tok * r + j] = __float2bfloat16_rn(__fsub_rn(tv, __bfloat162float(h)));
+        for (int h = 16; h >= 1; h >>= 1) v = __fadd_rn(v, __shfl_xor_sync(kFull, v, h));
+    }
+    if (lane == 0) part[warp >> 2][quarter] = v;
+    __syncthreads();
+    if (threadIdx.x < 2) {
+        const int jj = static_cast<int>(blockIdx.y) * 2 + threadIdx.x;
+        if (jj < r) {
+            const float* pq = part[threadIdx.x];
+            const float tv = __fmul_rn(__fadd_rn(__fadd_rn(pq[0], pq[1]), __fadd_rn(pq[2], pq[3])), scale);
+            t[tok * r + jj] = tv;
+            if (t_hi) {
+                const __nv_bfloat16 h = __float2bfloat16_rn(tv);
+                t_hi[tok * r + jj] = h;
+                t_lo[tok * r + jj] = __float2bfloat16_rn(__fsub_rn(tv, __bfloat162float(h)));
+            }
         }
     }
 }
-
 
 // ---------------------------------------------------------------------------
 // Merge + requantize (page "LLM 相關知識" (technicalnotes), section "8. LoRA 的
@@ -165,12 +184,18 @@ __global__ void __launch_bounds__(256) k_nf4_merge_lora(const uint32_t* __restri
 }  // namespace lora
 
 cudaError_t launch_lora_down(const void* X, int64_t m, int64_t k, const void* down, int r, float scale, float* t,
-                             __nv_bfloat16* t_hi, __nv_bfloat16* t_lo, cudaStream_t stream) {
-    const dim3 grid(static_cast<unsigned>(m), static_cast<unsigned>((r + 7) / 8));
-    lora::k_lora_down<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), k,
-                                                                      static_cast<const __nv_bfloat16*>(down), r,
-                                                                      scale, t, t_hi, t_lo);
-    return cudaGetLastError();
+                             __nv_bfloat16* t_hi, __nv_bfloat16* t_lo, bool early, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(m), static_cast<unsigned>((r + 1) / 2), 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = early ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, lora::k_lora_down, static_cast<const __nv_bfloat16*>(X), k,
+                              static_cast<const __nv_bfloat16*>(down), r, scale, t, t_hi, t_lo);
 }
 
 cudaError_t launch_merge_lora(const uint8_t* wq, const int8_t* absmax_q, const float* absmax_scale,
