@@ -6,9 +6,11 @@
 // base is dequantized in forward and backward.
 //
 // HBM-bound: reads 0.5 B/param of codes (+1 B per 64 of absmax codes) and
-// writes 2 (bf16) or 4 (fp32) B/param.  Each lane decodes one 32-bit word of
-// codes (8 elements) with the 16 levels held in shared memory and writes 16 or
-// 32 bytes with 128-bit stores.
+// writes 2 (bf16) or 4 (fp32) B/param.  Each lane decodes 32-bit words of codes
+// (8 elements each) with the 16 levels held in shared memory and writes 16 or
+// 32 bytes per word with 128-bit stores; a warp takes four words per lane per
+// pass (a warp's loads and stores stay contiguous) with all four loads issued
+// before the first decode.
 #include "nf4_common.cuh"
 #include "nf4_internal.h"
 
@@ -25,30 +27,46 @@ __global__ void __launch_bounds__(256) k_nf4_dequantize(const uint32_t* __restri
     if (threadIdx.x < 16) lv[threadIdx.x] = kCodebook[codebook][threadIdx.x];
     __syncthreads();
     const float mu = __ldg(mu_ptr);
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < n_groups;
-         g += stride) {
-        const uint32_t packed = __ldcs(wq32 + g);
-        const int64_t b = g >> 3;  // 64-element block
-        const float a = absmax_hat(__ldg(absmax_q + b), __ldg(absmax_scale + (b >> 8)), mu);
-        float v[8];
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    constexpr int kUnroll = 4;
+    // a pass of a warp: words base + 32 q + lane, q = 0 .. 3 (128 consecutive
+    // words, all loads issued before the first decode)
+    for (int64_t base = warp * 32 * kUnroll; base < n_groups; base += n_warps * 32 * kUnroll) {
+        uint32_t packed[kUnroll];
+        float a[kUnroll];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t byte = (packed >> (8 * i)) & 0xffu;
-            v[2 * i] = __fmul_rn(lv[byte >> 4], a);        // element 2i: high nibble
-            v[2 * i + 1] = __fmul_rn(lv[byte & 15u], a);
+        for (int q = 0; q < kUnroll; ++q) {
+            const int64_t g = base + 32 * q + lane;
+            const int64_t gg = g < n_groups ? g : base;      // a valid word (base always is)
+            packed[q] = __ldcs(wq32 + gg);
+            const int64_t b = gg >> 3;                       // 64-element block
+            a[q] = absmax_hat(__ldg(absmax_q + b), __ldg(absmax_scale + (b >> 8)), mu);
         }
-        if (kBf16Out) {
-            uint4 o;
-            o.x = pack_bf16x2(v[0], v[1]);
-            o.y = pack_bf16x2(v[2], v[3]);
-            o.z = pack_bf16x2(v[4], v[5]);
-            o.w = pack_bf16x2(v[6], v[7]);
-            __stcs(reinterpret_cast<uint4*>(out) + g, o);
-        } else {
-            float4* o = reinterpret_cast<float4*>(out) + 2 * g;
-            __stcs(o, make_float4(v[0], v[1], v[2], v[3]));
-            __stcs(o + 1, make_float4(v[4], v[5], v[6], v[7]));
+#pragma unroll
+        for (int q = 0; q < kUnroll; ++q) {
+            const int64_t g = base + 32 * q + lane;
+            if (g >= n_groups) break;
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t byte = (packed[q] >> (8 * i)) & 0xffu;
+                v[2 * i] = __fmul_rn(lv[byte >> 4], a[q]);        // element 2i: high nibble
+                v[2 * i + 1] = __fmul_rn(lv[byte & 15u], a[q]);
+            }
+            if (kBf16Out) {
+                uint4 o;
+                o.x = pack_bf16x2(v[0], v[1]);
+                o.y = pack_bf16x2(v[2], v[3]);
+                o.z = pack_bf16x2(v[4], v[5]);
+                o.w = pack_bf16x2(v[6], v[7]);
+                __stcs(reinterpret_cast<uint4*>(out) + g, o);
+            } else {
+                float4* o = reinterpret_cast<float4*>(out) + 2 * g;
+                __stcs(o, make_float4(v[0], v[1], v[2], v[3]));
+                __stcs(o + 1, make_float4(v[4], v[5], v[6], v[7]));
+            }
         }
     }
 }
@@ -57,7 +75,7 @@ cudaError_t launch_dequantize(const uint8_t* wq, const int8_t* absmax_q, const f
                               const float* absmax_offset, int64_t n_elem, void* out, bool out_bf16, int codebook,
                               const DeviceInfo& dev, cudaStream_t stream) {
     const int64_t n_groups = n_elem / 8;
-    int64_t blocks = (n_groups + 255) / 256;
+    int64_t blocks = (n_groups + 1023) / 1024;
     const int64_t cap = static_cast<int64_t>(dev.sm_count) * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;

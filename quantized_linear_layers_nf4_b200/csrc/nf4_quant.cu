@@ -11,9 +11,9 @@
 // Both kernels are HBM-bound streams.  Quantization reads the weight once
 // (2 or 4 B/param) and writes 0.5 B/param of codes plus 4 B per 64 params of
 // absmax: 128-bit loads, 8 lanes per 64-block, a 3-step xor-shuffle absmax and
-// one packed 32-bit store per lane.  Double quantization is three small
-// launches: per-256 fp64 partial sums, a one-CTA fixed-order reduction to the
-// mean, and the int8 encode.
+// one packed 32-bit store per lane.  Double quantization is two small
+// launches: per-256 fp64 partial sums, then the int8 encode, whose CTAs each
+// finish the mean's fixed-order reduction from the partial sums first.
 #include "nf4_common.cuh"
 #include "nf4_internal.h"
 
@@ -41,40 +41,114 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* __restrict__ W, int64
     }
 }
 
+// The code of each element without a division and without a search.
+//
+// Quotient: q = RN(w / a) by Markstein's correction of a product with the
+// correctly rounded reciprocal (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
+// 1990): with r = RN(1 / a), q0 = RN(w r), e = w - a q0 (exact, one FMA) and
+// q = RN(q0 + e r) is the IEEE quotient when nothing leaves the normal range.
+// It is used for blocks whose absmax lies in [2^-60, 2^60]; for them every
+// quotient that can reach a threshold (|q| >= 2^-8, far inside the band that
+// maps to the zero level) keeps e exact.  Other blocks (zero, tiny, huge or
+// non-finite absmax) divide.
+//
+// NF4 code of q in [-1, 1]: bucket b = round_half_even(128 q + 128) (one FMA
+// onto the mantissa of 1.5 * 2^23) of a 257-entry table; at most one threshold
+// falls in the closed q range of a bucket (NF4 thresholds are more than 1/128
+// apart), so idx = base[b] + (q > thr[b]) with base[b] = #{j : t_j below the
+// bucket}.  The table lives in shared memory, 16 copies so the 16 lanes of a
+// half-warp never share a bank.
+constexpr int kBuckets = 257;
+constexpr int kTabCopies = 16;
+constexpr float kBucketMagic = 12582912.0f + 128.0f;  // 1.5 * 2^23 + 128
+
+__device__ __forceinline__ float quotient(float w, float a, float r) {
+    const float q0 = __fmul_rn(w, r);
+    const float e = __fmaf_rn(-q0, a, w);
+    return __fmaf_rn(e, r, q0);
+}
+
+__device__ __forceinline__ bool markstein_ok(float a) {
+    return a >= 0x1p-60f && a <= 0x1p60f;  // false for 0, NaN and +inf too
+}
+
 template <typename T, int CB>
 __global__ void __launch_bounds__(256) k_nf4_quantize(const T* __restrict__ W, int64_t n_groups,
                                                       uint32_t* __restrict__ wq32,
                                                       float* __restrict__ absmax) {
+    __shared__ uint2 tab[CB == kCbNf4 ? kBuckets * kTabCopies : 1];
+    if (CB == kCbNf4) {
+        for (int e = threadIdx.x; e < kBuckets * kTabCopies; e += blockDim.x) {
+            const int b = e / kTabCopies;
+            const float lo = (static_cast<float>(b) - 0.5f) / 128.0f - 1.0f;
+            const float hi = (static_cast<float>(b) + 0.5f) / 128.0f - 1.0f;
+            uint32_t base = 0;
+            float thr = __int_as_float(0x7f800000);  // +inf: no threshold in the bucket
+#pragma unroll
+            for (int j = 0; j < 15; ++j) {
+                const float t = kThresh[j];
+                if (t < lo) ++base;
+                else if (t <= hi) thr = t;
+            }
+            tab[e] = make_uint2(__float_as_uint(thr), base);
+        }
+        __syncthreads();
+    }
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     const int64_t n_chunks = (n_groups + 31) >> 5;
-    for (int64_t chunk = warp; chunk < n_chunks; chunk += n_warps) {
-        const int64_t g = (chunk << 5) + lane;          // group of 8 elements
-        const bool valid = g < n_groups;                 // whole 8-lane blocks agree
-        float w[8];
-        if (valid) {
-            load8(W, g * 8, w);
-        } else {
+    // a warp takes kUnroll chunks per pass (chunk = 256 contiguous elements):
+    // all their loads go out before any of them is encoded
+    constexpr int kUnroll = 4;
+    for (int64_t c0 = warp; c0 < n_chunks; c0 += n_warps * kUnroll) {
+        float w[kUnroll][8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) w[j] = 0.0f;
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t g = ((c0 + u * n_warps) << 5) + lane;  // group of 8 elements
+            if (g < n_groups) {
+                load8(W, g * 8, w[u]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) w[u][j] = 0.0f;
+            }
         }
-        float a = 0.0f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) a = fmaxf(a, fabsf(w[j]));
-        a = fmaxf(a, __shfl_xor_sync(kFull, a, 1));
-        a = fmaxf(a, __shfl_xor_sync(kFull, a, 2));
-        a = fmaxf(a, __shfl_xor_sync(kFull, a, 4));
-        uint32_t packed = 0;
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t g = ((c0 + u * n_warps) << 5) + lane;
+            const bool valid = g < n_groups;                 // whole 8-lane blocks agree
+            float a = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t hi = static_cast<uint32_t>(quantize_code<CB>(w[2 * i], a));
-            const uint32_t lo = static_cast<uint32_t>(quantize_code<CB>(w[2 * i + 1], a));
-            packed |= ((hi << 4) | lo) << (8 * i);      // element 2i in the high nibble
-        }
-        if (valid) {
-            wq32[g] = packed;
-            if ((lane & 7) == 0) absmax[g >> 3] = a;
+            for (int j = 0; j < 8; ++j) a = fmaxf(a, fabsf(w[u][j]));
+            a = fmaxf(a, __shfl_xor_sync(kFull, a, 1));
+            a = fmaxf(a, __shfl_xor_sync(kFull, a, 2));
+            a = fmaxf(a, __shfl_xor_sync(kFull, a, 4));
+            uint32_t code[8];
+            if (markstein_ok(a)) {
+                const float r = __frcp_rn(a);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float q = quotient(w[u][j], a, r);
+                    if (CB == kCbNf4) {
+                        const uint32_t b = __float_as_uint(__fmaf_rn(q, 128.0f, kBucketMagic)) & 0x1ffu;
+                        const uint2 ent = tab[b * kTabCopies + (threadIdx.x & 15)];
+                        code[j] = ent.y + (q > __uint_as_float(ent.x) ? 1u : 0u);
+                    } else {
+                        code[j] = static_cast<uint32_t>(encode_fp4(q));
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) code[j] = static_cast<uint32_t>(quantize_code<CB>(w[u][j], a));
+            }
+            uint32_t packed = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) packed |= ((code[2 * i] << 4) | code[2 * i + 1]) << (8 * i);  // element 2i high
+            if (valid) {
+                wq32[g] = packed;
+                if ((lane & 7) == 0) absmax[g >> 3] = a;
+            }
         }
     }
 }
@@ -95,7 +169,9 @@ cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n_elem, uint8_t*
     const int64_t n_groups = n_elem / 8;
     const int64_t n_chunks = (n_groups + 31) / 32;
     int64_t blocks = (n_chunks + 7) / 8;
-    const int64_t cap = static_cast<int64_t>(dev.sm_count) * 8;
+    // one wave of CTAs that stay resident (four per SM by their registers) and
+    // walk the chunks with a grid stride
+    const int64_t cap = static_cast<int64_t>(dev.sm_count) * 4;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     if (codebook == kCbFp4)
@@ -148,7 +224,6 @@ __global__ void __launch_bounds__(256) k_dq_partials(const float* __restrict__ a
     }
 }
 
-constexpr int kMeanThreads = 1024;
 constexpr int kMeanLevel2 = 4096;  // max chunks after the first reduction (shared memory)
 
 int64_t dq_max_nb() { return static_cast<int64_t>(256) * 256 * kMeanLevel2; }
@@ -159,15 +234,17 @@ size_t dq_workspace_bytes(int64_t nb) {
     return static_cast<size_t>(nb2) * sizeof(double);
 }
 
-// Remaining levels, one CTA: mu = fp32(S / nb).
-__global__ void __launch_bounds__(kMeanThreads) k_dq_mean(const double* __restrict__ partials,
-                                                          int64_t nb2, int64_t nb,
-                                                          float* __restrict__ mu_out) {
-    __shared__ double buf_a[kMeanLevel2];
-    __shared__ double buf_b[kMeanLevel2 / 256 + 1];
+// The remaining levels of the mean's tree over the nb2 chunk sums, by one CTA
+// of `kEncodeThreads` threads: S, then mu = fp32(S / nb).  Every encode CTA
+// does this for itself (the same adds in the same order, so every CTA gets the
+// same bits), which saves a launch between the two passes.
+constexpr int kEncodeThreads = 256;
+
+__device__ float cta_mean(const double* __restrict__ partials, int64_t nb2, int64_t nb, double* buf_a,
+                          double* buf_b) {
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    const int n_warps = kMeanThreads / 32;
+    const int n_warps = kEncodeThreads / 32;
     const double* src = partials;
     double* dst = buf_a;
     int64_t n = nb2;
@@ -188,21 +265,23 @@ __global__ void __launch_bounds__(kMeanThreads) k_dq_mean(const double* __restri
         dst = (dst == buf_a) ? buf_b : buf_a;
         n = m;
     }
-    if (threadIdx.x == 0) {
-        const double S = src[0];
-        *mu_out = __double2float_rn(__ddiv_rn(S, static_cast<double>(nb)));
-    }
+    return __double2float_rn(__ddiv_rn(src[0], static_cast<double>(nb)));
 }
 
-// Encode: one warp per block of 256 absmax values.
-__global__ void __launch_bounds__(256) k_dq_encode(const float* __restrict__ absmax, int64_t nb,
-                                                   int64_t nb2, const float* __restrict__ mu_ptr,
-                                                   int8_t* __restrict__ absmax_q,
-                                                   float* __restrict__ absmax_scale) {
+// Encode: the mean (above), then one warp per block of 256 absmax values.
+// CTA 0 writes the mean.
+__global__ void __launch_bounds__(kEncodeThreads) k_dq_encode(const float* __restrict__ absmax, int64_t nb,
+                                                              int64_t nb2, const double* __restrict__ partials,
+                                                              float* __restrict__ mu_out,
+                                                              int8_t* __restrict__ absmax_q,
+                                                              float* __restrict__ absmax_scale) {
+    __shared__ double buf_a[kMeanLevel2];
+    __shared__ double buf_b[kMeanLevel2 / 256 + 1];
+    const float mu = cta_mean(partials, nb2, nb, buf_a, buf_b);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *mu_out = mu;
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    const float mu = __ldg(mu_ptr);
     for (int64_t c = warp; c < nb2; c += n_warps) {
         float r[8];
         float s = 0.0f;
@@ -236,9 +315,9 @@ cudaError_t launch_double_quant(const float* absmax, int64_t nb, double* workspa
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     k_dq_partials<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(absmax, nb, workspace, nb2);
-    k_dq_mean<<<1, kMeanThreads, 0, stream>>>(workspace, nb2, nb, absmax_offset);
-    k_dq_encode<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(absmax, nb, nb2, absmax_offset,
-                                                                    absmax_q, absmax_scale);
+    k_dq_encode<<<static_cast<unsigned>(blocks), kEncodeThreads, 0, stream>>>(absmax, nb, nb2, workspace,
+                                                                               absmax_offset, absmax_q,
+                                                                               absmax_scale);
     return cudaGetLastError();
 }
 

@@ -153,6 +153,36 @@ def test_edge_values(nf4):
     _check_quant(nf4, W)
 
 
+@pytest.mark.parametrize("quant_type", ["nf4", "fp4"])
+def test_quantize_near_thresholds(nf4, quant_type):
+    """Codes of weights within a few ulps of every decision boundary (w / a at and
+    around each midpoint between adjacent levels), for absmax values inside and
+    outside the range where the quotient is formed without a division: bit-exact
+    against the oracle's IEEE division and nearest-level search."""
+    lv = O.codebook(quant_type).astype(np.float64)
+    mids = (lv[:-1] + lv[1:]) / 2
+    rows = []
+    for a in (1.0, 0.37, 3.1e-5, 1234.5, 2.0 ** -59, 2.0 ** 59, 2.0 ** -61, 2.0 ** 61, 0.0123456):
+        a32 = np.float32(a)
+        vals = [a32]
+        for c in mids:
+            x = np.float32(c * float(a32))
+            for d in range(-3, 4):
+                y = x
+                step = np.float32(np.inf) if d > 0 else np.float32(-np.inf)
+                for _ in range(abs(d)):
+                    y = np.nextafter(y, step)
+                if abs(float(y)) <= float(a32):
+                    vals.append(y)
+        vals = np.array(vals, dtype=np.float32)
+        vals = np.concatenate([vals, np.zeros((-len(vals)) % 64, np.float32)])
+        for i in range(0, len(vals), 63):   # every block starts with a (its absmax)
+            blk = np.concatenate([[a32], vals[i:i + 63]]).astype(np.float32)
+            rows.append(np.concatenate([blk, np.zeros(64 - len(blk), np.float32)]))
+    W = torch.from_numpy(np.concatenate(rows).reshape(-1, 256 if len(rows) % 4 == 0 else 64)).cuda()
+    _check_quant(nf4, W, quant_type=quant_type)
+
+
 def test_cfg1_full_chain_and_linear(nf4):
     """1024 x 1024 fp32 weight (seed 0), X 16 x 1024 bf16 (seed 1): everything
     checked on the whole output."""
