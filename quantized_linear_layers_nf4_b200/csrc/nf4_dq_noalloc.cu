@@ -17,6 +17,8 @@
 // are never used.
 #include <mutex>
 
+#include <cuda.h>
+
 #include "nf4.h"
 #include "nf4_internal.h"
 
@@ -26,23 +28,57 @@ constexpr int64_t kMaxPartials = NF4_DQ_NOALLOC_MAX_NB / 256;
 
 // File-scope scratch for the fp64 per-256 partial sums.  In host code this name
 // is only a stand-in for the device symbol: its device address comes from
-// cudaGetSymbolAddress, once per device.
+// cudaGetSymbolAddress, once per context.
 static __device__ __align__(256) double g_dq_partials[kMaxPartials];
 
-// Device address of g_dq_partials for the current device, looked up on the
-// first call with that device current.
-cudaError_t scratch_address(int device, double** out) {
-    static std::mutex mu;
-    static double* addr[64] = {};
-    if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(mu);
-    if (addr[device] == nullptr) {
+// Device address of g_dq_partials in the current context.  Each context (a
+// device's primary context, or one the caller created) has its own copy of the
+// module, so the address is cached per context, looked up the first time a
+// context makes the call.  The context comes from cuCtxGetCurrent, fetched
+// through the runtime's driver entry point (no link-time driver dependency);
+// without it the address is looked up on every call.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
         void* p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_dq_partials);
-        if (e != cudaSuccess) return e;
-        addr[device] = static_cast<double*>(p);
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+cudaError_t scratch_address(double** out) {
+    constexpr int kSlots = 64;
+    static std::mutex mu;
+    static CUcontext ctx_of[kSlots] = {};
+    static double* addr_of[kSlots] = {};
+    static int used = 0;
+    CUcontext ctx = nullptr;
+    const CtxGetCurrentFn get = ctx_get_current();
+    const bool keyed = get != nullptr && get(&ctx) == CUDA_SUCCESS && ctx != nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (keyed)
+        for (int i = 0; i < used; ++i)
+            if (ctx_of[i] == ctx) {
+                *out = addr_of[i];
+                return cudaSuccess;
+            }
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_dq_partials);
+    if (e != cudaSuccess) return e;
+    *out = static_cast<double*>(p);
+    if (keyed && used < kSlots) {
+        ctx_of[used] = ctx;
+        addr_of[used] = *out;
+        ++used;
     }
-    *out = addr[device];
     return cudaSuccess;
 }
 
@@ -64,7 +100,7 @@ extern "C" nf4_status_t nf4_double_quant_noalloc(const float* absmax, int64_t nb
     }
     if (dev.major != 10) return NF4_ERR_UNSUPPORTED;
     double* scratch = nullptr;
-    if (scratch_address(dev.device, &scratch) != cudaSuccess) {
+    if (scratch_address(&scratch) != cudaSuccess) {
         cudaGetLastError();
         return NF4_ERR_CUDA;
     }

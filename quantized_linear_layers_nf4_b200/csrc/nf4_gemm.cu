@@ -31,6 +31,8 @@
 // Every mbarrier wait is bounded; a wait that runs out records
 // NF4_ERR_DEVICE_TIMEOUT, the CTA drains what it issued and frees its tensor
 // memory before returning.
+#include <mutex>
+
 #include "nf4_common.cuh"
 #include "nf4_decode.cuh"
 #include "nf4_internal.h"
@@ -643,10 +645,15 @@ cudaError_t launch_gemm(const void* X, int64_t m, const uint8_t* wq, const int8_
                             : (lo ? reinterpret_cast<const void*>(&gemm::k_nf4_gemm<false, true>)
                                   : reinterpret_cast<const void*>(&gemm::k_nf4_gemm<false, false>));
     const int vi = (y_bf16 ? 1 : 0) + (lo ? 2 : 0);
-    if (!attr_set[dev.device][vi]) {
-        const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set[dev.device][vi] = true;
+    {
+        static std::mutex mu;
+        std::lock_guard<std::mutex> lock(mu);
+        if (!attr_set[dev.device][vi]) {
+            const cudaError_t e =
+                cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::kSmemBytes);
+            if (e != cudaSuccess) return e;
+            attr_set[dev.device][vi] = true;
+        }
     }
     CUtensorMap tm_x, tm_w;
     cudaError_t e = tmap_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, static_cast<uint64_t>(k),
@@ -696,10 +703,15 @@ cudaError_t launch_gemm_dx(const void* dY, int64_t m, const uint8_t* wq, const i
     if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
     const void* fn = dx_bf16 ? reinterpret_cast<const void*>(&gemm::k_nf4_gemm_dx<true>)
                              : reinterpret_cast<const void*>(&gemm::k_nf4_gemm_dx<false>);
-    if (!attr_set[dev.device][dx_bf16]) {
-        const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set[dev.device][dx_bf16] = true;
+    {
+        static std::mutex mu;
+        std::lock_guard<std::mutex> lock(mu);
+        if (!attr_set[dev.device][dx_bf16]) {
+            const cudaError_t e =
+                cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::kSmemBytes);
+            if (e != cudaSuccess) return e;
+            attr_set[dev.device][dx_bf16] = true;
+        }
     }
     CUtensorMap tm_dy, tm_w;
     // dY [m, n] bf16, K-major boxes [256 tokens x 64 rows of W]

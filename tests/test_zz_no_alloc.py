@@ -69,9 +69,19 @@ def test_noalloc_matches_the_workspace_entry_point_on_consecutive_calls(nf4):
             assert _same(x, y), name
 
 
+def _header_limit() -> int:
+    """NF4_DQ_NOALLOC_MAX_NB as the C header defines it."""
+    import os
+    import re
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "nf4.h")
+    with open(path) as f:
+        return int(re.search(r"#define\s+NF4_DQ_NOALLOC_MAX_NB\s+(\d+)", f.read()).group(1))
+
+
 def test_noalloc_largest_size_and_the_limit(nf4):
     L = nf4._lib.lib()
-    limit = nf4._lib.NF4_DQ_NOALLOC_MAX_NB
+    limit = _header_limit()
+    assert limit == nf4._lib.NF4_DQ_NOALLOC_MAX_NB, "the binding's copy of the limit is stale"
     absmax = torch.rand(limit, device="cuda") * 0.1
     got = _noalloc(nf4, absmax)
     want = _with_workspace(nf4, absmax)
