@@ -459,8 +459,8 @@ def run_ours(args, rank, world, local):
     t_step_max = max_over_ranks(t_step, world)
     total_bytes = sum_over_ranks(float(step_bytes), world)
     value = total_bytes / t_step_max / 1e9
-    # nf4_linear_group launches one dequant-GEMV per weight (m <= 16)
-    launches_per_step = sum(len(grp) for grp in groups)
+    # nf4_linear_group makes one launch for a group it runs together, else one per weight
+    launches_per_step = sum(nf4.nf4_linear_group_launches(args.m, [w.n for w in grp], grp[0].k) for grp in groups)
     avg_launch_s = t_step / launches_per_step
     bytes_per_launch = step_bytes / launches_per_step
 
@@ -730,7 +730,7 @@ def run_ours(args, rank, world, local):
                        "launch": ("CUDA graph of %d launches per step (%s)%s"
                                   % (launches_per_step, "nf4_linear_ws per weight" if args.no_group else
                                      "per layer: nf4_linear_group q/k/v, o, nf4_linear_group gate/up, down; "
-                                     "one launch per weight",
+                                     "a group runs as one launch when that is predicted faster",
                                      ", NF4_LINEAR_WEIGHTS_EARLY: programmatic dependent launches, weight loads "
                                      "overlap the previous launch" if early else "")),
                        "split_k": "thread-block clusters, partial sums through distributed shared memory"

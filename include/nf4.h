@@ -360,9 +360,10 @@ nf4_status_t nf4_merge_lora(const nf4_weight_t* w, const void* lora_down, const 
  * nf4_linear_ws / nf4_linear_group can use for Y[m, n] = X[m, k] * What^T on the
  * current device; 0 when that product splits no k range (then no workspace is
  * needed), and always for m > 16 (the dequant-GEMM path).  The workspace holds
- * one counter per 128-row tile and the fp32 partial sums of every CTA; one
- * buffer serves every call whose requirement it meets.  Returns 0 for invalid
- * sizes.  Same source passages as nf4_linear.
+ * 1024 counters (one per 128-row tile of a launch) and room for the fp32 partial
+ * sums of two CTAs per SM; the non-zero size is the same for every shape, so one
+ * buffer serves every call and group of a model.  Returns 0 for invalid sizes.
+ * Same source passages as nf4_linear.
  */
 size_t nf4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k);
 
@@ -398,11 +399,14 @@ nf4_status_t nf4_linear_ws(const void* X, int64_t m, const nf4_weight_t* w, void
  * weights that share the input X (the query, key and value projections of an
  * attention block, the gate and up projections of an MLP), in one call.  Same
  * source passages as nf4_linear: per layer, each 4-bit weight is dequantized on
- * chip and multiplied in bf16 ([P4] §5; [P5] §2.2 code walk).  The weights are
- * launched one after another on the stream (the dequant-GEMV for m <= 16, the
- * dequant-GEMM above), each spreading its own tiles over every SM; every output
- * has the bits nf4_linear_ws gives for that weight alone, with or without a
- * workspace.
+ * chip and multiplied in bf16 ([P4] §5; [P5] §2.2 code walk).  For m <= 16 the
+ * weights run as one dequant-GEMV launch over all their row tiles when that is
+ * predicted to be faster than one launch per weight (the query, key and value
+ * projections of a layer), otherwise one launch each; larger m runs the
+ * dequant-GEMM once per weight.  A grouped launch may split k differently from a
+ * single-weight one, so an output can differ from nf4_linear_ws on that weight
+ * alone in the fp32 summation order (not beyond it); with and without a
+ * workspace the bits are the same.
  *   X          device, bf16 [m, k], 16-byte aligned
  *   w          host array of `count` pointers to weight structs, all with the same
  *              k and the same codebook (magic)
@@ -417,6 +421,15 @@ nf4_status_t nf4_linear_ws(const void* X, int64_t m, const nf4_weight_t* w, void
 nf4_status_t nf4_linear_group(const void* X, int64_t m, const nf4_weight_t* const* w, int32_t count,
                               void* const* Y, nf4_dtype_t y_dtype, int32_t* dev_status, uint32_t flags,
                               void* workspace, size_t ws_bytes, nf4_stream_t stream);
+
+/*
+ * nf4_linear_group_launches -- how many kernel launches nf4_linear_group makes
+ * for weights of rows n[0 .. count-1] and width k at m tokens on the current
+ * device: 1 when they run as one grouped launch, count otherwise.  Returns -1
+ * for invalid sizes or when no usable device is current.  Host only; n is a
+ * host array.
+ */
+int32_t nf4_linear_group_launches(int64_t m, const int64_t* n, int32_t count, int64_t k);
 
 #ifdef __cplusplus
 }

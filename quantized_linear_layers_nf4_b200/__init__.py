@@ -217,13 +217,24 @@ def _ws(workspace):
     return _ptr(workspace), workspace.numel() * workspace.element_size()
 
 
+def nf4_linear_group_launches(m: int, ns, k: int) -> int:
+    """Kernel launches nf4_linear_group makes for weights of rows `ns` and width k
+    at m tokens on the current device (1 when grouped into one launch)."""
+    arr = (ctypes.c_int64 * len(ns))(*[int(n) for n in ns])
+    r = _lib.lib().nf4_linear_group_launches(int(m), arr, len(ns), int(k))
+    if r < 0:
+        raise ValueError("invalid sizes or no usable device")
+    return int(r)
+
+
 def nf4_linear_group(X: torch.Tensor, weights, dtype=torch.bfloat16, outs=None,
                      dev_status: torch.Tensor | None = None, stream=None, weights_early: bool = False,
                      workspace: torch.Tensor | None = None, flags: int = 0):
     """[X @ W_i^T for W_i in weights] in one call for weights that share X and k
-    (at most NF4_LINEAR_GROUP_MAX), launched one after another on the stream;
-    each output has the bits of nf4_linear on that weight alone.  Returns the
-    list of outputs."""
+    (at most NF4_LINEAR_GROUP_MAX): one launch over all their row tiles when
+    that is faster than one launch per weight.  Each output equals nf4_linear on
+    that weight alone up to the fp32 summation order.  Returns the list of
+    outputs."""
     _need_cuda(X, "X")
     if X.dtype != torch.bfloat16 or X.dim() != 2:
         raise ValueError("X must be a 2-D bfloat16 tensor")

@@ -68,6 +68,7 @@ SIGNATURES = {
     "nf4_linear_group": (ctypes.c_int, [_p, _i64, ctypes.POINTER(ctypes.POINTER(nf4_weight_t)), ctypes.c_int32,
                                         ctypes.POINTER(_p), ctypes.c_int, _p, ctypes.c_uint32, _p, ctypes.c_size_t,
                                         _p]),
+    "nf4_linear_group_launches": (ctypes.c_int32, [_i64, ctypes.POINTER(_i64), ctypes.c_int32, _i64]),
 }
 
 

@@ -270,6 +270,15 @@ nf4_status_t nf4_linear_group(const void* X, int64_t m, const nf4_weight_t* cons
                                               codebook_of(w[0]), test, dev, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int32_t nf4_linear_group_launches(int64_t m, const int64_t* n, int32_t count, int64_t k) {
+    if (!n || count < 1 || count > nf4::kMaxGroup || m < 1 || k < 1 || k % NF4_BLOCKSIZE != 0) return -1;
+    for (int32_t i = 0; i < count; ++i)
+        if (n[i] < 1) return -1;
+    nf4::DeviceInfo dev;
+    if (device_ok(&dev) != NF4_OK) return -1;
+    return nf4::group_in_one_launch(m, n, count, k, false, dev) ? 1 : count;
+}
+
 nf4_status_t nf4_linear_ws(const void* X, int64_t m, const nf4_weight_t* w, void* Y,
                            nf4_dtype_t y_dtype, int32_t* dev_status, uint32_t flags, void* workspace,
                            size_t ws_bytes, nf4_stream_t stream) {

@@ -31,6 +31,7 @@
 // * Split-k: the CTAs of a thread-block cluster share a row tile and split k;
 //   their fp32 partials are added through distributed shared memory in a fixed
 //   rank order, so results are deterministic and no global scratch is needed.
+#include <cstring>
 #include <mutex>
 
 #include "nf4_common.cuh"
@@ -215,12 +216,24 @@ __device__ __forceinline__ void pin(AbsmaxIn& a) {
 
 constexpr int kPrefetch = 3;  // stages of absmax inputs in flight per producer lane
 
+// The weights of one launch (1 .. kMaxGroup, same k, same X): row tiles
+// tile0[i] .. tile0[i+1]-1 of the grid belong to weight i.
+struct GemvGroup {
+    CUtensorMap tm_w[kMaxGroup];  // codes [n x k/2 bytes], boxes [128 rows x 128 B], 128-byte swizzle
+    const int8_t* absmax_q[kMaxGroup];
+    const float* absmax_scale[kMaxGroup];
+    const float* mu[kMaxGroup];
+    void* y[kMaxGroup];
+    int64_t n[kMaxGroup];
+    int tile0[kMaxGroup];
+    int count;
+};
+
 template <bool kBf16Out, bool kM16, bool kLora>
 __global__ void __launch_bounds__(kThreads, 2)
-k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
-           const int8_t* __restrict__ absmax_q, const float* __restrict__ absmax_scale,
-           const float* __restrict__ mu_ptr, int m, int64_t n, int64_t k, int cluster, int weights_early,
-           void* __restrict__ Y, int32_t* __restrict__ dev_status, uint32_t* __restrict__ ws_cnt,
+k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtensorMap tm_x,
+           int m, int64_t k, int cluster, int weights_early,
+           int32_t* __restrict__ dev_status, uint32_t* __restrict__ ws_cnt,
            float4* __restrict__ ws_part, const float* __restrict__ lora_t, const __nv_bfloat16* __restrict__ lora_up,
            int lora_r, int codebook, uint32_t lim, int stall) {
     extern __shared__ uint8_t smem_raw[];
@@ -232,7 +245,18 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRows;
+    // this CTA's weight: the last one whose tiles start at or before blockIdx.x
+    int wi = 0;
+#pragma unroll
+    for (int i = 1; i < kMaxGroup; ++i)
+        if (i < grp.count && static_cast<int>(blockIdx.x) >= grp.tile0[i]) wi = i;
+    const CUtensorMap* tm_w = &grp.tm_w[wi];
+    const int8_t* __restrict__ absmax_q = grp.absmax_q[wi];
+    const float* __restrict__ absmax_scale = grp.absmax_scale[wi];
+    const float* __restrict__ mu_ptr = grp.mu[wi];
+    void* __restrict__ Y = grp.y[wi];
+    const int64_t n = grp.n[wi];
+    const int64_t row0 = static_cast<int64_t>(static_cast<int>(blockIdx.x) - grp.tile0[wi]) * kRows;
     const int64_t kblocks = k / 64;
     const int n_stages = static_cast<int>((k + kStageK - 1) / kStageK);
     const int rank = static_cast<int>(blockIdx.y);
@@ -254,7 +278,7 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
     if (warp == kConsumers) {
         // ------------------------------ producer ------------------------------
         if (lane == 0) {
-            prefetch_tensormap(&tm_w);
+            prefetch_tensormap(tm_w);
             prefetch_tensormap(&tm_x);
         }
         if (!weights_early) grid_dependency_wait();
@@ -284,7 +308,7 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
                 uint8_t* stage = ring + slot * kStageBytes;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&full[slot], kTmaBytes);
-                    tma_load_2d(stage, &tm_w, st * (kStageK / 2), static_cast<int32_t>(row0), &full[slot]);
+                    tma_load_2d(stage, tm_w, st * (kStageK / 2), static_cast<int32_t>(row0), &full[slot]);
                     if (x_ready) {
 #pragma unroll
                         for (int b = 0; b < 4; ++b)
@@ -567,27 +591,27 @@ k_nf4_gemv(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUt
 
 }  // namespace gemv
 
-// Cluster size (k split) for a weight of n rows and k columns.  The default is
-// the smallest of 1, 2, 4, 8 that gives at least one CTA per SM without giving
-// any CTA fewer than two stages.  Two CTAs fit on an SM, so the busiest SM's
-// work is (CTAs on it) x (stages per CTA); another size of 1 .. 8 that stays in
-// one wave replaces the default when it cuts that work by at least a fifth
-// (11008 rows: 258 CTAs of 6 stages instead of 172 of 8, i.e. 12 instead of 16).
-static int gemv_cluster(int64_t n, int64_t k, int sm_count) {
-    const int64_t tiles = (n + gemv::kRows - 1) / gemv::kRows;
-    const int64_t stages = (k + gemv::kStageK - 1) / gemv::kStageK;
+// Cluster size (k split) for `tiles` row tiles of `stages` k stages.  The
+// default is the smallest of 1, 2, 4, 8 that gives at least one CTA per SM
+// without giving any CTA fewer than two stages.  Two CTAs fit on an SM, so the
+// busiest SM's work is (CTAs on it) x (stages per CTA); another size of 1 .. 8
+// that stays in one wave replaces the default when it cuts that work by at least
+// a fifth (11008 rows: 258 CTAs of 6 stages instead of 172 of 8, i.e. 12 instead
+// of 16).  Any size above 1 keeps tiles x size within two CTAs per SM.
+static int64_t gemv_busiest(int64_t tiles, int64_t stages, int c, int sm_count) {
+    const int64_t per_sm = (tiles * c + sm_count - 1) / sm_count;
+    return per_sm * ((stages + c - 1) / c);
+}
+
+static int gemv_cluster_tiles(int64_t tiles, int64_t stages, int sm_count) {
     int c = 1;
     while (c < 8 && tiles * c < sm_count && 2 * c <= stages) c *= 2;
-    auto busiest = [&](int cc) {
-        const int64_t per_sm = (tiles * cc + sm_count - 1) / sm_count;
-        return per_sm * ((stages + cc - 1) / cc);
-    };
-    const int64_t base = busiest(c);
+    const int64_t base = gemv_busiest(tiles, stages, c, sm_count);
     int best = c;
     int64_t best_cost = base;
     for (int cc = 2; cc <= 8; ++cc) {
         if (2 * cc > stages || tiles * cc > 2 * static_cast<int64_t>(sm_count)) break;
-        const int64_t cost = busiest(cc);
+        const int64_t cost = gemv_busiest(tiles, stages, cc, sm_count);
         if (5 * cost <= 4 * base && cost < best_cost) {
             best = cc;
             best_cost = cost;
@@ -596,30 +620,34 @@ static int gemv_cluster(int64_t n, int64_t k, int sm_count) {
     return best;
 }
 
+static int64_t gemv_tiles(int64_t n) { return (n + gemv::kRows - 1) / gemv::kRows; }
+static int64_t gemv_stages(int64_t k) { return (k + gemv::kStageK - 1) / gemv::kStageK; }
+
+static int gemv_cluster(int64_t n, int64_t k, int sm_count) {
+    return gemv_cluster_tiles(gemv_tiles(n), gemv_stages(k), sm_count);
+}
+
 // Workspace layout, the same for every shape so that one buffer can serve a
-// sequence of different linears: kWsCounters 32-bit counters (one per 128-row
-// tile), then C fp32 partial tiles [16 tokens x 128 rows] per row tile.  A
-// split k only happens with at most one row tile per SM, far below kWsCounters.
+// sequence of different linears and groups: kWsCounters 32-bit counters (one per
+// 128-row tile of a launch), then C fp32 partial tiles [16 tokens x 128 rows] per
+// row tile.  A split k keeps tiles x C within two CTAs per SM, so the partials
+// never take more than 2 x SMs tiles.
 constexpr int64_t kWsCounters = 1024;
 constexpr size_t kWsCounterBytes = kWsCounters * 4;
+constexpr size_t kWsPartBytes = 16 * gemv::kRows * sizeof(float);
 
-static bool gemv_ws_usable(int64_t n, int cluster) {
-    return cluster > 1 && (n + gemv::kRows - 1) / gemv::kRows <= kWsCounters;
-}
+static bool gemv_ws_usable(int64_t tiles, int cluster) { return cluster > 1 && tiles <= kWsCounters; }
 
 size_t linear_workspace_bytes(int64_t m, int64_t n, int64_t k, const DeviceInfo& dev) {
     if (m > kGemvMaxTokens) return 0;
-    const int cluster = gemv_cluster(n, k, dev.sm_count);
-    if (!gemv_ws_usable(n, cluster)) return 0;
-    const size_t tiles = static_cast<size_t>((n + gemv::kRows - 1) / gemv::kRows);
-    return kWsCounterBytes + tiles * cluster * 16 * gemv::kRows * sizeof(float);
+    if (!gemv_ws_usable(gemv_tiles(n), gemv_cluster(n, k, dev.sm_count))) return 0;
+    return kWsCounterBytes + 2 * static_cast<size_t>(dev.sm_count) * kWsPartBytes;
 }
 
 template <bool kBf16Out, bool kM16, bool kLora>
-static cudaError_t launch_gemv(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const int8_t* absmax_q,
-                               const float* absmax_scale, const float* absmax_offset, int mt, int64_t n,
-                               int64_t k, int cluster, bool weights_early, void* Yt, int32_t* dev_status,
-                               void* ws, const LoraArgs& lora, int codebook, uint32_t test_flags, int device,
+static cudaError_t launch_gemv(const gemv::GemvGroup& grp, int64_t tiles, const CUtensorMap& tm_x, int mt,
+                               int64_t k, int cluster, bool weights_early, int32_t* dev_status, void* ws,
+                               const LoraArgs& lora, int codebook, uint32_t test_flags, int device,
                                cudaStream_t stream) {
     static std::mutex mu;
     static bool attr_set[64] = {};
@@ -633,12 +661,12 @@ static cudaError_t launch_gemv(const CUtensorMap& tm_w, const CUtensorMap& tm_x,
         }
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>((n + gemv::kRows - 1) / gemv::kRows), cluster, 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles), cluster, 1);
     cfg.blockDim = dim3(gemv::kThreads, 1, 1);
     cfg.dynamicSmemBytes = gemv::kSmemBytes;
     cfg.stream = stream;
     // With a workspace (and a split k) the CTAs of a tile need not be co-scheduled: no cluster.
-    const bool use_ws = ws != nullptr && gemv_ws_usable(n, cluster);
+    const bool use_ws = ws != nullptr && gemv_ws_usable(tiles, cluster);
     uint32_t* ws_cnt = use_ws ? static_cast<uint32_t*>(ws) : nullptr;
     float4* ws_part = use_ws ? reinterpret_cast<float4*>(static_cast<char*>(ws) + kWsCounterBytes) : nullptr;
     cudaLaunchAttribute attr[2];
@@ -657,22 +685,20 @@ static cudaError_t launch_gemv(const CUtensorMap& tm_w, const CUtensorMap& tm_x,
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    return cudaLaunchKernelEx(&cfg, gemv::k_nf4_gemv<kBf16Out, kM16, kLora>, tm_w, tm_x, absmax_q, absmax_scale,
-                              absmax_offset, mt, n, k, cluster, weights_early ? 1 : 0, Yt, dev_status, ws_cnt,
-                              ws_part, lora.t, lora.up, lora.r, codebook,
+    return cudaLaunchKernelEx(&cfg, gemv::k_nf4_gemv<kBf16Out, kM16, kLora>, grp, tm_x, mt, k, cluster,
+                              weights_early ? 1 : 0, dev_status, ws_cnt, ws_part, lora.t, lora.up, lora.r, codebook,
                               (test_flags & kTestStall) ? 64u : kWaitLimit, (test_flags & kTestStall) ? 1 : 0);
 }
 
 // One of the eight instantiations: output type, more than 8 tokens, LoRA term.
-static cudaError_t dispatch_gemv(bool bf16, bool m16, bool lora_on, const CUtensorMap& tm_w, const CUtensorMap& tm_x,
-                                 const int8_t* absmax_q, const float* absmax_scale, const float* absmax_offset,
-                                 int mt, int64_t n, int64_t k, int cluster, bool early, void* Yt, int32_t* ds,
+static cudaError_t dispatch_gemv(bool bf16, bool m16, bool lora_on, const gemv::GemvGroup& grp, int64_t tiles,
+                                 const CUtensorMap& tm_x, int mt, int64_t k, int cluster, bool early, int32_t* ds,
                                  void* ws, const LoraArgs& lora, int codebook, uint32_t test_flags, int device,
                                  cudaStream_t stream) {
 #define NF4_GEMV_CASE(B, M, L)                                                                                   \
     if (bf16 == B && m16 == M && lora_on == L)                                                                  \
-        return launch_gemv<B, M, L>(tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt, n, k, cluster, early, \
-                                    Yt, ds, ws, lora, codebook, test_flags, device, stream);
+        return launch_gemv<B, M, L>(grp, tiles, tm_x, mt, k, cluster, early, ds, ws, lora, codebook, test_flags, \
+                                    device, stream);
     NF4_GEMV_CASE(true, true, false)
     NF4_GEMV_CASE(true, false, false)
     NF4_GEMV_CASE(false, true, false)
@@ -685,37 +711,49 @@ static cudaError_t dispatch_gemv(bool bf16, bool m16, bool lora_on, const CUtens
     return cudaErrorInvalidValue;
 }
 
-static cudaError_t linear_one(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
-                              const float* absmax_scale, const float* absmax_offset, int64_t n, int64_t k, void* Y,
-                              bool y_bf16, int32_t* dev_status, bool weights_early, void* ws, const LoraArgs& lora,
-                              int codebook, uint32_t test_flags, const DeviceInfo& dev, cudaStream_t stream) {
-    if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
-    if (m > kGemvMaxTokens)
-        return launch_gemm(X, m, wq, absmax_q, absmax_scale, absmax_offset, n, k, Y, y_bf16, dev_status, lora,
-                           codebook, test_flags, dev, stream);
-    CUtensorMap tm_w;
-    cudaError_t e = tmap_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, static_cast<uint64_t>(k / 2),
-                            static_cast<uint64_t>(n), static_cast<uint64_t>(k / 2), 128, gemv::kRows,
-                            CU_TENSOR_MAP_SWIZZLE_128B);
-    if (e != cudaSuccess) return e;
-    const int cluster = gemv_cluster(n, k, dev.sm_count);
+// One dequant-GEMV launch over the row tiles of `count` weights (m <= 16).
+static cudaError_t gemv_launch_group(const void* X, int64_t m, int64_t k, const LinearWeight* w, int count,
+                                     bool y_bf16, int32_t* dev_status, bool weights_early, void* ws,
+                                     const LoraArgs& lora, int codebook, uint32_t test_flags, const DeviceInfo& dev,
+                                     cudaStream_t stream) {
+    gemv::GemvGroup grp;
+    memset(&grp, 0, sizeof(grp));
+    int64_t tiles = 0;
+    for (int i = 0; i < count; ++i) {
+        const cudaError_t e = tmap_2d(&grp.tm_w[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, w[i].wq, static_cast<uint64_t>(k / 2),
+                                      static_cast<uint64_t>(w[i].n), static_cast<uint64_t>(k / 2), 128, gemv::kRows,
+                                      CU_TENSOR_MAP_SWIZZLE_128B);
+        if (e != cudaSuccess) return e;
+        grp.absmax_q[i] = w[i].absmax_q;
+        grp.absmax_scale[i] = w[i].absmax_scale;
+        grp.mu[i] = w[i].absmax_offset;
+        grp.y[i] = w[i].y;
+        grp.n[i] = w[i].n;
+        grp.tile0[i] = static_cast<int>(tiles);
+        tiles += gemv_tiles(w[i].n);
+    }
+    grp.count = count;
+    if (tiles > 0x7fffffff) return cudaErrorInvalidValue;
+    const int cluster = gemv_cluster_tiles(tiles, gemv_stages(k), dev.sm_count);
     // portable cluster sizes only (the split-k epilogue handles any of 1 .. 8)
     if (cluster < 1 || cluster > 8) return cudaErrorInvalidConfiguration;
-    const size_t ybytes = y_bf16 ? 2 : 4;
-    const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
-    for (int64_t t0 = 0; t0 < m; t0 += 16) {
-        const int mt = static_cast<int>((m - t0) < 16 ? (m - t0) : 16);
-        CUtensorMap tm_x;
-        e = tmap_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Xb + t0 * k, static_cast<uint64_t>(k),
-                    static_cast<uint64_t>(mt), static_cast<uint64_t>(k * 2), 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
-        if (e != cudaSuccess) return e;
-        void* Yt = static_cast<char*>(Y) + static_cast<size_t>(t0) * n * ybytes;
-        e = dispatch_gemv(y_bf16, mt > 8, lora.t != nullptr, tm_w, tm_x, absmax_q, absmax_scale, absmax_offset, mt,
-                          n, k, cluster, weights_early, Yt, dev_status, ws, lora, codebook, test_flags, dev.device,
-                          stream);
-        if (e != cudaSuccess) return e;
-    }
-    return cudaSuccess;
+    CUtensorMap tm_x;
+    const cudaError_t e = tmap_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, static_cast<uint64_t>(k),
+                                  static_cast<uint64_t>(m), static_cast<uint64_t>(k * 2), 64, 16,
+                                  CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    return dispatch_gemv(y_bf16, m > 8, lora.t != nullptr, grp, tiles, tm_x, static_cast<int>(m), k, cluster,
+                         weights_early, dev_status, ws, lora, codebook, test_flags, dev.device, stream);
+}
+
+static cudaError_t linear_one(const void* X, int64_t m, const LinearWeight& w, int64_t k, bool y_bf16,
+                              int32_t* dev_status, bool weights_early, void* ws, const LoraArgs& lora, int codebook,
+                              uint32_t test_flags, const DeviceInfo& dev, cudaStream_t stream) {
+    if (m > kGemvMaxTokens)
+        return launch_gemm(X, m, w.wq, w.absmax_q, w.absmax_scale, w.absmax_offset, w.n, k, w.y, y_bf16, dev_status,
+                           lora, codebook, test_flags, dev, stream);
+    return gemv_launch_group(X, m, k, &w, 1, y_bf16, dev_status, weights_early, ws, lora, codebook, test_flags, dev,
+                             stream);
 }
 
 cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
@@ -723,21 +761,56 @@ cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int
                           int64_t k, void* Y, bool y_bf16, int32_t* dev_status, bool weights_early,
                           void* ws, const LoraArgs& lora, int codebook, const DeviceInfo& dev,
                           cudaStream_t stream) {
-    return linear_one(X, m, wq, absmax_q, absmax_scale, absmax_offset, n, k, Y, y_bf16, dev_status, weights_early,
-                      ws, lora, codebook, 0u, dev, stream);
+    if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
+    LinearWeight w;
+    w.wq = wq;
+    w.absmax_q = absmax_q;
+    w.absmax_scale = absmax_scale;
+    w.absmax_offset = absmax_offset;
+    w.n = n;
+    w.y = Y;
+    return linear_one(X, m, w, k, y_bf16, dev_status, weights_early, ws, lora, codebook, 0u, dev, stream);
 }
 
-// The weights of a group are launched one after the other on the stream (each
-// launch spreads its own tiles over every SM); one workspace serves them all,
-// since each launch leaves its counters at zero.
+// Fixed cost of one launch, in units of one k stage of the busiest SM (a stage
+// of two CTAs streams 32 KB of codes, about a microsecond): what a launch costs
+// beyond its streaming (start-up, ring fill, split-k exchange).
+constexpr int64_t kLaunchCostStages = 4;
+
+// The weights of a group share X and k.  For m <= 16 they run as one launch over
+// all their row tiles when the model of the busiest SM's work (stages, plus a
+// fixed cost per launch) says it beats one launch per weight; q / k / v of a
+// 4096-wide layer (3 x 32 tiles) do, gate / up of an 11008-wide MLP (2 x 86
+// tiles, already one wave each) do not.  Larger m runs the GEMM once per weight.
+bool group_in_one_launch(int64_t m, const int64_t* n, int count, int64_t k, bool lora, const DeviceInfo& dev) {
+    if (m > kGemvMaxTokens || count < 2 || lora) return false;
+    const int64_t stages = gemv_stages(k);
+    int64_t separate = 0, tiles = 0;
+    for (int i = 0; i < count; ++i) {
+        const int64_t ti = gemv_tiles(n[i]);
+        separate += gemv_busiest(ti, stages, gemv_cluster_tiles(ti, stages, dev.sm_count), dev.sm_count) +
+                    kLaunchCostStages;
+        tiles += ti;
+    }
+    const int64_t grouped =
+        gemv_busiest(tiles, stages, gemv_cluster_tiles(tiles, stages, dev.sm_count), dev.sm_count) +
+        kLaunchCostStages;
+    return grouped < separate && tiles <= kWsCounters;
+}
+
 cudaError_t launch_linear_group(const void* X, int64_t m, int64_t k, const LinearWeight* w, int count,
                                 bool y_bf16, int32_t* dev_status, bool weights_early, void* ws, const LoraArgs& lora,
                                 int codebook, uint32_t test_flags, const DeviceInfo& dev, cudaStream_t stream) {
+    if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
     if (count < 1 || count > kMaxGroup) return cudaErrorInvalidValue;
+    int64_t ns[kMaxGroup];
+    for (int i = 0; i < count; ++i) ns[i] = w[i].n;
+    if (group_in_one_launch(m, ns, count, k, lora.t != nullptr, dev))
+        return gemv_launch_group(X, m, k, w, count, y_bf16, dev_status, weights_early, ws, lora, codebook,
+                                 test_flags, dev, stream);
     for (int i = 0; i < count; ++i) {
-        const cudaError_t e = linear_one(X, m, w[i].wq, w[i].absmax_q, w[i].absmax_scale, w[i].absmax_offset, w[i].n,
-                                         k, w[i].y, y_bf16, dev_status, weights_early, ws, lora, codebook, test_flags,
-                                         dev, stream);
+        const cudaError_t e = linear_one(X, m, w[i], k, y_bf16, dev_status, weights_early, ws, lora, codebook,
+                                         test_flags, dev, stream);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

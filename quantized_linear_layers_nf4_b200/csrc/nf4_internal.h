@@ -74,6 +74,10 @@ cudaError_t launch_linear_group(const void* X, int64_t m, int64_t k, const Linea
                                 bool y_bf16, int32_t* dev_status, bool weights_early, void* ws, const LoraArgs& lora,
                                 int codebook, uint32_t test_flags, const DeviceInfo& dev, cudaStream_t stream);
 
+// True when launch_linear_group runs these weights (rows n[0 .. count-1], one
+// k) as a single dequant-GEMV launch rather than one launch per weight.
+bool group_in_one_launch(int64_t m, const int64_t* n, int count, int64_t k, bool lora, const DeviceInfo& dev);
+
 // `ws` (nullable) must hold linear_workspace_bytes(m, n, k, dev) bytes, 16-byte aligned.
 cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int8_t* absmax_q,
                           const float* absmax_scale, const float* absmax_offset, int64_t n,
