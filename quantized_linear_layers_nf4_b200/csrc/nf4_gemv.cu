@@ -509,11 +509,16 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
         __syncthreads();
         if (!*last) return;
         for (int e = threadIdx.x; e < m * (kRows / 4); e += kThreads) {
-            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int q = 0; q < cluster; ++q) {
-                const float4 v = (q == rank) ? part4[e] : __ldcg(part_g + q * kQ + e);
-                sum = (q == 0) ? v : make_float4(sum.x + v.x, sum.y + v.y, sum.z + v.z, sum.w + v.w);
-            }
+            // every part's load goes out before the first add (one L2 round trip,
+            // not one per part); the adds keep rank order
+            float4 v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (q < cluster) v[q] = (q == rank) ? part4[e] : __ldcg(part_g + q * kQ + e);
+            float4 sum = v[0];
+#pragma unroll
+            for (int q = 1; q < 8; ++q)
+                if (q < cluster) sum = make_float4(sum.x + v[q].x, sum.y + v[q].y, sum.z + v[q].z, sum.w + v[q].w);
             const int tok = e / (kRows / 4);
             const int r = 4 * (e % (kRows / 4));
             float o[4] = {sum.x, sum.y, sum.z, sum.w};
