@@ -22,8 +22,9 @@
 //   of the 128 rows, so one X fragment serves 8 MMAs.  The multiply-adds run on the tensor
 //   cores (mma.sync m16n8k16, bf16 in, fp32 accumulate) with the 16 token slots
 //   as the MMA's M side (zero-filled beyond m) and 8 weight rows as its N side.
-//   Each lane owns 16 consecutive weights of a block row; the MMA k order is a
-//   permutation of the true k order applied identically to X and the weights.
+//   X fragments come from ldmatrix in the MMA's own layout; for k chunk s of a
+//   block, lane (g, i) decodes bytes 8s + i and 8s + 4 + i of row g (weights
+//   16s + 2i, +1 and 16s + 8 + 2i, +1), so the k order is the true one.
 // * Decode: a 256-entry table maps a packed byte to the two fp32 levels it
 //   encodes (replicated 16x so a half-warp's lookups never share a bank); each
 //   level is multiplied by the block's reconstructed absmax in fp32 and rounded
@@ -98,22 +99,19 @@ __device__ __forceinline__ float lora_term(float v, const float* __restrict__ lt
     return v;
 }
 
-// Byte `b` (0..3) of `word` in the low 8 bits, zeros above (one byte permute).
-__device__ __forceinline__ uint32_t byte_of(uint32_t word, uint32_t b) {
-    uint32_t d;
-    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(d) : "r"(word), "r"(0x4440u | b));
-    return d;
-}
-
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
     return v;
 }
 
-__device__ __forceinline__ uint2 lds64(uint32_t addr) {
-    uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+// Four 8x8 bf16 matrices, one 16-byte row address per lane: the registers come
+// back in the layout of an m16n8k16 A fragment.
+__device__ __forceinline__ uint4 ldsm_x4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
     return v;
 }
 
@@ -152,6 +150,43 @@ __device__ __forceinline__ uint32_t scale_pack(uint64_t levels, uint64_t aa) {
         : "=r"(out)
         : "l"(levels), "l"(aa));
     return out;
+}
+
+// Rows grow0 .. grow0 + 3 of token `tok` (rows past n are dropped), the
+// low-rank term added first when there is one: one vector store when all four
+// rows are in range and the address is aligned, else one store per row.
+template <bool kBf16Out, bool kLora>
+__device__ __forceinline__ void store_quad(void* __restrict__ Y, int64_t n, int tok, int64_t grow0, float (&o)[4],
+                                           const float* __restrict__ lt, const __nv_bfloat16* __restrict__ up,
+                                           int r) {
+    if (kLora) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            if (grow0 + c < n) o[c] = lora_term(o[c], lt, up, r, tok, grow0 + c);
+    }
+    const int64_t idx = static_cast<int64_t>(tok) * n + grow0;
+    if (kBf16Out) {
+        __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(Y) + idx;
+        if (grow0 + 3 < n && (reinterpret_cast<uintptr_t>(y) & 7) == 0) {
+            const __nv_bfloat162 p0 = __floats2bfloat162_rn(o[0], o[1]);
+            const __nv_bfloat162 p1 = __floats2bfloat162_rn(o[2], o[3]);
+            *reinterpret_cast<uint2*>(y) =
+                make_uint2(*reinterpret_cast<const uint32_t*>(&p0), *reinterpret_cast<const uint32_t*>(&p1));
+            return;
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            if (grow0 + c < n) y[c] = __float2bfloat16_rn(o[c]);
+    } else {
+        float* y = reinterpret_cast<float*>(Y) + idx;
+        if (grow0 + 3 < n && (reinterpret_cast<uintptr_t>(y) & 15) == 0) {
+            *reinterpret_cast<float4*>(y) = make_float4(o[0], o[1], o[2], o[3]);
+            return;
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            if (grow0 + c < n) y[c] = o[c];
+    }
 }
 
 // The producer's per-stage absmax inputs.  Lane l owns rows l + 32 u (u = 0..3)
@@ -410,6 +445,12 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
         const int blk = warp & 3;          // 64-block of the stage
         const int rbase = (warp >> 2) * 64;  // first of this warp's 64 rows
         const uint32_t lut_lane = smem_u32(lut) + (lane & 15) * 8u;
+        // the X row this lane addresses for ldmatrix: token (lane & 7) + 8 ((lane >> 3) & 1)
+        const uint32_t x_lane = ((lane & 7) + 8 * ((lane >> 3) & 1)) * 128;
+        // the two 16-byte chunks of a block row (128-byte swizzle, row & 7 == g);
+        // lane i decodes byte i of each of their 8 words
+        const uint32_t wc0 = ((2 * blk) ^ g) << 4, wc1 = ((2 * blk + 1) ^ g) << 4;
+        const uint32_t sel_i = 0x4440u | static_cast<uint32_t>(i);
         float acc[kTiles][4];
 #pragma unroll
         for (int t = 0; t < kTiles; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
@@ -424,31 +465,30 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
             }
             const uint32_t stage = smem_u32(ring + slot * kStageBytes);
             // X fragments: tokens g and g + 8, k = 16 i .. 16 i + 15 of this warp's block
+            // A fragments of the block's four k16 chunks: tokens 0-7 / 8-15 x the
+            // chunk's two 16-byte halves (128-byte swizzle, row & 7 == lane & 7)
             const uint32_t xb = stage + kWBytes + blk * kXBox;
-            const uint4 xa0 = lds128(xb + g * 128 + (((2 * i) ^ g) << 4));
-            const uint4 xa1 = lds128(xb + g * 128 + (((2 * i + 1) ^ g) << 4));
-            uint4 xc0 = make_uint4(0u, 0u, 0u, 0u), xc1 = xc0;
-            if (kM16) {
-                xc0 = lds128(xb + (g + 8) * 128 + (((2 * i) ^ g) << 4));
-                xc1 = lds128(xb + (g + 8) * 128 + (((2 * i + 1) ^ g) << 4));
-            }
-            const uint32_t xa[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
-            const uint32_t xc[8] = {xc0.x, xc0.y, xc0.z, xc0.w, xc1.x, xc1.y, xc1.z, xc1.w};
-            const uint32_t wb = stage + (rbase + g) * 128 + ((((2 * blk + (i >> 1)) ^ g) << 4) + ((i & 1) << 3));
+            uint4 xf[4];
+#pragma unroll
+            for (int s = 0; s < 4; ++s) xf[s] = ldsm_x4(xb + x_lane + (((2 * s + (lane >> 4)) ^ (lane & 7)) << 4));
+            const uint32_t wrow = stage + (rbase + g) * 128;
             const uint32_t ab = stage + kTmaBytes + ((rbase + g) * 4 + blk) * 4;
 #pragma unroll
             for (int t = 0; t < kTiles; ++t) {
-                const uint2 raw = lds64(wb + t * 8 * 128);
+                const uint4 w0 = lds128(wrow + t * 8 * 128 + wc0);
+                const uint4 w1 = lds128(wrow + t * 8 * 128 + wc1);
+                const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
                 const uint64_t aa = dup_f32x2(lds_f32(ab + 128 * t));
                 uint32_t bw[8];
 #pragma unroll
                 for (int b = 0; b < 8; ++b) {
-                    const uint32_t word = (b < 4) ? raw.x : raw.y;
-                    bw[b] = scale_pack(lds_b64(lut_lane + (byte_of(word, b & 3) << 7)), aa);
+                    uint32_t byte;
+                    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(byte) : "r"(wv[b]), "r"(sel_i));
+                    bw[b] = scale_pack(lds_b64(lut_lane + (byte << 7)), aa);
                 }
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_16816(acc[t], xa[2 * s], xc[2 * s], xa[2 * s + 1], xc[2 * s + 1], bw[2 * s], bw[2 * s + 1]);
+                    mma_16816(acc[t], xf[s].x, xf[s].y, xf[s].z, xf[s].w, bw[2 * s], bw[2 * s + 1]);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);
@@ -508,30 +548,33 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
         }
         __syncthreads();
         if (!*last) return;
-        for (int e = threadIdx.x; e < m * (kRows / 4); e += kThreads) {
-            // every part's load goes out before the first add (one L2 round trip,
-            // not one per part); the adds keep rank order
-            float4 v[8];
+        // Each thread owns at most two float4s of the tile; every load of both
+        // (all C parts) goes out before the first add, so the reduction costs one
+        // L2 round trip.  The adds keep rank order.
+        static_assert(2 * kThreads >= kQ, "two float4s per thread cover the tile");
+        const int ne = m * (kRows / 4);
+        float4 v[2][8];
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-                if (q < cluster) v[q] = (q == rank) ? part4[e] : __ldcg(part_g + q * kQ + e);
-            float4 sum = v[0];
+        for (int h = 0; h < 2; ++h) {
+            const int e = static_cast<int>(threadIdx.x) + h * kThreads;
+            if (e < ne) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    if (q < cluster) v[h][q] = (q == rank) ? part4[e] : __ldcg(part_g + q * kQ + e);
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int e = static_cast<int>(threadIdx.x) + h * kThreads;
+            if (e >= ne) break;
+            float4 sum = v[h][0];
 #pragma unroll
             for (int q = 1; q < 8; ++q)
-                if (q < cluster) sum = make_float4(sum.x + v[q].x, sum.y + v[q].y, sum.z + v[q].z, sum.w + v[q].w);
-            const int tok = e / (kRows / 4);
-            const int r = 4 * (e % (kRows / 4));
+                if (q < cluster)
+                    sum = make_float4(sum.x + v[h][q].x, sum.y + v[h][q].y, sum.z + v[h][q].z, sum.w + v[h][q].w);
             float o[4] = {sum.x, sum.y, sum.z, sum.w};
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int64_t grow = row0 + r + c;
-                if (grow >= n) break;
-                if (kLora) o[c] = lora_term(o[c], lora_t, lora_up, lora_r, tok, grow);
-                if (kBf16Out)
-                    reinterpret_cast<__nv_bfloat16*>(Y)[static_cast<int64_t>(tok) * n + grow] = __float2bfloat16_rn(o[c]);
-                else
-                    reinterpret_cast<float*>(Y)[static_cast<int64_t>(tok) * n + grow] = o[c];
-            }
+            store_quad<kBf16Out, kLora>(Y, n, e / (kRows / 4), row0 + 4 * (e % (kRows / 4)), o, lora_t, lora_up,
+                                        lora_r);
         }
         if (threadIdx.x == 0) ws_cnt[tile] = 0;  // ready for the next call
         return;
@@ -580,16 +623,7 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
         for (int q = 1; q < 8; ++q)
             if (q < cluster) sum = make_float4(sum.x + v[q].x, sum.y + v[q].y, sum.z + v[q].z, sum.w + v[q].w);
         float o[4] = {sum.x, sum.y, sum.z, sum.w};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const int64_t grow = row0 + r + c;
-            if (grow >= n) break;
-            if (kLora) o[c] = lora_term(o[c], lora_t, lora_up, lora_r, tok, grow);
-            if (kBf16Out)
-                reinterpret_cast<__nv_bfloat16*>(Y)[static_cast<int64_t>(tok) * n + grow] = __float2bfloat16_rn(o[c]);
-            else
-                reinterpret_cast<float*>(Y)[static_cast<int64_t>(tok) * n + grow] = o[c];
-        }
+        store_quad<kBf16Out, kLora>(Y, n, tok, row0 + r, o, lora_t, lora_up, lora_r);
     }
     cluster_sync();  // keep this CTA's partials alive until every rank has read them
 }
