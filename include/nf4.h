@@ -302,9 +302,13 @@ size_t nf4_linear_lora_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t 
  * low-rank update, Y = X * What^T + scale * (X * down^T) * up^T ([P4] "2-2. LoRA
  * （低秩適應）": W acts as W + dW with dW = A x B of rank r; section 4: base frozen
  * INT4, LoRA matrices bf16).  With W stored [n, k], dW = up * down.
- * t = scale * X down^T is computed first (fp32, fixed summation order).  For
- * m <= 16 the linear then adds sum_j t[i][j] * up[o][j] (j in order, fp32) to
- * each fp32 output before rounding it to y_dtype.  For larger m with r % 8 == 0
+ * t = scale * X down^T is formed in fp32.  For m <= 16 with r = 8 or 16 the
+ * dequant-GEMV forms it itself: tensor-core products over the same X tiles as
+ * the base, each CTA's share of k added into the split-k exchange in a fixed
+ * order (no separate launch).  Other m <= 16 cases compute it first in a small
+ * kernel (fixed summation order).  For m <= 16 the linear then adds
+ * sum_j t[i][j] * up[o][j] (j in order, fp32) to each fp32 output before
+ * rounding it to y_dtype.  For larger m with r % 8 == 0
  * the term runs on the tensor cores as extra K steps, t_hi up^T + t_lo up^T
  * with t = t_hi + t_lo split into bf16 halves (t kept to about 16 bits) and
  * accumulated in fp32; other ranks use the fp32 epilogue.  Same path and flags
@@ -361,7 +365,8 @@ nf4_status_t nf4_merge_lora(const nf4_weight_t* w, const void* lora_down, const 
  * current device; 0 when that product splits no k range (then no workspace is
  * needed), and always for m > 16 (the dequant-GEMM path).  The workspace holds
  * 1024 counters (one per 128-row tile of a launch) and room for the fp32 partial
- * sums of two CTAs per SM; the non-zero size is the same for every shape, so one
+ * sums of two CTAs per SM (each with the CTA's share of a fused LoRA
+ * down-projection); the non-zero size is the same for every shape, so one
  * buffer serves every call and group of a model.  Returns 0 for invalid sizes.
  * Same source passages as nf4_linear.
  */

@@ -189,18 +189,24 @@ nf4_status_t nf4_linear_lora(const void* X, int64_t m, const nf4_weight_t* w, co
     const size_t tb = lora_t_bytes(m, r);
     if (ws_bytes < tb + nf4::linear_workspace_bytes(m, w->n, w->k, dev)) return NF4_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    float* t = static_cast<float*>(workspace);
-    __nv_bfloat16* t_hi = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(workspace) + lora_t_region(m, r, 4));
-    __nv_bfloat16* t_lo = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<char*>(t_hi) + lora_t_region(m, r, 2));
-    st = from_cuda(nf4::launch_lora_down(X, m, w->k, lora_down, r, scale, t, t_hi, t_lo,
-                                         (flags & NF4_LINEAR_WEIGHTS_EARLY) != 0, s));
-    if (st != NF4_OK) return st;
     nf4::LoraArgs lora;
-    lora.t = t;
     lora.up = static_cast<const __nv_bfloat16*>(lora_up);
     lora.r = r;
-    lora.t_hi = t_hi;
-    lora.t_lo = t_lo;
+    if (nf4::gemv_fuses_lora(m, w->n, w->k, r, true, dev)) {
+        // decode with r = 8 or 16: the dequant-GEMV forms t itself
+        lora.down = static_cast<const __nv_bfloat16*>(lora_down);
+        lora.scale = scale;
+    } else {
+        float* t = static_cast<float*>(workspace);
+        __nv_bfloat16* t_hi = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(workspace) + lora_t_region(m, r, 4));
+        __nv_bfloat16* t_lo = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<char*>(t_hi) + lora_t_region(m, r, 2));
+        st = from_cuda(nf4::launch_lora_down(X, m, w->k, lora_down, r, scale, t, t_hi, t_lo,
+                                             (flags & NF4_LINEAR_WEIGHTS_EARLY) != 0, s));
+        if (st != NF4_OK) return st;
+        lora.t = t;
+        lora.t_hi = t_hi;
+        lora.t_lo = t_lo;
+    }
     return from_cuda(nf4::launch_linear(X, m, w->wq, w->absmax_q, w->absmax_scale, w->absmax_offset, w->n, w->k,
                                         Y, y_dtype == NF4_BF16, dev_status, (flags & NF4_LINEAR_WEIGHTS_EARLY) != 0,
                                         static_cast<char*>(workspace) + tb, lora, codebook_of(w), dev, s));

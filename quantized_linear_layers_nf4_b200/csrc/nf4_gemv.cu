@@ -63,6 +63,13 @@ static_assert(kStageBytes % 1024 == 0, "stages keep the 1 KiB alignment the 128-
 // that the 8 row groups of a warp write distinct banks.
 constexpr int kRedPitch = kRows + 8;
 static_assert(4 * 16 * kRedPitch * 4 + 16 * kRows * 4 <= kRingBytes, "reduction fits in the ring");
+// After the block partials (red) and the CTA's partial tile (part4): the four
+// blocks' down-projection sums [4][16 tokens][16 ranks] and the CTA's t (the
+// fused LoRA down-projection), in floats from the start of the ring.
+constexpr int kTredOff = 4 * 16 * kRedPitch + 16 * kRows;
+constexpr int kTOff = kTredOff + 4 * 256;
+// Then the tile's up rows, transposed: [16 ranks][128 rows] bf16.
+static_assert((kTOff + 256) * 4 + 16 * kRows * 2 <= kRingBytes, "down-projection sums fit in the ring");
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
@@ -97,6 +104,21 @@ __device__ __forceinline__ float lora_term(float v, const float* __restrict__ lt
     }
     for (; j < r; ++j) v = __fmaf_rn(__ldg(tr + j), __bfloat162float(ur[j]), v);
     return v;
+}
+
+// The same sums for four consecutive rows with t and up in shared memory (the
+// fused down-projection): ts [token][16], ut [rank][128 rows] bf16, rl the
+// first row's index in the tile.
+__device__ __forceinline__ void lora_quad_shared(float (&o)[4], const float* ts, const __nv_bfloat16* ut, int r,
+                                                 int tok, int rl) {
+    for (int j = 0; j < r; ++j) {
+        const float tj = ts[tok * 16 + j];
+        const uint2 u = *reinterpret_cast<const uint2*>(ut + j * 128 + rl);
+        o[0] = __fmaf_rn(tj, bf16_bits_to_float(u.x & 0xffffu), o[0]);
+        o[1] = __fmaf_rn(tj, bf16_bits_to_float(u.x >> 16), o[1]);
+        o[2] = __fmaf_rn(tj, bf16_bits_to_float(u.y & 0xffffu), o[2]);
+        o[3] = __fmaf_rn(tj, bf16_bits_to_float(u.y >> 16), o[3]);
+    }
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -152,17 +174,46 @@ __device__ __forceinline__ uint32_t scale_pack(uint64_t levels, uint64_t aa) {
     return out;
 }
 
+// B fragments of down for k stage `st`, block blk: the k pairs 8q + 2i of the
+// block (q = 2s + half), zero past k or for a rank past r.
+__device__ __forceinline__ void load_down(uint32_t (&b)[8], const __nv_bfloat16* __restrict__ drow, int st, int blk,
+                                          int i, int64_t k, bool rank_ok) {
+    const int64_t kb = static_cast<int64_t>(st) * kStageK;
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+        b[q] = (rank_ok && kb + 64 * blk + 8 * q + 2 * i < k) ? __ldg(reinterpret_cast<const uint32_t*>(drow + kb + 8 * q))
+                                                              : 0u;
+}
+
+// Thread 2 row + h holds up[row0 + row][8h .. 8h + 7] (zeros past n or r);
+// ut[j][row] = up[row0 + row][j].
+__device__ __forceinline__ void stage_up(__nv_bfloat16* ut, uint4 v, int row, int h, int r) {
+    if (threadIdx.x >= 256 || 8 * h >= r) return;
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint16_t* u = reinterpret_cast<uint16_t*>(ut);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        u[(8 * h + 2 * q) * 128 + row] = static_cast<uint16_t>(w[q] & 0xffffu);
+        u[(8 * h + 2 * q + 1) * 128 + row] = static_cast<uint16_t>(w[q] >> 16);
+    }
+}
+
 // Rows grow0 .. grow0 + 3 of token `tok` (rows past n are dropped), the
-// low-rank term added first when there is one: one vector store when all four
+// low-rank term added first when there is one (t and up from shared memory, ts
+// and ut, when ts is set, else from lt and up): one vector store when all four
 // rows are in range and the address is aligned, else one store per row.
 template <bool kBf16Out, bool kLora>
 __device__ __forceinline__ void store_quad(void* __restrict__ Y, int64_t n, int tok, int64_t grow0, float (&o)[4],
-                                           const float* __restrict__ lt, const __nv_bfloat16* __restrict__ up,
-                                           int r) {
+                                           const float* __restrict__ lt, const __nv_bfloat16* __restrict__ up, int r,
+                                           const float* ts, const __nv_bfloat16* ut, int rl) {
     if (kLora) {
+        if (ts) {
+            lora_quad_shared(o, ts, ut, r, tok, rl);
+        } else {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-            if (grow0 + c < n) o[c] = lora_term(o[c], lt, up, r, tok, grow0 + c);
+            for (int c = 0; c < 4; ++c)
+                if (grow0 + c < n) o[c] = lora_term(o[c], lt, up, r, tok, grow0 + c);
+        }
     }
     const int64_t idx = static_cast<int64_t>(tok) * n + grow0;
     if (kBf16Out) {
@@ -270,7 +321,8 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
            int m, int64_t k, int cluster, int weights_early,
            int32_t* __restrict__ dev_status, uint32_t* __restrict__ ws_cnt,
            float4* __restrict__ ws_part, const float* __restrict__ lora_t, const __nv_bfloat16* __restrict__ lora_up,
-           int lora_r, int codebook, uint32_t lim, int stall) {
+           int lora_r, const __nv_bfloat16* __restrict__ lora_down, float lora_scale, int codebook, uint32_t lim,
+           int stall) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* ring = smem;
@@ -298,7 +350,8 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
     const int s0 = static_cast<int>((static_cast<int64_t>(n_stages) * rank) / cluster);
     const int s1 = static_cast<int>((static_cast<int64_t>(n_stages) * (rank + 1)) / cluster);
 
-    __shared__ int s_bad;  // some warp of this CTA gave up a wait
+    __shared__ int s_bad;   // some warp of this CTA gave up a wait
+    __shared__ int s_last;  // this CTA is the last of its tile to finish (workspace split-k)
     if (threadIdx.x == 0) {
         s_bad = 0;
         for (int s = 0; s < kRing; ++s) {
@@ -451,6 +504,18 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
         // lane i decodes byte i of each of their 8 words
         const uint32_t wc0 = ((2 * blk) ^ g) << 4, wc1 = ((2 * blk + 1) ^ g) << 4;
         const uint32_t sel_i = 0x4440u | static_cast<uint32_t>(i);
+        // Fused down-projection of a LoRA layer (r = 8 or 16): warp (blk, h) adds
+        // X[:, block] down[8h .. 8h + 7, block]^T into tacc with the same X
+        // fragments; lane (g, i) reads rank 8h + g of down at the MMA's k pairs.
+        const bool t_on = kLora && lora_down != nullptr && 8 * (warp >> 2) < lora_r;
+        const int t_rank = 8 * (warp >> 2) + g;
+        const __nv_bfloat16* __restrict__ drow =
+            kLora && lora_down != nullptr
+                ? lora_down + static_cast<int64_t>(t_rank < lora_r ? t_rank : 0) * k + 64 * blk + 2 * i
+                : nullptr;
+        float tacc[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t bA[8];  // the current stage's down fragments
+        if (kLora && t_on) load_down(bA, drow, s0, blk, i, k, t_rank < lora_r);
         float acc[kTiles][4];
 #pragma unroll
         for (int t = 0; t < kTiles; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
@@ -490,6 +555,11 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
                 for (int s = 0; s < 4; ++s)
                     mma_16816(acc[t], xf[s].x, xf[s].y, xf[s].z, xf[s].w, bw[2 * s], bw[2 * s + 1]);
             }
+            if (kLora && t_on) {
+#pragma unroll
+                for (int s = 0; s < 4; ++s) mma_16816(tacc, xf[s].x, xf[s].y, xf[s].z, xf[s].w, bA[2 * s], bA[2 * s + 1]);
+                if (st + 1 < s1) load_down(bA, drow, st + 1, blk, i, k, t_rank < lora_r);  // next stage's, in flight
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);
         }
@@ -498,6 +568,15 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
         // block land in disjoint rows of the same buffer)
         __syncwarp();
         named_bar_sync(1, 32 * kConsumers);  // every consumer is done with the ring
+        if (kLora && t_on) {
+            // tred[blk][token][rank]
+            float* tr = reinterpret_cast<float*>(ring) + kTredOff + blk * 256;
+            const int j = 8 * (warp >> 2) + 2 * i;
+            tr[g * 16 + j] = tacc[0];
+            tr[g * 16 + j + 1] = tacc[1];
+            tr[(g + 8) * 16 + j] = tacc[2];
+            tr[(g + 8) * 16 + j + 1] = tacc[3];
+        }
         float* red = reinterpret_cast<float*>(ring) + blk * 16 * kRedPitch;
 #pragma unroll
         for (int t = 0; t < kTiles; ++t) {
@@ -517,6 +596,7 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
     const float* redf = reinterpret_cast<const float*>(ring);
     float4* part4 = reinterpret_cast<float4*>(ring) + 4 * 16 * kRedPitch / 4;
     constexpr int kQ = 16 * kRows / 4;  // float4s of partial sums per CTA
+    constexpr int kQS = kQ + 64;         // a workspace slot: the partial tile, then the CTA's t [16][16]
     constexpr int kB = 16 * kRedPitch;  // floats per block buffer
     for (int e = threadIdx.x; e < kQ; e += kThreads) {
         const int off = (e / (kRows / 4)) * kRedPitch + 4 * (e % (kRows / 4));
@@ -527,6 +607,22 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
         part4[e] = make_float4(((a.x + b.x) + c.x) + d.x, ((a.y + b.y) + c.y) + d.y,
                                ((a.z + b.z) + c.z) + d.z, ((a.w + b.w) + c.w) + d.w);
     }
+    // The CTA's share of the fused down-projection: thread e < 256 holds
+    // t[e / 16][e % 16], the four blocks added in order (ranks >= r unused).
+    // Its up rows are fetched now and staged (transposed, [rank][row]) once the
+    // tile's t is known.
+    const bool t_fused = kLora && lora_down != nullptr;
+    float* tful = reinterpret_cast<float*>(ring) + kTOff;
+    __nv_bfloat16* utile = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<float*>(ring) + kTOff + 256);
+    float tv = 0.f;
+    uint4 upv = make_uint4(0u, 0u, 0u, 0u);
+    const int up_row = static_cast<int>(threadIdx.x) / 2, up_h = static_cast<int>(threadIdx.x) & 1;  // r = 16
+    if (t_fused && threadIdx.x < 256) {
+        const float* tr = redf + kTredOff + threadIdx.x;
+        tv = ((tr[0] + tr[256]) + tr[512]) + tr[768];
+        if (8 * up_h < lora_r && row0 + up_row < n)
+            upv = __ldg(reinterpret_cast<const uint4*>(lora_up + (row0 + up_row) * lora_r + 8 * up_h));
+    }
 
     if (ws_part != nullptr) {
         // Split-k through the caller's workspace: each CTA stores its partial
@@ -534,20 +630,20 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
         // partials in rank order (the order the cluster path uses) and writes Y.
         if (bad) return;
         const int tile = static_cast<int>(blockIdx.x);
-        float4* part_g = ws_part + static_cast<int64_t>(tile) * cluster * kQ;
-        for (int e = threadIdx.x; e < m * (kRows / 4); e += kThreads) part_g[rank * kQ + e] = part4[e];
+        float4* part_g = ws_part + static_cast<int64_t>(tile) * cluster * kQS;
+        for (int e = threadIdx.x; e < m * (kRows / 4); e += kThreads) part_g[rank * kQS + e] = part4[e];
+        if (t_fused && threadIdx.x < m * 16) reinterpret_cast<float*>(part_g + rank * kQS + kQ)[threadIdx.x] = tv;
         __syncthreads();
         // One acquire-release add at GPU scope publishes the whole CTA's stores
         // (ordered before it by the barrier) and, for the last CTA, makes every
         // other CTA's partials visible to the loads below.
-        volatile int* last = reinterpret_cast<volatile int*>(part4 + kQ);  // a free word of the ring
         if (threadIdx.x == 0) {
             uint32_t old;
             asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(ws_cnt + tile) : "memory");
-            *last = old == static_cast<uint32_t>(cluster - 1);
+            s_last = old == static_cast<uint32_t>(cluster - 1);
         }
         __syncthreads();
-        if (!*last) return;
+        if (!s_last) return;
         // Each thread owns at most two float4s of the tile; every load of both
         // (all C parts) goes out before the first add, so the reduction costs one
         // L2 round trip.  The adds keep rank order.
@@ -560,8 +656,26 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
             if (e < ne) {
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
-                    if (q < cluster) v[h][q] = (q == rank) ? part4[e] : __ldcg(part_g + q * kQ + e);
+                    if (q < cluster) v[h][q] = (q == rank) ? part4[e] : __ldcg(part_g + q * kQS + e);
             }
+        }
+        if (t_fused) {
+            stage_up(utile, upv, up_row, up_h, lora_r);
+            // t = scale * (the parts' shares added in rank order)
+            if (threadIdx.x < m * 16) {
+                float pv[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    if (q < cluster)
+                        pv[q] = (q == rank) ? tv
+                                            : __ldcg(reinterpret_cast<const float*>(part_g + q * kQS + kQ) + threadIdx.x);
+                float ts = pv[0];
+#pragma unroll
+                for (int q = 1; q < 8; ++q)
+                    if (q < cluster) ts += pv[q];
+                tful[threadIdx.x] = ts * lora_scale;
+            }
+            __syncthreads();
         }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -574,13 +688,18 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
                     sum = make_float4(sum.x + v[h][q].x, sum.y + v[h][q].y, sum.z + v[h][q].z, sum.w + v[h][q].w);
             float o[4] = {sum.x, sum.y, sum.z, sum.w};
             store_quad<kBf16Out, kLora>(Y, n, e / (kRows / 4), row0 + 4 * (e % (kRows / 4)), o, lora_t, lora_up,
-                                        lora_r);
+                                        lora_r, t_fused ? tful : nullptr, utile, 4 * (e % (kRows / 4)));
         }
         if (threadIdx.x == 0) ws_cnt[tile] = 0;  // ready for the next call
         return;
     }
 
     // cluster split-k: rank r adds rows [r * 128 / C, (r + 1) * 128 / C) over all ranks in rank order
+    // (a fused down-projection runs here only with C = 1: the CTA's t is the whole t)
+    if (t_fused) {
+        if (threadIdx.x < 256) tful[threadIdx.x] = tv * lora_scale;
+        stage_up(utile, upv, up_row, up_h, lora_r);
+    }
     cluster_sync();
     const int r_lo = (rank * kRows) / cluster;
     const int rows_per_rank = ((rank + 1) * kRows) / cluster - r_lo;
@@ -623,7 +742,8 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
         for (int q = 1; q < 8; ++q)
             if (q < cluster) sum = make_float4(sum.x + v[q].x, sum.y + v[q].y, sum.z + v[q].z, sum.w + v[q].w);
         float o[4] = {sum.x, sum.y, sum.z, sum.w};
-        store_quad<kBf16Out, kLora>(Y, n, tok, row0 + r, o, lora_t, lora_up, lora_r);
+        store_quad<kBf16Out, kLora>(Y, n, tok, row0 + r, o, lora_t, lora_up, lora_r, t_fused ? tful : nullptr, utile,
+                                    r);
     }
     cluster_sync();  // keep this CTA's partials alive until every rank has read them
 }
@@ -668,14 +788,21 @@ static int gemv_cluster(int64_t n, int64_t k, int sm_count) {
 
 // Workspace layout, the same for every shape so that one buffer can serve a
 // sequence of different linears and groups: kWsCounters 32-bit counters (one per
-// 128-row tile of a launch), then C fp32 partial tiles [16 tokens x 128 rows] per
-// row tile.  A split k keeps tiles x C within two CTAs per SM, so the partials
-// never take more than 2 x SMs tiles.
+// 128-row tile of a launch), then C slots per row tile, each an fp32 partial tile
+// [16 tokens x 128 rows] followed by the CTA's share of a fused LoRA
+// down-projection [16 tokens x 16 ranks].  A split k keeps tiles x C within two
+// CTAs per SM, so the slots never number more than 2 x SMs.
 constexpr int64_t kWsCounters = 1024;
 constexpr size_t kWsCounterBytes = kWsCounters * 4;
-constexpr size_t kWsPartBytes = 16 * gemv::kRows * sizeof(float);
+constexpr size_t kWsPartBytes = (16 * gemv::kRows + 16 * 16) * sizeof(float);
 
 static bool gemv_ws_usable(int64_t tiles, int cluster) { return cluster > 1 && tiles <= kWsCounters; }
+
+bool gemv_fuses_lora(int64_t m, int64_t n, int64_t k, int r, bool has_ws, const DeviceInfo& dev) {
+    if (m > kGemvMaxTokens || (r != 8 && r != 16)) return false;
+    const int cluster = gemv_cluster(n, k, dev.sm_count);
+    return cluster == 1 || (has_ws && gemv_ws_usable(gemv_tiles(n), cluster));
+}
 
 size_t linear_workspace_bytes(int64_t m, int64_t n, int64_t k, const DeviceInfo& dev) {
     if (m > kGemvMaxTokens) return 0;
@@ -725,8 +852,9 @@ static cudaError_t launch_gemv(const gemv::GemvGroup& grp, int64_t tiles, const 
     cfg.attrs = attr;
     cfg.numAttrs = na;
     return cudaLaunchKernelEx(&cfg, gemv::k_nf4_gemv<kBf16Out, kM16, kLora>, grp, tm_x, mt, k, cluster,
-                              weights_early ? 1 : 0, dev_status, ws_cnt, ws_part, lora.t, lora.up, lora.r, codebook,
-                              (test_flags & kTestStall) ? 64u : kWaitLimit, (test_flags & kTestStall) ? 1 : 0);
+                              weights_early ? 1 : 0, dev_status, ws_cnt, ws_part, lora.t, lora.up, lora.r, lora.down,
+                              lora.scale, codebook, (test_flags & kTestStall) ? 64u : kWaitLimit,
+                              (test_flags & kTestStall) ? 1 : 0);
 }
 
 // One of the eight instantiations: output type, more than 8 tokens, LoRA term.
@@ -781,7 +909,10 @@ static cudaError_t gemv_launch_group(const void* X, int64_t m, int64_t k, const 
                                   static_cast<uint64_t>(m), static_cast<uint64_t>(k * 2), 64, 16,
                                   CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
-    return dispatch_gemv(y_bf16, m > 8, lora.t != nullptr, grp, tiles, tm_x, static_cast<int>(m), k, cluster,
+    if (lora.down != nullptr && cluster > 1 && !(ws != nullptr && gemv_ws_usable(tiles, cluster)))
+        return cudaErrorInvalidValue;  // a fused down-projection needs C = 1 or the workspace split-k
+    return dispatch_gemv(y_bf16, m > 8, lora.t != nullptr || lora.down != nullptr, grp, tiles, tm_x,
+                         static_cast<int>(m), k, cluster,
                          weights_early, dev_status, ws, lora, codebook, test_flags, dev.device, stream);
 }
 

@@ -27,6 +27,10 @@ struct LoraArgs {
     int r = 0;
     const __nv_bfloat16* t_hi = nullptr;
     const __nv_bfloat16* t_lo = nullptr;
+    // Set (with t null) when the dequant-GEMV computes t = scale * X down^T
+    // itself, in its k loop (see gemv_fuses_lora).
+    const __nv_bfloat16* down = nullptr;
+    float scale = 0.f;
 };
 
 // Properties of the current device (cached per device).
@@ -73,6 +77,11 @@ struct LinearWeight {
 cudaError_t launch_linear_group(const void* X, int64_t m, int64_t k, const LinearWeight* w, int count,
                                 bool y_bf16, int32_t* dev_status, bool weights_early, void* ws, const LoraArgs& lora,
                                 int codebook, uint32_t test_flags, const DeviceInfo& dev, cudaStream_t stream);
+
+// True when the dequant-GEMV of an [n, k] weight at m tokens computes a LoRA
+// down-projection of rank r in its own k loop (r = 8 or 16, and the split of k
+// is 1 or runs through a workspace): no separate down-projection launch.
+bool gemv_fuses_lora(int64_t m, int64_t n, int64_t k, int r, bool has_ws, const DeviceInfo& dev);
 
 // True when launch_linear_group runs these weights (rows n[0 .. count-1], one
 // k) as a single dequant-GEMV launch rather than one launch per weight.
