@@ -68,8 +68,8 @@ static_assert(4 * 16 * kRedPitch * 4 + 16 * kRows * 4 <= kRingBytes, "reduction 
 // fused LoRA down-projection), in floats from the start of the ring.
 constexpr int kTredOff = 4 * 16 * kRedPitch + 16 * kRows;
 constexpr int kTOff = kTredOff + 4 * 256;
-// Then the tile's up rows, transposed: [16 ranks][128 rows] bf16.
-static_assert((kTOff + 256) * 4 + 16 * kRows * 2 <= kRingBytes, "down-projection sums fit in the ring");
+// Then the tile's up rows, transposed: [16 ranks][128 rows] fp32.
+static_assert((kTOff + 256 + 16 * kRows) * 4 <= kRingBytes, "down-projection sums fit in the ring");
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
@@ -107,17 +107,17 @@ __device__ __forceinline__ float lora_term(float v, const float* __restrict__ lt
 }
 
 // The same sums for four consecutive rows with t and up in shared memory (the
-// fused down-projection): ts [token][16], ut [rank][128 rows] bf16, rl the
-// first row's index in the tile.
-__device__ __forceinline__ void lora_quad_shared(float (&o)[4], const float* ts, const __nv_bfloat16* ut, int r,
-                                                 int tok, int rl) {
+// fused down-projection): ts [token][16], ut [rank][128 rows] (up as fp32), rl
+// the first row's index in the tile.
+__device__ __forceinline__ void lora_quad_shared(float (&o)[4], const float* ts, const float* ut, int r, int tok,
+                                                 int rl) {
     for (int j = 0; j < r; ++j) {
         const float tj = ts[tok * 16 + j];
-        const uint2 u = *reinterpret_cast<const uint2*>(ut + j * 128 + rl);
-        o[0] = __fmaf_rn(tj, bf16_bits_to_float(u.x & 0xffffu), o[0]);
-        o[1] = __fmaf_rn(tj, bf16_bits_to_float(u.x >> 16), o[1]);
-        o[2] = __fmaf_rn(tj, bf16_bits_to_float(u.y & 0xffffu), o[2]);
-        o[3] = __fmaf_rn(tj, bf16_bits_to_float(u.y >> 16), o[3]);
+        const float4 u = *reinterpret_cast<const float4*>(ut + j * 128 + rl);
+        o[0] = __fmaf_rn(tj, u.x, o[0]);
+        o[1] = __fmaf_rn(tj, u.y, o[1]);
+        o[2] = __fmaf_rn(tj, u.z, o[2]);
+        o[3] = __fmaf_rn(tj, u.w, o[3]);
     }
 }
 
@@ -186,15 +186,14 @@ __device__ __forceinline__ void load_down(uint32_t (&b)[8], const __nv_bfloat16*
 }
 
 // Thread 2 row + h holds up[row0 + row][8h .. 8h + 7] (zeros past n or r);
-// ut[j][row] = up[row0 + row][j].
-__device__ __forceinline__ void stage_up(__nv_bfloat16* ut, uint4 v, int row, int h, int r) {
+// ut[j][row] = fp32(up[row0 + row][j]).
+__device__ __forceinline__ void stage_up(float* ut, uint4 v, int row, int h, int r) {
     if (threadIdx.x >= 256 || 8 * h >= r) return;
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint16_t* u = reinterpret_cast<uint16_t*>(ut);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        u[(8 * h + 2 * q) * 128 + row] = static_cast<uint16_t>(w[q] & 0xffffu);
-        u[(8 * h + 2 * q + 1) * 128 + row] = static_cast<uint16_t>(w[q] >> 16);
+        ut[(8 * h + 2 * q) * 128 + row] = bf16_bits_to_float(w[q] & 0xffffu);
+        ut[(8 * h + 2 * q + 1) * 128 + row] = bf16_bits_to_float(w[q] >> 16);
     }
 }
 
@@ -205,7 +204,7 @@ __device__ __forceinline__ void stage_up(__nv_bfloat16* ut, uint4 v, int row, in
 template <bool kBf16Out, bool kLora>
 __device__ __forceinline__ void store_quad(void* __restrict__ Y, int64_t n, int tok, int64_t grow0, float (&o)[4],
                                            const float* __restrict__ lt, const __nv_bfloat16* __restrict__ up, int r,
-                                           const float* ts, const __nv_bfloat16* ut, int rl) {
+                                           const float* ts, const float* ut, int rl) {
     if (kLora) {
         if (ts) {
             lora_quad_shared(o, ts, ut, r, tok, rl);
@@ -613,7 +612,7 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
     // tile's t is known.
     const bool t_fused = kLora && lora_down != nullptr;
     float* tful = reinterpret_cast<float*>(ring) + kTOff;
-    __nv_bfloat16* utile = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<float*>(ring) + kTOff + 256);
+    float* utile = reinterpret_cast<float*>(ring) + kTOff + 256;
     float tv = 0.f;
     uint4 upv = make_uint4(0u, 0u, 0u, 0u);
     const int up_row = static_cast<int>(threadIdx.x) / 2, up_h = static_cast<int>(threadIdx.x) & 1;  // r = 16
@@ -660,15 +659,17 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
             }
         }
         if (t_fused) {
-            stage_up(utile, upv, up_row, up_h, lora_r);
             // t = scale * (the parts' shares added in rank order)
+            float pv[8];
             if (threadIdx.x < m * 16) {
-                float pv[8];
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
                     if (q < cluster)
                         pv[q] = (q == rank) ? tv
                                             : __ldcg(reinterpret_cast<const float*>(part_g + q * kQS + kQ) + threadIdx.x);
+            }
+            stage_up(utile, upv, up_row, up_h, lora_r);
+            if (threadIdx.x < m * 16) {
                 float ts = pv[0];
 #pragma unroll
                 for (int q = 1; q < 8; ++q)
