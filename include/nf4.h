@@ -292,8 +292,9 @@ nf4_status_t nf4_linear_dx(const void* dY, int64_t m, const nf4_weight_t* w, voi
 /*
  * nf4_linear_lora_workspace_bytes -- bytes of the workspace nf4_linear_lora
  * needs for m tokens, an [n, k] weight and rank r: the low-rank projection
- * t [m, r] in fp32 and as two bf16 halves, then the split-k area of
- * nf4_linear_ws.  0 for invalid sizes.
+ * t [m, r] in fp32 and as two bf16 halves, for m > 16 the counters and
+ * partial sums of its k-split tensor-core computation, then the split-k area
+ * of nf4_linear_ws.  0 for invalid sizes.
  */
 size_t nf4_linear_lora_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t r);
 
@@ -306,7 +307,9 @@ size_t nf4_linear_lora_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t 
  * dequant-GEMV forms it itself: tensor-core products over the same X tiles as
  * the base, each CTA's share of k added into the split-k exchange in a fixed
  * order (no separate launch).  Other m <= 16 cases compute it first in a small
- * kernel (fixed summation order).  For m <= 16 the linear then adds
+ * kernel (fixed summation order); m > 16 computes it first on the tensor cores
+ * (fp32 accumulation, k split into ranges whose partial sums are added in
+ * range order).  For m <= 16 the linear then adds
  * sum_j t[i][j] * up[o][j] (j in order, fp32) to each fp32 output before
  * rounding it to y_dtype.  For larger m with r % 8 == 0
  * the term runs on the tensor cores as extra K steps, t_hi up^T + t_lo up^T

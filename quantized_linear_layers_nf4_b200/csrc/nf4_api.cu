@@ -162,12 +162,16 @@ nf4_status_t nf4_dequantize(const nf4_weight_t* w, void* out, nf4_dtype_t out_dt
 }
 
 // LoRA workspace: t fp32 [m, r], then its bf16 halves t_hi, t_lo [m, r] (each
-// region padded to 256 bytes), then the split-k area of the decode path.
+// region padded to 256 bytes), then for m > 16 the scratch of the tensor-core
+// down-projection, then the split-k area of the decode path.
 static size_t lora_t_region(int64_t m, int32_t r, size_t elem) {
     return (static_cast<size_t>(m) * static_cast<size_t>(r) * elem + 255) / 256 * 256;
 }
-static size_t lora_t_bytes(int64_t m, int32_t r) {
-    return lora_t_region(m, r, sizeof(float)) + 2 * lora_t_region(m, r, 2);
+static size_t lora_tc_region(int64_t m, int64_t k, int32_t r) {
+    return m > nf4::kGemvMaxTokens ? (nf4::lora_tc_scratch_bytes(m, k, r) + 255) / 256 * 256 : 0;
+}
+static size_t lora_t_bytes(int64_t m, int64_t k, int32_t r) {
+    return lora_t_region(m, r, sizeof(float)) + 2 * lora_t_region(m, r, 2) + lora_tc_region(m, k, r);
 }
 
 nf4_status_t nf4_linear_lora(const void* X, int64_t m, const nf4_weight_t* w, const void* lora_down,
@@ -186,7 +190,7 @@ nf4_status_t nf4_linear_lora(const void* X, int64_t m, const nf4_weight_t* w, co
         return NF4_ERR_ALIGN;
     nf4::DeviceInfo dev;
     if ((st = device_ok(&dev)) != NF4_OK) return st;
-    const size_t tb = lora_t_bytes(m, r);
+    const size_t tb = lora_t_bytes(m, w->k, r);
     if (ws_bytes < tb + nf4::linear_workspace_bytes(m, w->n, w->k, dev)) return NF4_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     nf4::LoraArgs lora;
@@ -200,8 +204,14 @@ nf4_status_t nf4_linear_lora(const void* X, int64_t m, const nf4_weight_t* w, co
         float* t = static_cast<float*>(workspace);
         __nv_bfloat16* t_hi = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(workspace) + lora_t_region(m, r, 4));
         __nv_bfloat16* t_lo = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<char*>(t_hi) + lora_t_region(m, r, 2));
-        st = from_cuda(nf4::launch_lora_down(X, m, w->k, lora_down, r, scale, t, t_hi, t_lo,
-                                             (flags & NF4_LINEAR_WEIGHTS_EARLY) != 0, s));
+        const bool early = (flags & NF4_LINEAR_WEIGHTS_EARLY) != 0;
+        if (m > nf4::kGemvMaxTokens) {
+            void* scratch = lora_tc_region(m, w->k, r) ? reinterpret_cast<char*>(t_lo) + lora_t_region(m, r, 2) : nullptr;
+            st = from_cuda(nf4::launch_lora_down_tc(X, m, w->k, lora_down, r, scale, t, t_hi, t_lo, scratch, early,
+                                                    dev, s));
+        } else {
+            st = from_cuda(nf4::launch_lora_down(X, m, w->k, lora_down, r, scale, t, t_hi, t_lo, early, s));
+        }
         if (st != NF4_OK) return st;
         lora.t = t;
         lora.t_hi = t_hi;
@@ -234,7 +244,7 @@ size_t nf4_linear_lora_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t 
     if (m < 1 || n < 1 || k < 1 || k % NF4_BLOCKSIZE != 0 || r < 1 || r > 256) return 0;
     nf4::DeviceInfo dev;
     if (device_ok(&dev) != NF4_OK) return 0;
-    return lora_t_bytes(m, r) + nf4::linear_workspace_bytes(m, n, k, dev);
+    return lora_t_bytes(m, k, r) + nf4::linear_workspace_bytes(m, n, k, dev);
 }
 
 nf4_status_t nf4_linear_group(const void* X, int64_t m, const nf4_weight_t* const* w, int32_t count,

@@ -101,6 +101,17 @@ cudaError_t launch_linear(const void* X, int64_t m, const uint8_t* wq, const int
 cudaError_t launch_lora_down(const void* X, int64_t m, int64_t k, const void* down, int r, float scale, float* t,
                              __nv_bfloat16* t_hi, __nv_bfloat16* t_lo, bool early, cudaStream_t stream);
 
+// The same t on the tensor cores for the prefill path (m > 16): k split into up
+// to kLoraTcMaxSplit ranges whose fp32 partials are added in split order.
+// `scratch` (zero-filled before first use; the kernel leaves it zeroed) holds
+// lora_tc_scratch_bytes(m, k, r) bytes: counters, then the partials.
+constexpr int kLoraTcMaxSplit = 16;
+int lora_tc_splits(int64_t m, int64_t k, int r, int sm_count);
+size_t lora_tc_scratch_bytes(int64_t m, int64_t k, int r);
+cudaError_t launch_lora_down_tc(const void* X, int64_t m, int64_t k, const void* down, int r, float scale, float* t,
+                                __nv_bfloat16* t_hi, __nv_bfloat16* t_lo, void* scratch, bool early,
+                                const DeviceInfo& dev, cudaStream_t stream);
+
 // Merge a LoRA update into the quantized weight and requantize: w_new (bf16
 // [n, k], may be null), wq_out [n*k/2] and absmax_out [n*k/64] fp32.
 cudaError_t launch_merge_lora(const uint8_t* wq, const int8_t* absmax_q, const float* absmax_scale,

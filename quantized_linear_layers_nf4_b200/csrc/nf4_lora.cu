@@ -83,6 +83,126 @@ __global__ void __launch_bounds__(256) k_lora_down(const __nv_bfloat16* __restri
     }
 }
 
+// t for the prefill path (m > 16) on the tensor cores.  CTA (64-token block,
+// k split, group of 16 ranks); warp w takes tokens 16w .. 16w + 15 of the block.
+// Per 32 k a lane (g, i) loads 16 bytes of X rows g and g + 8 and of down rows g
+// and g + 8 of the group, at k offset 8i: the first 8 bytes feed one
+// m16n8k16 MMA and the second 8 bytes another, the MMA's k index 2i + e (e < 2)
+// standing for k offset 8i + e and 2i + 8 + e for 8i + 2 + e (the same map for
+// both operands, so the products are those of X down^T).  Rows past m or r are
+// clamped: they only reach outputs that are not stored.  With nsplit > 1 every
+// CTA stores its partial tile, and the last CTA of a (token block, rank group)
+// to count in (one acquire-release add after a block barrier) adds the nsplit
+// partials in split order and writes t = scale * sum, t_hi and t_lo.
+constexpr int kTcTokens = 64;
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void put_t(int64_t idx, float v, float* __restrict__ t, __nv_bfloat16* __restrict__ t_hi,
+                                      __nv_bfloat16* __restrict__ t_lo) {
+    t[idx] = v;
+    if (t_hi) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(v);
+        t_hi[idx] = h;
+        t_lo[idx] = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(h)));
+    }
+}
+
+__global__ void __launch_bounds__(128) k_lora_down_tc(const __nv_bfloat16* __restrict__ X, int64_t m, int64_t k,
+                                                      const __nv_bfloat16* __restrict__ down, int r, int nsplit,
+                                                      float scale, float* __restrict__ part, uint32_t* __restrict__ cnt,
+                                                      float* __restrict__ t, __nv_bfloat16* __restrict__ t_hi,
+                                                      __nv_bfloat16* __restrict__ t_lo) {
+    __shared__ int s_last;
+    grid_launch_dependents();
+    grid_dependency_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, i = lane & 3;
+    const int64_t tok0 = static_cast<int64_t>(blockIdx.x) * kTcTokens + 16 * warp;
+    const int rank0 = 16 * static_cast<int>(blockIdx.z);
+    const int split = static_cast<int>(blockIdx.y);
+    const int64_t n32 = k / 32;
+    const int64_t c0 = n32 * split / nsplit * 32, c1 = n32 * (split + 1) / nsplit * 32;
+    auto clamp_row = [](int64_t v, int64_t hi) { return v < hi ? v : hi - 1; };
+    const __nv_bfloat16* x0 = X + clamp_row(tok0 + g, m) * k + 8 * i;
+    const __nv_bfloat16* x1 = X + clamp_row(tok0 + g + 8, m) * k + 8 * i;
+    const __nv_bfloat16* d0 = down + clamp_row(rank0 + g, r) * k + 8 * i;
+    const __nv_bfloat16* d1 = down + clamp_row(rank0 + 8 + g, r) * k + 8 * i;
+    float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int64_t c = c0; c < c1; c += 32) {
+        const uint4 xa = __ldg(reinterpret_cast<const uint4*>(x0 + c));
+        const uint4 xb = __ldg(reinterpret_cast<const uint4*>(x1 + c));
+        const uint4 da = __ldg(reinterpret_cast<const uint4*>(d0 + c));
+        const uint4 db = __ldg(reinterpret_cast<const uint4*>(d1 + c));
+        mma_bf16_16816(acc0, xa.x, xb.x, xa.y, xb.y, da.x, da.y);
+        mma_bf16_16816(acc1, xa.x, xb.x, xa.y, xb.y, db.x, db.y);
+        mma_bf16_16816(acc0, xa.z, xb.z, xa.w, xb.w, da.z, da.w);
+        mma_bf16_16816(acc1, xa.z, xb.z, xa.w, xb.w, db.z, db.w);
+    }
+    // this lane's outputs: tokens tok0 + g (+ 8), ranks rank0 + 2i (+ 1) and rank0 + 8 + 2i (+ 1)
+    const float* accs[2] = {acc0, acc1};
+    if (nsplit == 1) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int64_t tok = tok0 + g + 8 * (e >> 1);
+                const int rank = rank0 + 8 * h + 2 * i + (e & 1);
+                if (tok < m && rank < r) put_t(tok * r + rank, __fmul_rn(accs[h][e], scale), t, t_hi, t_lo);
+            }
+        return;
+    }
+    // partials [nsplit][m][16 x groups]
+    const int rpad = 16 * static_cast<int>(gridDim.z);
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int e = 0; e < 4; e += 2) {
+            const int64_t tok = tok0 + g + 8 * (e >> 1);
+            if (tok < m)
+                *reinterpret_cast<float2*>(part + (static_cast<int64_t>(split) * m + tok) * rpad + rank0 + 8 * h + 2 * i) =
+                    make_float2(accs[h][e], accs[h][e + 1]);
+        }
+    __syncthreads();
+    uint32_t* c = cnt + static_cast<int64_t>(blockIdx.z) * gridDim.x + blockIdx.x;
+    if (threadIdx.x == 0) {
+        uint32_t old;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(c) : "memory");
+        s_last = old == static_cast<uint32_t>(nsplit - 1);
+    }
+    __syncthreads();
+    if (!s_last) return;
+    // four consecutive ranks of one token per step, every split's partial
+    // requested before the first add
+    for (int e = threadIdx.x; e < kTcTokens * 4; e += blockDim.x) {
+        const int64_t tok = static_cast<int64_t>(blockIdx.x) * kTcTokens + e / 4;
+        const int rq = rank0 + 4 * (e % 4);
+        if (tok >= m || rq >= r) continue;
+        float4 v[kLoraTcMaxSplit];
+#pragma unroll
+        for (int q = 0; q < kLoraTcMaxSplit; ++q)
+            if (q < nsplit) v[q] = __ldcg(reinterpret_cast<const float4*>(part + (static_cast<int64_t>(q) * m + tok) * rpad + rq));
+        float4 sum = v[0];
+#pragma unroll
+        for (int q = 1; q < kLoraTcMaxSplit; ++q)
+            if (q < nsplit)
+                sum = make_float4(__fadd_rn(sum.x, v[q].x), __fadd_rn(sum.y, v[q].y), __fadd_rn(sum.z, v[q].z),
+                                  __fadd_rn(sum.w, v[q].w));
+        const float o[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            if (rq + c < r) put_t(tok * r + rq + c, __fmul_rn(o[c], scale), t, t_hi, t_lo);
+    }
+    if (threadIdx.x == 0) *c = 0;  // ready for the next call
+}
+
 // ---------------------------------------------------------------------------
 // Merge + requantize (page "LLM 相關知識" (technicalnotes), section "8. LoRA 的
 // 合併（Merge）": the 4-bit weight is dequantized to bf16, the product of the two
@@ -196,6 +316,51 @@ cudaError_t launch_lora_down(const void* X, int64_t m, int64_t k, const void* do
     cfg.numAttrs = early ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, lora::k_lora_down, static_cast<const __nv_bfloat16*>(X), k,
                               static_cast<const __nv_bfloat16*>(down), r, scale, t, t_hi, t_lo);
+}
+
+int lora_tc_splits(int64_t m, int64_t k, int r, int sm_count) {
+    const int64_t blocks = ((m + lora::kTcTokens - 1) / lora::kTcTokens) * ((r + 15) / 16);
+    int64_t s = (8 * static_cast<int64_t>(sm_count) + blocks - 1) / blocks;
+    const int64_t cap_k = k / 32, cap_mem = (int64_t(1) << 22) / (m * 16 * ((r + 15) / 16));
+    if (s > kLoraTcMaxSplit) s = kLoraTcMaxSplit;
+    if (s > cap_k) s = cap_k;
+    if (s > cap_mem) s = cap_mem;
+    return s < 1 ? 1 : static_cast<int>(s);
+}
+
+size_t lora_tc_scratch_bytes(int64_t m, int64_t k, int r) {
+    const int64_t blocks = ((m + lora::kTcTokens - 1) / lora::kTcTokens) * ((r + 15) / 16);
+    const int64_t cap_mem = (int64_t(1) << 22) / (m * 16 * ((r + 15) / 16));
+    int64_t s = kLoraTcMaxSplit;
+    if (s > k / 32) s = k / 32;
+    if (s > cap_mem) s = cap_mem;
+    if (s <= 1) return 0;
+    return static_cast<size_t>((blocks * 4 + 255) / 256 * 256) +
+           static_cast<size_t>(s) * static_cast<size_t>(m) * 16 * static_cast<size_t>((r + 15) / 16) * sizeof(float);
+}
+
+cudaError_t launch_lora_down_tc(const void* X, int64_t m, int64_t k, const void* down, int r, float scale, float* t,
+                                __nv_bfloat16* t_hi, __nv_bfloat16* t_lo, void* scratch, bool early,
+                                const DeviceInfo& dev, cudaStream_t stream) {
+    const int64_t tb = (m + lora::kTcTokens - 1) / lora::kTcTokens;
+    const int groups = (r + 15) / 16;
+    const int nsplit = lora_tc_splits(m, k, r, dev.sm_count);
+    if (tb > 0x7fffffff) return cudaErrorInvalidValue;
+    uint32_t* cnt = static_cast<uint32_t*>(scratch);
+    float* part = scratch ? reinterpret_cast<float*>(static_cast<char*>(scratch) + (tb * groups * 4 + 255) / 256 * 256)
+                          : nullptr;
+    if (nsplit > 1 && scratch == nullptr) return cudaErrorInvalidValue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(tb), static_cast<unsigned>(nsplit), static_cast<unsigned>(groups));
+    cfg.blockDim = dim3(128, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = early ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, lora::k_lora_down_tc, static_cast<const __nv_bfloat16*>(X), m, k,
+                              static_cast<const __nv_bfloat16*>(down), r, nsplit, scale, part, cnt, t, t_hi, t_lo);
 }
 
 cudaError_t launch_merge_lora(const uint8_t* wq, const int8_t* absmax_q, const float* absmax_scale,
