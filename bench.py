@@ -666,27 +666,32 @@ def run_ours(args, rank, world, local):
     # quantize + double quant, and dequantize, over the stack
     qd = None
     if not args.skip_quant:
-        maxn = max(n * k for n, k in shapes)
-        Wb = torch.empty(maxn, dtype=torch.bfloat16, device=dev)
-        out = torch.empty(maxn, dtype=torch.bfloat16, device=dev)
-        wq = torch.empty(maxn // 2, dtype=torch.uint8, device=dev)
-        am = torch.empty(maxn // 64, dtype=torch.float32, device=dev)
-        aq = torch.empty(maxn // 64, dtype=torch.int8, device=dev)
-        sc = torch.empty(maxn // 64 // 256 + 1, dtype=torch.float32, device=dev)
-        mu = torch.empty(1, dtype=torch.float32, device=dev)
-        ws = torch.empty(maxn // 64 // 256 + 2, dtype=torch.float64, device=dev)
-        Wb.normal_(0.0, 0.02)
         sub = weights[:7]
+        # every tensor has its own input and output buffers (0.4 GB of bf16 weights
+        # in, as much out: one rep's working set is several times L2), and each leg
+        # runs as a CUDA graph of its 7 (or 14) launches, so host launch overhead is
+        # not in the timed region
+        Wbs = [torch.empty((w.n, w.k), dtype=torch.bfloat16, device=dev).normal_(0.0, 0.02) for w in sub]
+        outs = [torch.empty((w.n, w.k), dtype=torch.bfloat16, device=dev) for w in sub]
+        qbufs = [(torch.empty(w.n * w.k // 2, dtype=torch.uint8, device=dev),
+                  torch.empty(w.n * w.k // 64, dtype=torch.float32, device=dev),
+                  torch.empty(w.n * w.k // 64, dtype=torch.int8, device=dev),
+                  torch.empty(w.n * w.k // 64 // 256 + 1, dtype=torch.float32, device=dev),
+                  torch.empty(1, dtype=torch.float32, device=dev),
+                  torch.empty(w.n * w.k // 64 // 256 + 2, dtype=torch.float64, device=dev)) for w in sub]
 
         def qstep():
-            for w in sub:
-                v = Wb[: w.n * w.k].view(w.n, w.k)
+            for w, v, (wq, am, aq, sc, mu, ws) in zip(sub, Wbs, qbufs):
                 nf4.nf4_quantize(v, wq, am)
-                nf4.nf4_double_quant(am[: w.n * w.k // 64], aq, sc, mu, ws)
+                nf4.nf4_double_quant(am, aq, sc, mu, ws)
 
         def dstep():
-            for w in sub:
-                nf4.nf4_dequantize(w, torch.bfloat16, out=out[: w.n * w.k].view(w.n, w.k))
+            # the layer's 7 weights in one launch
+            nf4.nf4_dequantize_batch(sub, torch.bfloat16, outs=outs)
+
+        def dstep_each():
+            for w, o in zip(sub, outs):
+                nf4.nf4_dequantize(w, torch.bfloat16, out=o)
         # merge a rank-16 LoRA update into every tensor of the layer and requantize
         # (codes + fp32 absmax out, the merged bf16 weight not written)
         rm = 16
@@ -696,21 +701,34 @@ def run_ours(args, rank, world, local):
                       .to(torch.bfloat16)) for i, w in enumerate(sub)]
 
         def mstep():
-            for w, (dm, um) in zip(sub, lora_mats):
+            for w, (dm, um), (wq, am, _, _, _, _) in zip(sub, lora_mats, qbufs):
                 nf4.nf4_merge_lora(w, dm, um, 2.0, wq=wq, absmax=am)
-        qstep(); dstep(); mstep()
-        tq = _events_time(qstep, 5, stream)
-        td = _events_time(dstep, 5, stream)
-        tm = _events_time(mstep, 5, stream)
+        graphs = {}
+        for name, fn in (("q", qstep), ("d", dstep), ("d1", dstep_each), ("m", mstep)):
+            fn()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            for _ in range(3):
+                g.replay()
+            graphs[name] = g
+        tq = _events_time(graphs["q"].replay, 10, stream)
+        td = _events_time(graphs["d"].replay, 10, stream)
+        td1 = _events_time(graphs["d1"].replay, 10, stream)
+        tm = _events_time(graphs["m"].replay, 10, stream)
+        del graphs
         qb = sum(quant_bytes(w.n, w.k) for w in sub)
         db = sum(dequant_bytes(w.n, w.k) for w in sub)
         mb = sum(merge_bytes(w.n, w.k, rm) for w in sub)
         qd = {"quantize_dq_gbs": round(qb / tq / 1e9, 1), "dequantize_bf16_gbs": round(db / td / 1e9, 1),
+              "dequantize_bf16_gbs_one_call_per_weight": round(db / td1 / 1e9, 1),
               "merge_lora_gbs": round(mb / tm / 1e9, 1), "merge_lora_ms_per_layer": round(tm * 1e3, 3),
               "merge_lora_r": rm,
-              "sample": "one decoder layer (7 tensors, 202M params) per rep, bf16 in/out"}
-        del lora_mats
-        del Wb, out
+              "sample": "one decoder layer (7 tensors, 202M params) per rep, bf16 in/out, distinct buffers per "
+                        "tensor, each leg a CUDA graph; dequantize as one nf4_dequantize_batch launch (and as one "
+                        "call per weight)"}
+        del lora_mats, Wbs, outs, qbufs
 
     clocks = clk.summary()
     result = None

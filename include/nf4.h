@@ -218,6 +218,23 @@ nf4_status_t nf4_dequantize(const nf4_weight_t* w, void* out, nf4_dtype_t out_dt
                             nf4_stream_t stream);
 
 /*
+ * nf4_dequantize_batch -- nf4_dequantize of up to NF4_DEQUANT_BATCH_MAX weights
+ * in one launch (the weights of a layer restored together, [P4] §5), with the
+ * same bits as one call per weight.  The weights may differ in shape and
+ * codebook; every output has out_dtype.
+ *   w      host array of count weight structs (each validated as for nf4_dequantize)
+ *   count  1 .. NF4_DEQUANT_BATCH_MAX
+ *   out    host array of count device pointers, out[i] [n_i, k_i] of out_dtype,
+ *          16-byte aligned (outputs; they must not overlap each other or any input)
+ * Errors: NF4_ERR_NULL (w, out or an entry NULL), NF4_ERR_SHAPE (count out of
+ * range, or a weight's), NF4_ERR_STATE, NF4_ERR_ALIGN, NF4_ERR_DTYPE,
+ * NF4_ERR_UNSUPPORTED, NF4_ERR_CUDA.  Nothing is launched on an error.
+ */
+#define NF4_DEQUANT_BATCH_MAX 16
+nf4_status_t nf4_dequantize_batch(const nf4_weight_t* const* w, int32_t count, void* const* out,
+                                  nf4_dtype_t out_dtype, nf4_stream_t stream);
+
+/*
  * nf4_linear -- Y = X * What^T with What the bf16 dequantized weight, fused:
  * the weight is dequantized tile by tile on chip and never written out ([P5]
  * §2.2 code walk: matmul_4bit(x, weight, bias, quant_state) dequantizes and

@@ -36,7 +36,7 @@ from ._lib import NF4_BF16, NF4_F32, NF4Error, nf4_weight_t
 
 __all__ = ["NF4Weight", "NF4Error", "nf4_quantize", "nf4_double_quant", "nf4_dequantize",
            "nf4_linear", "nf4_linear_ex", "nf4_linear_group", "nf4_linear_dx", "nf4_linear_lora", "lora_workspace",
-           "nf4_merge_lora", "merge_lora",
+           "nf4_merge_lora", "merge_lora", "nf4_dequantize_batch",
            "nf4_linear_workspace_bytes", "linear_workspace",
            "quantize_weight", "nf4_codebook", "library_path"]
 
@@ -158,6 +158,25 @@ def nf4_dequantize(weight: NF4Weight, dtype=torch.bfloat16, out: torch.Tensor | 
     _lib.check(_lib.lib().nf4_dequantize(ctypes.byref(st), _ptr(out), _DTYPES[dtype],
                                          _stream(stream)), "nf4_dequantize")
     return out
+
+
+def nf4_dequantize_batch(weights, dtype=torch.bfloat16, outs=None, stream=None):
+    """[nf4_dequantize(w) for w in weights] in one launch (at most
+    NF4_DEQUANT_BATCH_MAX weights; the same bits).  Returns the list of outputs."""
+    if dtype not in _DTYPES:
+        raise ValueError("dtype must be float32 or bfloat16")
+    weights = list(weights)
+    count = len(weights)
+    if outs is None:
+        outs = [torch.empty((w.n, w.k), dtype=dtype, device=w.wq.device) for w in weights]
+    for o in outs:
+        _need_cuda(o, "out")
+    structs = [w.struct() for w in weights]
+    wptrs = (ctypes.POINTER(nf4_weight_t) * max(count, 1))(*[ctypes.pointer(s) for s in structs])
+    optrs = (ctypes.c_void_p * max(count, 1))(*[o.data_ptr() for o in outs])
+    _lib.check(_lib.lib().nf4_dequantize_batch(wptrs, count, optrs, _DTYPES[dtype], _stream(stream)),
+               "nf4_dequantize_batch")
+    return outs
 
 
 def nf4_linear_ex(X, weight, dtype=torch.bfloat16, out=None, dev_status=None, stream=None,

@@ -27,6 +27,7 @@ NF4_DQ_NOALLOC_MAX_NB = 16777216
 NF4_LINEAR_WEIGHTS_EARLY = 1
 NF4_LINEAR_TEST_TIMEOUT = 0x80000000
 NF4_LINEAR_GROUP_MAX = 4
+NF4_DEQUANT_BATCH_MAX = 16
 
 # Every function include/nf4.h declares, with (restype, argtypes).
 _p = ctypes.c_void_p
@@ -69,6 +70,8 @@ SIGNATURES = {
                                         ctypes.POINTER(_p), ctypes.c_int, _p, ctypes.c_uint32, _p, ctypes.c_size_t,
                                         _p]),
     "nf4_linear_group_launches": (ctypes.c_int32, [_i64, ctypes.POINTER(_i64), ctypes.c_int32, _i64]),
+    "nf4_dequantize_batch": (ctypes.c_int, [ctypes.POINTER(ctypes.POINTER(nf4_weight_t)), ctypes.c_int32,
+                                            ctypes.POINTER(_p), ctypes.c_int, _p]),
 }
 
 

@@ -161,6 +161,29 @@ nf4_status_t nf4_dequantize(const nf4_weight_t* w, void* out, nf4_dtype_t out_dt
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
+static_assert(NF4_DEQUANT_BATCH_MAX == nf4::kMaxDequantBatch, "batch bound of the header and the kernel agree");
+
+nf4_status_t nf4_dequantize_batch(const nf4_weight_t* const* w, int32_t count, void* const* out,
+                                  nf4_dtype_t out_dtype, nf4_stream_t stream) {
+    if (!w || !out) return NF4_ERR_NULL;
+    if (count < 1 || count > NF4_DEQUANT_BATCH_MAX) return NF4_ERR_SHAPE;
+    if (out_dtype != NF4_F32 && out_dtype != NF4_BF16) return NF4_ERR_DTYPE;
+    nf4::DequantItem items[NF4_DEQUANT_BATCH_MAX];
+    for (int32_t i = 0; i < count; ++i) {
+        if (!w[i] || !out[i]) return NF4_ERR_NULL;
+        const nf4_status_t st = check_weight(w[i]);
+        if (st != NF4_OK) return st;
+        if (!aligned(out[i], 16)) return NF4_ERR_ALIGN;
+        items[i] = {w[i]->wq, w[i]->absmax_q, w[i]->absmax_scale, w[i]->absmax_offset, w[i]->n * w[i]->k, out[i],
+                    codebook_of(w[i])};
+    }
+    nf4::DeviceInfo dev;
+    nf4_status_t st;
+    if ((st = device_ok(&dev)) != NF4_OK) return st;
+    return from_cuda(nf4::launch_dequantize_batch(items, count, out_dtype == NF4_BF16, dev,
+                                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
 // LoRA workspace: t fp32 [m, r], then its bf16 halves t_hi, t_lo [m, r] (each
 // region padded to 256 bytes), then for m > 16 the scratch of the tensor-core
 // down-projection, then the split-k area of the decode path.

@@ -51,6 +51,20 @@ cudaError_t launch_dequantize(const uint8_t* wq, const int8_t* absmax_q, const f
                               const float* absmax_offset, int64_t n_elem, void* out, bool out_bf16, int codebook,
                               const DeviceInfo& dev, cudaStream_t stream);
 
+// Several weights dequantized by one launch (same output dtype).
+constexpr int kMaxDequantBatch = 16;
+struct DequantItem {
+    const uint8_t* wq;
+    const int8_t* absmax_q;
+    const float* absmax_scale;
+    const float* absmax_offset;
+    int64_t n_elem;
+    void* out;
+    int codebook;
+};
+cudaError_t launch_dequantize_batch(const DequantItem* items, int count, bool out_bf16, const DeviceInfo& dev,
+                                    cudaStream_t stream);
+
 // Bytes of the split-k workspace the decode path needs for (m, n, k); 0 if none.
 size_t linear_workspace_bytes(int64_t m, int64_t n, int64_t k, const DeviceInfo& dev);
 

@@ -49,6 +49,7 @@ def test_header_constants_match_binding():
     assert define("NF4_WEIGHT_MAGIC") == _lib.NF4_WEIGHT_MAGIC
     assert define("NF4_WEIGHT_VERSION") == _lib.NF4_WEIGHT_VERSION
     assert define("NF4_ABI_VERSION") == _lib.NF4_ABI_VERSION
+    assert define("NF4_DEQUANT_BATCH_MAX") == _lib.NF4_DEQUANT_BATCH_MAX == 16
     assert ctypes.sizeof(_lib.nf4_weight_t) == 64
 
 
@@ -141,6 +142,28 @@ def test_weight_struct_validation(L):
     assert lex(FAKE, 4, ctypes.byref(_weight()), FAKE, 1, None, 2, None) == -4   # unknown flag bit
     assert lex(FAKE, 4, ctypes.byref(_weight(magic=3)), FAKE, 1, None, 1, None) == -5
     assert lex(FAKE, 0, ctypes.byref(_weight()), FAKE, 1, None, 1, None) == -2
+
+
+def test_dequantize_batch_validation(L):
+    """Argument checks of nf4_dequantize_batch, all before any device query."""
+    db = L.nf4_dequantize_batch
+    W = ctypes.POINTER(_lib.nf4_weight_t)
+    good = [_weight(), _weight(n=128, k=64)]
+    wp = (W * 2)(*[ctypes.pointer(x) for x in good])
+    op = (ctypes.c_void_p * 2)(FAKE.value, FAKE.value + 4096)
+    assert db(None, 2, op, 1, None) == -1
+    assert db(wp, 2, None, 1, None) == -1
+    assert db(wp, 0, op, 1, None) == -2                         # count out of range
+    assert db(wp, _lib.NF4_DEQUANT_BATCH_MAX + 1, op, 1, None) == -2
+    assert db(wp, 2, op, 7, None) == -4                         # dtype
+    bad = (W * 2)(ctypes.pointer(good[0]), ctypes.pointer(_weight(magic=1)))
+    assert db(bad, 2, op, 1, None) == -5                        # second weight's state
+    holes = (W * 2)(ctypes.pointer(good[0]), None)
+    assert db(holes, 2, op, 1, None) == -1
+    odd = (ctypes.c_void_p * 2)(FAKE.value, ODD.value)
+    assert db(wp, 2, odd, 1, None) == -3
+    nulls = (ctypes.c_void_p * 2)(FAKE.value, None)
+    assert db(wp, 2, nulls, 1, None) == -1
 
 
 def test_linear_workspace_validation(L):

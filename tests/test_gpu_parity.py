@@ -96,6 +96,34 @@ def _check_quant(nf4, W, full_dequant=True, rows=None, quant_type="nf4"):
     return weight, (owq, oq, os_, omu)
 
 
+def test_dequantize_batch(nf4):
+    """nf4_dequantize_batch over weights of different shapes and codebooks (word
+    counts that are and are not whole warp passes) gives, for each, the oracle's
+    dequantization, fp32 and bf16."""
+    shapes = [(64, 64, "nf4"), (96, 128, "fp4"), (1000, 320, "nf4"), (4096, 4096, "nf4"), (520, 640, "fp4")]
+    weights, refs = [], []
+    for i, (n, k, qt) in enumerate(shapes):
+        W = synth.weight_normal(n, k, seed=2100 + i, dtype=torch.bfloat16, device="cuda")
+        weight, orc = _check_quant(nf4, W, full_dequant=False, rows=[0], quant_type=qt)
+        weights.append(weight)
+        refs.append(orc)
+    for dtype in (torch.float32, torch.bfloat16):
+        outs = nf4.nf4_dequantize_batch(weights, dtype)
+        torch.cuda.synchronize()
+        for weight, (owq, oq, os_, omu), out in zip(weights, refs, outs):
+            ref = O.dequantize(owq, oq, os_, omu, weight.quant_type)
+            if dtype == torch.float32:
+                _assert_equal(out, ref, "batch dequant fp32 %dx%d" % (weight.n, weight.k))
+            else:
+                _assert_equal(out.view(torch.int16).view(-1), O.f32_to_bf16(ref).view(np.int16),
+                              "batch dequant bf16 %dx%d" % (weight.n, weight.k))
+    # one weight alone, and the batch bound
+    one = nf4.nf4_dequantize_batch(weights[2:3], torch.bfloat16)[0]
+    assert torch.equal(one, nf4.nf4_dequantize(weights[2], torch.bfloat16))
+    with pytest.raises(nf4.NF4Error):
+        nf4.nf4_dequantize_batch([weights[0]] * 17, torch.bfloat16)
+
+
 def _rel_fro(y: np.ndarray, ref: np.ndarray) -> float:
     return float(np.linalg.norm(y.astype(np.float64) - ref) / max(np.linalg.norm(ref), 1e-300))
 
