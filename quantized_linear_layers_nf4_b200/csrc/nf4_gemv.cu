@@ -537,12 +537,20 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
             for (int s = 0; s < 4; ++s) xf[s] = ldsm_x4(xb + x_lane + (((2 * s + (lane >> 4)) ^ (lane & 7)) << 4));
             const uint32_t wrow = stage + (rbase + g) * 128;
             const uint32_t ab = stage + kTmaBytes + ((rbase + g) * 4 + blk) * 4;
+            // each tile's codes and reconstructed absmax are read one tile ahead
+            uint4 c0 = lds128(wrow + wc0), c1 = lds128(wrow + wc1);
+            float av = lds_f32(ab);
 #pragma unroll
             for (int t = 0; t < kTiles; ++t) {
-                const uint4 w0 = lds128(wrow + t * 8 * 128 + wc0);
-                const uint4 w1 = lds128(wrow + t * 8 * 128 + wc1);
-                const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-                const uint64_t aa = dup_f32x2(lds_f32(ab + 128 * t));
+                uint4 n0 = c0, n1 = c1;
+                float an = av;
+                if (t + 1 < kTiles) {
+                    n0 = lds128(wrow + (t + 1) * 8 * 128 + wc0);
+                    n1 = lds128(wrow + (t + 1) * 8 * 128 + wc1);
+                    an = lds_f32(ab + 128 * (t + 1));
+                }
+                const uint32_t wv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                const uint64_t aa = dup_f32x2(av);
                 uint32_t bw[8];
 #pragma unroll
                 for (int b = 0; b < 8; ++b) {
@@ -553,6 +561,9 @@ k_nf4_gemv(const __grid_constant__ GemvGroup grp, const __grid_constant__ CUtens
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
                     mma_16816(acc[t], xf[s].x, xf[s].y, xf[s].z, xf[s].w, bw[2 * s], bw[2 * s + 1]);
+                c0 = n0;
+                c1 = n1;
+                av = an;
             }
             if (kLora && t_on) {
 #pragma unroll
