@@ -69,18 +69,35 @@ __device__ __forceinline__ float quotient(float w, float a, float r) {
     return __fmaf_rn(e, r, q0);
 }
 
+// Packed fp32 pairs: each half is rounded exactly as the scalar operation.
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 __device__ __forceinline__ bool markstein_ok(float a) {
     return a >= 0x1p-60f && a <= 0x1p60f;  // false for 0, NaN and +inf too
 }
 
 template <typename T, int CB>
-__global__ void __launch_bounds__(256) k_nf4_quantize(const T* __restrict__ W, int64_t n_groups,
+__global__ void __launch_bounds__(256, 4) k_nf4_quantize(const T* __restrict__ W, int64_t n_groups,
                                                       uint32_t* __restrict__ wq32,
                                                       float* __restrict__ absmax) {
     __shared__ uint2 tab[CB == kCbNf4 ? kBuckets * kTabCopies : 1];
     if (CB == kCbNf4) {
-        for (int e = threadIdx.x; e < kBuckets * kTabCopies; e += blockDim.x) {
-            const int b = e / kTabCopies;
+        // each bucket's entry is formed once (into its first copy), then copied
+        for (int b = threadIdx.x; b < kBuckets; b += blockDim.x) {
             const float lo = (static_cast<float>(b) - 0.5f) / 128.0f - 1.0f;
             const float hi = (static_cast<float>(b) + 0.5f) / 128.0f - 1.0f;
             uint32_t base = 0;
@@ -91,8 +108,11 @@ __global__ void __launch_bounds__(256) k_nf4_quantize(const T* __restrict__ W, i
                 if (t < lo) ++base;
                 else if (t <= hi) thr = t;
             }
-            tab[e] = make_uint2(__float_as_uint(thr), base);
+            tab[b * kTabCopies] = make_uint2(__float_as_uint(thr), base);
         }
+        __syncthreads();
+        for (int e = threadIdx.x; e < kBuckets * kTabCopies; e += blockDim.x)
+            if (e % kTabCopies != 0) tab[e] = tab[e - e % kTabCopies];
         __syncthreads();
     }
     const int lane = threadIdx.x & 31;
@@ -125,7 +145,29 @@ __global__ void __launch_bounds__(256) k_nf4_quantize(const T* __restrict__ W, i
             a = fmaxf(a, __shfl_xor_sync(kFull, a, 2));
             a = fmaxf(a, __shfl_xor_sync(kFull, a, 4));
             uint32_t code[8];
-            if (markstein_ok(a)) {
+            if (CB == kCbNf4 && markstein_ok(a)) {
+                // the same quotient and bucket, two elements per packed instruction
+                const float r = __frcp_rn(a);
+                const uint64_t rr = f2(r, r), na = f2(-a, -a), k128 = f2(128.0f, 128.0f);
+                const uint64_t mg = f2(kBucketMagic, kBucketMagic);
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const uint64_t w2 = f2(w[u][2 * p], w[u][2 * p + 1]);
+                    const uint64_t q0 = mul2(w2, rr);
+                    const uint64_t e = fma2(q0, na, w2);
+                    const uint64_t q2 = fma2(e, rr, q0);
+                    const uint64_t b2 = fma2(q2, k128, mg);
+                    float qv[2];
+                    uint32_t bv[2];
+                    asm("mov.b64 {%0, %1}, %2;" : "=f"(qv[0]), "=f"(qv[1]) : "l"(q2));
+                    asm("mov.b64 {%0, %1}, %2;" : "=r"(bv[0]), "=r"(bv[1]) : "l"(b2));
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint2 ent = tab[(bv[h] & 0x1ffu) * kTabCopies + (threadIdx.x & 15)];
+                        code[2 * p + h] = ent.y + (qv[h] > __uint_as_float(ent.x) ? 1u : 0u);
+                    }
+                }
+            } else if (markstein_ok(a)) {
                 const float r = __frcp_rn(a);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
