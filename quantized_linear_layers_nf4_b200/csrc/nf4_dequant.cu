@@ -16,6 +16,7 @@
 
 #include "nf4_common.cuh"
 #include "nf4_internal.h"
+#include "nf4_ptx.cuh"
 
 namespace nf4 {
 
@@ -76,6 +77,8 @@ __global__ void __launch_bounds__(256) k_nf4_dequantize(const uint32_t* __restri
                                                         int codebook) {
     const int lane = threadIdx.x & 31;
     const float lvr = kCodebook[codebook][lane & 15];
+    grid_dependency_wait();  // launched as a programmatic dependent: inputs may come from the preceding kernel
+    grid_launch_dependents();
     const float mu = __ldg(mu_ptr);
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -100,6 +103,8 @@ struct DequantBatch {
 template <bool kBf16Out>
 __global__ void __launch_bounds__(256) k_nf4_dequantize_batch(const __grid_constant__ DequantBatch bt) {
     const int lane = threadIdx.x & 31;
+    grid_dependency_wait();
+    grid_launch_dependents();
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     for (int64_t p = warp; p < bt.pass0[bt.count]; p += n_warps) {
@@ -122,12 +127,10 @@ cudaError_t launch_dequantize(const uint8_t* wq, const int8_t* absmax_q, const f
     if (blocks < 1) blocks = 1;
     const uint32_t* wq32 = reinterpret_cast<const uint32_t*>(wq);
     if (out_bf16)
-        k_nf4_dequantize<true><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-            wq32, absmax_q, absmax_scale, absmax_offset, n_groups, out, codebook);
-    else
-        k_nf4_dequantize<false><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-            wq32, absmax_q, absmax_scale, absmax_offset, n_groups, out, codebook);
-    return cudaGetLastError();
+        return launch_pdl(k_nf4_dequantize<true>, dim3(static_cast<unsigned>(blocks)), dim3(256), stream, wq32,
+                          absmax_q, absmax_scale, absmax_offset, n_groups, out, codebook);
+    return launch_pdl(k_nf4_dequantize<false>, dim3(static_cast<unsigned>(blocks)), dim3(256), stream, wq32, absmax_q,
+                      absmax_scale, absmax_offset, n_groups, out, codebook);
 }
 
 cudaError_t launch_dequantize_batch(const DequantItem* items, int count, bool out_bf16, const DeviceInfo& dev,
@@ -155,10 +158,8 @@ cudaError_t launch_dequantize_batch(const DequantItem* items, int count, bool ou
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     if (out_bf16)
-        k_nf4_dequantize_batch<true><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(bt);
-    else
-        k_nf4_dequantize_batch<false><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(bt);
-    return cudaGetLastError();
+        return launch_pdl(k_nf4_dequantize_batch<true>, dim3(static_cast<unsigned>(blocks)), dim3(256), stream, bt);
+    return launch_pdl(k_nf4_dequantize_batch<false>, dim3(static_cast<unsigned>(blocks)), dim3(256), stream, bt);
 }
 
 }  // namespace nf4

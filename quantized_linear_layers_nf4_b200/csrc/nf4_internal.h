@@ -7,6 +7,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace nf4 {
 
 struct DeviceInfo {
@@ -32,6 +34,23 @@ struct LoraArgs {
     const __nv_bfloat16* down = nullptr;
     float scale = 0.f;
 };
+
+// A launch as a programmatic dependent of the preceding kernel on the stream:
+// it may start while that kernel drains, and waits for it (griddepcontrol.wait)
+// before it touches memory.  Used for kernels that begin with that wait.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Properties of the current device (cached per device).
 cudaError_t current_device(DeviceInfo* out);

@@ -16,6 +16,7 @@
 // finish the mean's fixed-order reduction from the partial sums first.
 #include "nf4_common.cuh"
 #include "nf4_internal.h"
+#include "nf4_ptx.cuh"
 
 namespace nf4 {
 
@@ -115,6 +116,9 @@ __global__ void __launch_bounds__(256, 4) k_nf4_quantize(const T* __restrict__ W
             if (e % kTabCopies != 0) tab[e] = tab[e - e % kTabCopies];
         __syncthreads();
     }
+    // the table above uses constants only; W and the outputs wait for the
+    // preceding kernel (launched as its programmatic dependent)
+    grid_dependency_wait();
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -193,17 +197,17 @@ __global__ void __launch_bounds__(256, 4) k_nf4_quantize(const T* __restrict__ W
             }
         }
     }
+    grid_launch_dependents();
 }
 
 template <int CB>
-static void launch_quantize_cb(const void* W, bool w_bf16, int64_t n_groups, uint8_t* wq, float* absmax,
+static cudaError_t launch_quantize_cb(const void* W, bool w_bf16, int64_t n_groups, uint8_t* wq, float* absmax,
                                int64_t blocks, cudaStream_t stream) {
     if (w_bf16)
-        k_nf4_quantize<__nv_bfloat16, CB><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(W), n_groups, reinterpret_cast<uint32_t*>(wq), absmax);
-    else
-        k_nf4_quantize<float, CB><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-            static_cast<const float*>(W), n_groups, reinterpret_cast<uint32_t*>(wq), absmax);
+        return launch_pdl(k_nf4_quantize<__nv_bfloat16, CB>, dim3(static_cast<unsigned>(blocks)), dim3(256), stream,
+                          static_cast<const __nv_bfloat16*>(W), n_groups, reinterpret_cast<uint32_t*>(wq), absmax);
+    return launch_pdl(k_nf4_quantize<float, CB>, dim3(static_cast<unsigned>(blocks)), dim3(256), stream,
+                      static_cast<const float*>(W), n_groups, reinterpret_cast<uint32_t*>(wq), absmax);
 }
 
 cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n_elem, uint8_t* wq, float* absmax, int codebook,
@@ -216,11 +220,8 @@ cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n_elem, uint8_t*
     const int64_t cap = static_cast<int64_t>(dev.sm_count) * 4;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    if (codebook == kCbFp4)
-        launch_quantize_cb<kCbFp4>(W, w_bf16, n_groups, wq, absmax, blocks, stream);
-    else
-        launch_quantize_cb<kCbNf4>(W, w_bf16, n_groups, wq, absmax, blocks, stream);
-    return cudaGetLastError();
+    if (codebook == kCbFp4) return launch_quantize_cb<kCbFp4>(W, w_bf16, n_groups, wq, absmax, blocks, stream);
+    return launch_quantize_cb<kCbNf4>(W, w_bf16, n_groups, wq, absmax, blocks, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -251,6 +252,8 @@ __device__ __forceinline__ double warp_tree256(double (&v)[8]) {
 // Level 1: one fp64 partial per double-quantization block of 256 absmax.
 __global__ void __launch_bounds__(256) k_dq_partials(const float* __restrict__ absmax, int64_t nb,
                                                      double* __restrict__ partials, int64_t nb2) {
+    grid_dependency_wait();  // absmax comes from the preceding kernel
+    grid_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -319,6 +322,8 @@ __global__ void __launch_bounds__(kEncodeThreads) k_dq_encode(const float* __res
                                                               float* __restrict__ absmax_scale) {
     __shared__ double buf_a[kMeanLevel2];
     __shared__ double buf_b[kMeanLevel2 / 256 + 1];
+    grid_dependency_wait();  // the partial sums come from the preceding kernel
+    grid_launch_dependents();
     const float mu = cta_mean(partials, nb2, nb, buf_a, buf_b);
     if (blockIdx.x == 0 && threadIdx.x == 0) *mu_out = mu;
     const int lane = threadIdx.x & 31;
@@ -356,11 +361,12 @@ cudaError_t launch_double_quant(const float* absmax, int64_t nb, double* workspa
     const int64_t cap = static_cast<int64_t>(dev.sm_count) * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    k_dq_partials<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(absmax, nb, workspace, nb2);
-    k_dq_encode<<<static_cast<unsigned>(blocks), kEncodeThreads, 0, stream>>>(absmax, nb, nb2, workspace,
-                                                                               absmax_offset, absmax_q,
-                                                                               absmax_scale);
-    return cudaGetLastError();
+    // both as programmatic dependents: each launch overlaps the tail of the one before
+    cudaError_t e = launch_pdl(k_dq_partials, dim3(static_cast<unsigned>(blocks)), dim3(256), stream, absmax, nb,
+                               workspace, nb2);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(k_dq_encode, dim3(static_cast<unsigned>(blocks)), dim3(kEncodeThreads), stream, absmax, nb, nb2,
+                      static_cast<const double*>(workspace), absmax_offset, absmax_q, absmax_scale);
 }
 
 }  // namespace nf4
