@@ -387,14 +387,16 @@ def test_linear_dx_errors(nf4):
                                            (16, 11008, 4096, 8, 2.0), (5, 19200, 320, 16, 1.5),
                                            (9, 1000, 320, 16, 0.5), (1, 4096, 11008, 16, 2.0),
                                            (300, 520, 640, 16, 2.0), (1024, 1024, 1024, 64, 0.25),
-                                           (257, 136, 320, 5, 2.0), (512, 256, 512, 72, 1.0)])
+                                           (257, 136, 320, 5, 2.0), (512, 256, 512, 72, 1.0),
+                                           (18944, 64, 64, 64, 1.0)])
 def test_linear_lora(nf4, m, n, k, r, scale):
     """The QLoRA layer Y = X What^T + s (X down^T) up^T: decode path (k split 8, 3
     and 1; r = 8 and 16 with the down-projection formed inside the GEMV, over a
     ragged last k stage too, other ranks by a separate kernel) and prefill path
     (tensor-core term for r % 8 == 0 in one or two K tiles of 64 ranks, fp32
-    epilogue otherwise), against the oracle; the bf16 output is the rounded fp32
-    output."""
+    epilogue otherwise; the tensor-core down-projection with k split and, at
+    18944 tokens x 4 rank groups, unsplit), against the oracle; the bf16 output is
+    the rounded fp32 output."""
     W = synth.weight_normal(n, k, seed=1800 + n + r, dtype=torch.bfloat16, device="cuda")
     X = synth.activations(m, k, seed=1810 + m, device="cuda")
     down = (synth.activations(r, k, seed=1820 + r, device="cuda").float() * 0.02).to(torch.bfloat16)
