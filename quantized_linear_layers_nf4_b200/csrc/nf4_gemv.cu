@@ -29,9 +29,16 @@
 //   encodes (replicated 16x so a half-warp's lookups never share a bank); each
 //   level is multiplied by the block's reconstructed absmax in fp32 and rounded
 //   to bf16 -- the same values nf4_dequantize produces.
-// * Split-k: the CTAs of a thread-block cluster share a row tile and split k;
-//   their fp32 partials are added through distributed shared memory in a fixed
-//   rank order, so results are deterministic and no global scratch is needed.
+// * Split-k: the C CTAs of a row tile split k.  Without a workspace they form a
+//   thread-block cluster and add their fp32 partials through distributed shared
+//   memory; with a caller's workspace they store them there and the last to
+//   count in adds them.  Both add in rank order, so the bits are the same and
+//   deterministic.
+// * One launch may cover the row tiles of several weights that share X (a
+//   grid-constant group struct; each CTA picks its weight by its tile).
+// * LoRA layers (r = 8 or 16): the CTAs also form their share of
+//   t = scale * X down^T from the same X fragments and exchange it with the
+//   partial sums; the epilogue adds t up^T before rounding.
 #include <cstring>
 #include <mutex>
 

@@ -5,11 +5,10 @@
 // frozen W acts as W + dW with dW = A x B of low rank r, trained in bf16; with W
 // stored [n, k] that is dW = up [n, r] * down [r, k], so
 //   Y = X What^T + scale * (X down^T) up^T.
-// This kernel computes t = scale * X down^T [m, r] in fp32; the linear kernels add
-// t up^T in their epilogue.  One block per (token, 8 ranks), one warp per rank;
-// each lane sums a fixed subset of k into four partial sums combined in a fixed
-// order, and the warp adds the lanes in a fixed tree, so the result never
-// depends on scheduling.
+// The kernels here compute t = scale * X down^T [m, r] in fp32 ahead of the
+// linear, which adds t up^T: k_lora_down for decode-sized m (used when the GEMV
+// does not form t itself), k_lora_down_tc on the tensor cores for m > 16.  Both
+// add in a fixed order, so the result never depends on scheduling.
 #include <cuda_bf16.h>
 
 #include "nf4_common.cuh"
