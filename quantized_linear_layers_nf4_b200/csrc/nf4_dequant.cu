@@ -48,9 +48,12 @@ __device__ __forceinline__ void dequant_pass(const uint32_t* __restrict__ wq32, 
         float v[8];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const uint32_t byte = (packed[q] >> (8 * i)) & 0xffu;
-            v[2 * i] = __fmul_rn(__shfl_sync(kFull, lvr, static_cast<int>(byte >> 4)), a[q]);  // element 2i: high nibble
-            v[2 * i + 1] = __fmul_rn(__shfl_sync(kFull, lvr, static_cast<int>(byte & 15u)), a[q]);
+            // a shuffle takes the low 5 bits of its source lane, and lanes l and
+            // l + 16 hold the same level, so the shifted word needs no mask
+            const int hi = static_cast<int>(packed[q] >> (8 * i + 4));  // element 2i: high nibble
+            const int lo = static_cast<int>(packed[q] >> (8 * i));
+            v[2 * i] = __fmul_rn(__shfl_sync(kFull, lvr, hi), a[q]);
+            v[2 * i + 1] = __fmul_rn(__shfl_sync(kFull, lvr, lo), a[q]);
         }
         if (g >= n_groups) continue;
         if (kBf16Out) {
