@@ -149,8 +149,9 @@ __global__ void __launch_bounds__(256, 4) k_nf4_quantize(const T* __restrict__ W
             a = fmaxf(a, __shfl_xor_sync(kFull, a, 2));
             a = fmaxf(a, __shfl_xor_sync(kFull, a, 4));
             uint32_t code[8];
-            if (CB == kCbNf4 && markstein_ok(a)) {
+            if (CB == kCbNf4 && __all_sync(kFull, markstein_ok(a))) {
                 // the same quotient and bucket, two elements per packed instruction
+                // (taken by whole warps; a warp with any other block uses the paths below)
                 const float r = __frcp_rn(a);
                 const uint64_t rr = f2(r, r), na = f2(-a, -a), k128 = f2(128.0f, 128.0f);
                 const uint64_t mg = f2(kBucketMagic, kBucketMagic);
