@@ -166,6 +166,19 @@ def test_dequantize_batch_validation(L):
     assert db(wp, 2, nulls, 1, None) == -1
 
 
+def test_group_launch_plan_validation(L):
+    """nf4_linear_group_launches rejects invalid sizes before any device query."""
+    gl = L.nf4_linear_group_launches
+    ns = (ctypes.c_int64 * 5)(4096, 4096, 4096, 4096, 4096)
+    assert gl(16, None, 3, 4096) == -1
+    assert gl(16, ns, 0, 4096) == -1
+    assert gl(16, ns, 5, 4096) == -1          # more than NF4_LINEAR_GROUP_MAX
+    assert gl(0, ns, 3, 4096) == -1
+    assert gl(16, ns, 3, 100) == -1           # k % 64 != 0
+    zero = (ctypes.c_int64 * 2)(4096, 0)
+    assert gl(16, zero, 2, 4096) == -1
+
+
 def test_linear_workspace_validation(L):
     lws = L.nf4_linear_ws
     w = ctypes.byref(_weight())

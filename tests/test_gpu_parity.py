@@ -628,6 +628,13 @@ def test_linear_group_matches_single_launches(nf4, m):
             s1 = nf4.nf4_linear(Xg, w, torch.float32)
             assert float((a - s1).norm() / s1.norm()) <= FP32_ORDER_TOL
         assert int(ws2[:4 * 1024].view(torch.int32).abs().sum()) == 0, "split-k counters not reset"
+    # the launch plan on this device: q/k/v of a 4096-wide layer as one launch, gate/up
+    # (each already a full wave) as one launch per weight, the GEMM path one per weight
+    assert nf4.nf4_linear_group_launches(m, [4096, 4096, 4096], 4096) == 1
+    assert nf4.nf4_linear_group_launches(m, [11008, 11008], 4096) == 2
+    assert nf4.nf4_linear_group_launches(64, [4096, 4096, 4096], 4096) == 3
+    with pytest.raises(ValueError):
+        nf4.nf4_linear_group_launches(m, [4096] * 5, 4096)
     with pytest.raises(nf4.NF4Error):  # different k
         nf4.nf4_linear_group(X, [weights[0], nf4.quantize_weight(Ws[0][:, :1024].contiguous())])
     with pytest.raises(nf4.NF4Error):  # too many weights
