@@ -42,6 +42,9 @@ __device__ __forceinline__ void dequant_pass(const uint32_t* __restrict__ wq32, 
         const int64_t b = gg >> 3;                       // 64-element block
         a[q] = absmax_hat(__ldg(absmax_q + b), __ldg(absmax_scale + (b >> 8)), mu);
     }
+    uint64_t aa[kUnroll];  // {a, a}: the two levels of a byte scaled by one packed multiply
+#pragma unroll
+    for (int q = 0; q < kUnroll; ++q) asm("mov.b64 %0, {%1, %1};" : "=l"(aa[q]) : "f"(a[q]));
 #pragma unroll
     for (int q = 0; q < kUnroll; ++q) {
         const int64_t g = base + 32 * q + lane;
@@ -52,8 +55,12 @@ __device__ __forceinline__ void dequant_pass(const uint32_t* __restrict__ wq32, 
             // l + 16 hold the same level, so the shifted word needs no mask
             const int hi = static_cast<int>(packed[q] >> (8 * i + 4));  // element 2i: high nibble
             const int lo = static_cast<int>(packed[q] >> (8 * i));
-            v[2 * i] = __fmul_rn(__shfl_sync(kFull, lvr, hi), a[q]);
-            v[2 * i + 1] = __fmul_rn(__shfl_sync(kFull, lvr, lo), a[q]);
+            const float lh = __shfl_sync(kFull, lvr, hi), ll = __shfl_sync(kFull, lvr, lo);
+            uint64_t p2;  // each half rounded as the scalar fp32 multiply
+            asm("{\n\t.reg .b64 l;\n\tmov.b64 l, {%1, %2};\n\tmul.rn.f32x2 %0, l, %3;\n\t}"
+                : "=l"(p2)
+                : "f"(lh), "f"(ll), "l"(aa[q]));
+            asm("mov.b64 {%0, %1}, %2;" : "=f"(v[2 * i]), "=f"(v[2 * i + 1]) : "l"(p2));
         }
         if (g >= n_groups) continue;
         if (kBf16Out) {
