@@ -117,9 +117,13 @@ def test_dequantize_batch(nf4):
             else:
                 _assert_equal(out.view(torch.int16).view(-1), O.f32_to_bf16(ref).view(np.int16),
                               "batch dequant bf16 %dx%d" % (weight.n, weight.k))
-    # one weight alone, and the batch bound
+    # one weight alone, sixteen (the bound) of mixed sizes, and one more than the bound
     one = nf4.nf4_dequantize_batch(weights[2:3], torch.bfloat16)[0]
     assert torch.equal(one, nf4.nf4_dequantize(weights[2], torch.bfloat16))
+    many = [weights[i % len(weights)] for i in range(16)]
+    outs16 = nf4.nf4_dequantize_batch(many, torch.float32)
+    for weight, out in zip(many, outs16):
+        assert torch.equal(out, nf4.nf4_dequantize(weight, torch.float32))
     with pytest.raises(nf4.NF4Error):
         nf4.nf4_dequantize_batch([weights[0]] * 17, torch.bfloat16)
 
