@@ -325,18 +325,27 @@ __global__ void __launch_bounds__(kEncodeThreads) k_dq_encode(const float* __res
     __shared__ double buf_b[kMeanLevel2 / 256 + 1];
     grid_dependency_wait();  // the partial sums come from the preceding kernel
     grid_launch_dependents();
-    const float mu = cta_mean(partials, nb2, nb, buf_a, buf_b);
-    if (blockIdx.x == 0 && threadIdx.x == 0) *mu_out = mu;
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    // the warp's first block of absmax values is requested before the mean is
+    // formed, so the two loads overlap
+    float pre[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int64_t b = warp * 256 + lane + 32 * j;
+        pre[j] = (warp < nb2 && b < nb) ? __ldg(absmax + b) : 0.0f;
+    }
+    const float mu = cta_mean(partials, nb2, nb, buf_a, buf_b);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *mu_out = mu;
     for (int64_t c = warp; c < nb2; c += n_warps) {
         float r[8];
         float s = 0.0f;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int64_t b = c * 256 + lane + 32 * j;
-            r[j] = (b < nb) ? __fsub_rn(__ldg(absmax + b), mu) : 0.0f;
+            const float v = (c == warp) ? pre[j] : ((b < nb) ? __ldg(absmax + b) : 0.0f);
+            r[j] = (b < nb) ? __fsub_rn(v, mu) : 0.0f;
             s = fmaxf(s, fabsf(r[j]));
         }
 #pragma unroll
