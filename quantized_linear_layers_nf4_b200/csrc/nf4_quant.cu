@@ -15,6 +15,7 @@
 // launches: per-256 fp64 partial sums, then the int8 encode, whose CTAs each
 // finish the mean's fixed-order reduction from the partial sums first.
 #include "nf4_common.cuh"
+#include "nf4_encode.cuh"
 #include "nf4_internal.h"
 #include "nf4_ptx.cuh"
 
@@ -42,80 +43,12 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* __restrict__ W, int64
     }
 }
 
-// The code of each element without a division and without a search.
-//
-// Quotient: q = RN(w / a) by Markstein's correction of a product with the
-// correctly rounded reciprocal (P. Markstein, "Computation of elementary
-// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
-// 1990): with r = RN(1 / a), q0 = RN(w r), e = w - a q0 (exact, one FMA) and
-// q = RN(q0 + e r) is the IEEE quotient when nothing leaves the normal range.
-// It is used for blocks whose absmax lies in [2^-60, 2^60]; for them every
-// quotient that can reach a threshold (|q| >= 2^-8, far inside the band that
-// maps to the zero level) keeps e exact.  Other blocks (zero, tiny, huge or
-// non-finite absmax) divide.
-//
-// NF4 code of q in [-1, 1]: bucket b = round_half_even(128 q + 128) (one FMA
-// onto the mantissa of 1.5 * 2^23) of a 257-entry table; at most one threshold
-// falls in the closed q range of a bucket (NF4 thresholds are more than 1/128
-// apart), so idx = base[b] + (q > thr[b]) with base[b] = #{j : t_j below the
-// bucket}.  The table lives in shared memory, 16 copies so the 16 lanes of a
-// half-warp never share a bank.
-constexpr int kBuckets = 257;
-constexpr int kTabCopies = 16;
-constexpr float kBucketMagic = 12582912.0f + 128.0f;  // 1.5 * 2^23 + 128
-
-__device__ __forceinline__ float quotient(float w, float a, float r) {
-    const float q0 = __fmul_rn(w, r);
-    const float e = __fmaf_rn(-q0, a, w);
-    return __fmaf_rn(e, r, q0);
-}
-
-// Packed fp32 pairs: each half is rounded exactly as the scalar operation.
-__device__ __forceinline__ uint64_t f2(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-
-__device__ __forceinline__ bool markstein_ok(float a) {
-    return a >= 0x1p-60f && a <= 0x1p60f;  // false for 0, NaN and +inf too
-}
-
 template <typename T, int CB>
 __global__ void __launch_bounds__(256, 4) k_nf4_quantize(const T* __restrict__ W, int64_t n_groups,
                                                       uint32_t* __restrict__ wq32,
                                                       float* __restrict__ absmax) {
     __shared__ uint2 tab[CB == kCbNf4 ? kBuckets * kTabCopies : 1];
-    if (CB == kCbNf4) {
-        // each bucket's entry is formed once (into its first copy), then copied
-        for (int b = threadIdx.x; b < kBuckets; b += blockDim.x) {
-            const float lo = (static_cast<float>(b) - 0.5f) / 128.0f - 1.0f;
-            const float hi = (static_cast<float>(b) + 0.5f) / 128.0f - 1.0f;
-            uint32_t base = 0;
-            float thr = __int_as_float(0x7f800000);  // +inf: no threshold in the bucket
-#pragma unroll
-            for (int j = 0; j < 15; ++j) {
-                const float t = kThresh[j];
-                if (t < lo) ++base;
-                else if (t <= hi) thr = t;
-            }
-            tab[b * kTabCopies] = make_uint2(__float_as_uint(thr), base);
-        }
-        __syncthreads();
-        for (int e = threadIdx.x; e < kBuckets * kTabCopies; e += blockDim.x)
-            if (e % kTabCopies != 0) tab[e] = tab[e - e % kTabCopies];
-        __syncthreads();
-    }
+    if (CB == kCbNf4) build_bucket_table(tab);
     // the table above uses constants only; W and the outputs wait for the
     // preceding kernel (launched as its programmatic dependent)
     grid_dependency_wait();
@@ -177,13 +110,8 @@ __global__ void __launch_bounds__(256, 4) k_nf4_quantize(const T* __restrict__ W
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const float q = quotient(w[u][j], a, r);
-                    if (CB == kCbNf4) {
-                        const uint32_t b = __float_as_uint(__fmaf_rn(q, 128.0f, kBucketMagic)) & 0x1ffu;
-                        const uint2 ent = tab[b * kTabCopies + (threadIdx.x & 15)];
-                        code[j] = ent.y + (q > __uint_as_float(ent.x) ? 1u : 0u);
-                    } else {
-                        code[j] = static_cast<uint32_t>(encode_fp4(q));
-                    }
+                    code[j] = CB == kCbNf4 ? bucket_code(q, tab, threadIdx.x & 15)
+                                           : static_cast<uint32_t>(encode_fp4(q));
                 }
             } else {
 #pragma unroll
